@@ -1,0 +1,276 @@
+"""Benchmark of the routed-expert stack on B200.
+
+Default workload: the 35B-shaped MoE stack (40 layers x 256 routed experts,
+top-4, hidden 2048, int4 group-64 experts, 8-bit router and shared gate,
+shared expert with LoRA r=16, one Prerouter head per layer) decoding one token
+per step (batch 1).  A step is one token through all 40 layers.  Every rank is
+an independent replica (batch-1 decode does not shard; weak scaling).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gen import CONFIGS, inputs  # noqa: E402
+
+METRIC = "MoE-stack decode tok/s (35B-shape, bs=1) & HBM GB/s vs peak; prefill tok/s"
+CFG_ID = 1
+EPS = 1e-6
+N_TOKENS = 64  # distinct tokens cycled through the steps
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def token_layer_bytes(cfg) -> int:
+    """Algorithmic HBM bytes one token reads in one layer (batch-1 decode)."""
+    blk = cfg.expert_block_bytes
+    shared = 2 * cfg.I_s * (cfg.H // 2 + 4 * (cfg.H // 64)) + cfg.H * (cfg.I_s // 2 + 4 * (cfg.I_s // 64))
+    lora = 2 * (cfg.r * cfg.H * 2 + cfg.I_s * cfg.r * 2) + cfg.r * cfg.I_s * 2 + cfg.H * cfg.r * 2
+    router = cfg.E * (cfg.H + 4 * (cfg.H // 64))
+    sgate = cfg.H + 4 * (cfg.H // 64)
+    pre = cfg.P * cfg.H * 2 + cfg.P * cfg.K * 2 + cfg.P * 2 + cfg.E_next * cfg.P * 2 + cfg.E_next * 2
+    return cfg.K * blk + shared + lora + router + sgate + pre
+
+
+def launches_per_step(cfg, predicted=False) -> int:
+    per_layer = 1 + 2 + 1 + 1 + 1 + 1 + 3  # rmsnorm, router+topk, pre, gate/up, lora-mid, down, prerouter x3
+    return cfg.layers * per_layer + (cfg.layers - 1 if predicted else 0)
+
+
+class Clocks:
+    """nvidia-smi samples (SM clock, throttle reasons) during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_baseline(cfg, budget_s: float = 20.0):
+    """The float64 oracle on the host: tokens through the stack, layer by layer, bounded by a time budget."""
+    from oracle import moe_oracle as O
+    cores = len(os.sched_getaffinity(0))
+    x = inputs.bf16_bits_to_f32(inputs.activations(cfg, step=0, T=1)).astype(np.float64)
+    t_oracle, layers_done = 0.0, 0
+    for l in range(cfg.layers):
+        L = inputs.layer(cfg, l)  # input generation: not timed
+        t0 = time.perf_counter()
+        u = O.layer_input(x, EPS)
+        r = O.layer_forward(u, L, cfg.K)
+        x = x + r["out"]
+        t_oracle += time.perf_counter() - t0
+        layers_done += 1
+        del L
+        if t_oracle > budget_s:
+            break
+    per_token = t_oracle * cfg.layers / layers_done
+    return {"value": 1.0 / per_token, "unit": "tok/s", "cores": cores, "kind": "oracle",
+            "sample": f"1 token through {layers_done} of {cfg.layers} layers of the 35B-shaped stack "
+                      f"(float64 numpy, BLAS threads = {cores}), scaled to {cfg.layers} layers"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    cfg = CONFIGS[CFG_ID]
+    vals = []
+    for _ in range(args.warmup):
+        pass  # the oracle has no warm state; warm-up steps are not repeated
+    for _ in range(args.steps):
+        vals.append(cpu_baseline(cfg, budget_s=max(5.0, 150.0 / max(args.steps, 1))))
+    v = statistics.median(x["value"] for x in vals)
+    cb = dict(vals[0])
+    cb["value"] = v
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / v, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "35B-shaped MoE stack decode, batch 1 (40 layers, 256 experts, top-4, H 2048)",
+                   "tokens_per_step": 1, "layers": cfg.layers},
+        "cpu_baseline": cb,
+        "e2e": {"value": v, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import int4_expert_ffn_top_b200 as M
+
+    torch.cuda.set_device(local)
+    if dist is not None:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    cfg = CONFIGS[CFG_ID]
+    stack = M.DeviceStack(cfg, lambda l: inputs.layer(cfg, l), device=dev)
+    st = M.StackStructs(stack)
+    T = cfg.T
+    ws = M.workspace(M.moe_stack_workspace_size(st, T, cfg.K, cfg.K), device=dev)
+    toks = np.stack([inputs.bf16_bits_to_f32(inputs.activations(cfg, step=1 + rank * N_TOKENS + i, T=T))
+                     for i in range(N_TOKENS)])
+    xpool = torch.from_numpy(toks).to(dev)
+    x = torch.empty((T, cfg.H), device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        x.copy_(xpool[i % N_TOKENS])
+        M.moe_stack_decode(st, x, cfg.K, cfg.K, EPS, ws)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(local) as clk:
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1)
+    if dist is not None:
+        dist.barrier()
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    tokens_total = T * args.steps * world
+    value = tokens_total / (ms / 1000.0)
+
+    # end to end through the public API with host buffers: H2D of the token, D2H of the result
+    xh = torch.from_numpy(toks).pin_memory()
+    outh = torch.empty((T, cfg.H), dtype=torch.float32).pin_memory()
+    e2e_steps = max(args.steps // 4, 10)
+    for i in range(3):
+        x.copy_(xh[i], non_blocking=True)
+        M.moe_stack_decode(st, x, cfg.K, cfg.K, EPS, ws)
+        outh.copy_(x, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    e0.record(stream)
+    for i in range(e2e_steps):
+        x.copy_(xh[i % N_TOKENS], non_blocking=True)
+        M.moe_stack_decode(st, x, cfg.K, cfg.K, EPS, ws)
+        outh.copy_(x, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_e2e = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([ms_e2e], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    e2e_value = T * e2e_steps * world / (ms_e2e / 1000.0)
+
+    peak, peak_kind = peaks()
+    bytes_step = token_layer_bytes(cfg) * cfg.layers * T
+    achieved = bytes_step / (ms / args.steps / 1000.0) / 1e9
+    out = {
+        "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "35B-shaped MoE stack decode, batch 1 (40 layers, 256 experts, top-4, H 2048, "
+                               "I 512, shared expert I 512 + LoRA r16, Prerouter P 256)",
+                   "tokens_per_step": T, "layers": cfg.layers, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2: 433 MB of weights read per step, a distinct token per step",
+                   "path": "moe_stack_decode"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "peak_kind": peak_kind, "scope": "whole step (all launches)",
+                     "algorithmic_bytes_per_step": bytes_step},
+        "e2e": {"value": e2e_value, "unit": "tok/s", "h2d_bytes_per_step": T * cfg.H * 4,
+                "d2h_bytes_per_step": T * cfg.H * 4},
+        "gpu_launches": launches_per_step(cfg) * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(cfg)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

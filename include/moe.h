@@ -1,0 +1,205 @@
+/*
+ * moe.h -- C ABI of the B200 routed-expert layer library (libmoe.so).
+ *
+ * The layer is the one the Edge0 streaming-MoE pages describe: an 8-bit router
+ * with top-K softmax gating, routed experts stored as 4-bit affine group-64
+ * matrices (SwiGLU gate/up/down), an unmerged LoRA delta, a shared expert
+ * scaled by an 8-bit sigmoid gate, the weighted combine, and a Prerouter MLP
+ * head predicting the next layer's top-K.  Sources: 2kiu.com article "iPhone,
+ * Mac, Android, Windows measured: Edge0 on five platforms" (bullets "SSD expert
+ * offload", "Prerouter", "Recover-LoRA"; paragraph on config.json: group_size
+ * 64, bits 4, router gate and shared expert gate at 8 bits); autoark.ai Edge0
+ * blog (tier table: 40 layers / 256 experts / K=4 and 24 / 128 / K=8);
+ * news18a.com Edge0 article (Prerouter input = hidden state + executed experts;
+ * prediction, expert I/O and LoRA delta as separate native components).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Ownership:  the caller allocates every device buffer (weights, activations,
+ *             outputs, workspace).  The library allocates nothing and keeps no
+ *             state between calls.  All pointers are device pointers unless a
+ *             comment says "host".  Structs are read on the host during the call
+ *             and may be freed when it returns.
+ * Asynchrony: work is enqueued on `stream` (a cudaStream_t passed as void*;
+ *             NULL = legacy default stream).  A call returns after enqueueing.
+ * Errors:     argument/shape checks run on the host before any launch and return
+ *             MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED / MOE_ERR_WORKSPACE with
+ *             nothing enqueued.  A failed launch returns MOE_ERR_CUDA.  Calls
+ *             with device-side bounded waits also report through an error word.
+ * Determinism: results are bitwise reproducible for fixed inputs and launch
+ *             shapes; no atomics accumulate into outputs.
+ * Formats:    bf16/fp16 values are passed as their 16-bit patterns.
+ *   int4 matrix [out][in]: codes q[out][in/8] uint32; element k of a row sits at
+ *     bits 4*(k%8) of word k/8 (low nibble first); scale[out][in/64] and
+ *     bias[out][in/64] fp16; w[o][k] = q*scale + bias  (affine, group 64).
+ *   8-bit matrix [out][in]: q[out][in/4] uint32, element k at bits 8*(k%4) of
+ *     word k/4; same fp16 scale/bias per 64 inputs.
+ * Supported shapes: H % 64 == 0, I % 64 == 0, I_s % 64 == 0, 1 <= K <= 8,
+ *   K <= E <= 256, LoRA rank r <= 32, Prerouter P % 64 == 0.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned buffer */
+  MOE_ERR_UNSUPPORTED = 2,  /* shape outside the supported set above */
+  MOE_ERR_WORKSPACE = 3,    /* workspace smaller than moe_workspace_size() */
+  MOE_ERR_CUDA = 4,         /* a kernel launch failed (cudaGetLastError) */
+  MOE_ERR_TIMEOUT = 5       /* a device-side bounded wait gave up */
+} moe_status;
+
+/* A packed affine group-64 matrix (see Formats). `bits` is 4 or 8. */
+typedef struct {
+  const uint32_t* q;
+  const uint16_t* scale;
+  const uint16_t* bias;
+  int32_t out_dim, in_dim, bits;
+} moe_qmat;
+
+/*
+ * One routed-expert layer.
+ *
+ * Routed experts live in one HBM pool: expert e is the block at
+ * pool + e*expert_stride with the layout (offsets in bytes, I = expert
+ * intermediate size):
+ *   gate_up codes  [2I][H/8]  uint32   (rows 0..I-1 gate, I..2I-1 up)
+ *   gate_up scale  [2I][H/64] fp16
+ *   gate_up bias   [2I][H/64] fp16
+ *   down codes     [H][I/8]   uint32
+ *   down scale     [H][I/64]  fp16
+ *   down bias      [H][I/64]  fp16
+ * moe_expert_block_bytes(H, I) gives the block size; expert_stride must be at
+ * least that and a multiple of 256.
+ *
+ * LoRA (unmerged, 2kiu.com "Recover-LoRA" bullet): the delta on a projection
+ * with input x is lora_scale * B (A x), added before the activation; A is
+ * [r][in] fp16, B is [out][r] fp16.  Shared expert: index 0 gate, 1 up, 2 down;
+ * a NULL A disables that projection's delta.  Routed experts (optional, down
+ * projection only): ex_lora_A [E][r][I], ex_lora_B [E][H][r], or NULL.
+ */
+typedef struct {
+  int32_t H, E, I, I_s, r;
+  moe_qmat router;             /* 8-bit [E][H] */
+  const float* router_bias;    /* [E] fp32 added to the logits, or NULL */
+  moe_qmat shared_gate;        /* 8-bit [1][H]; g = sigmoid(w . u) */
+  moe_qmat sh_gate_up;         /* int4 [2*I_s][H], gate rows first */
+  moe_qmat sh_down;            /* int4 [H][I_s] */
+  const uint16_t* sh_lora_A[3];
+  const uint16_t* sh_lora_B[3];
+  float lora_scale;
+  const void* pool;
+  int64_t expert_stride;
+  const uint16_t* ex_lora_A;
+  const uint16_t* ex_lora_B;
+} moe_layer;
+
+/*
+ * Prerouter head (news18a.com Edge0 article, Prerouter paragraph; 2kiu.com
+ * "Prerouter" bullet): p = W2 silu(W1 [u ; multi_hot(sel)] + b1) + b2, then the
+ * top-K_next of p.  W1 [P][H+E] fp16 (first H columns act on u, last E on the
+ * multi-hot of the executed experts), b1 [P], W2 [E_next][P], b2 [E_next] fp16.
+ */
+typedef struct {
+  const uint16_t* W1;
+  const uint16_t* b1;
+  const uint16_t* W2;
+  const uint16_t* b2;
+  int32_t H, E, P, E_next;
+} moe_prerouter;
+
+/* Human-readable name of a status code (static string, host). */
+const char* moe_status_string(moe_status s);
+
+/* Bytes of one routed-expert block in the pool layout above (host). */
+size_t moe_expert_block_bytes(int32_t H, int32_t I);
+
+/*
+ * Stack glue between layers (the pages omit attention and norms; this is the
+ * plain reading used to stack MoE layers): u[t] = bf16(x[t] / sqrt(mean(x[t]^2)
+ * + eps)), computed in fp32.  x [T][H] fp32, u [T][H] bf16.
+ */
+moe_status moe_rmsnorm_bf16(const float* x, int32_t T, int32_t H, float eps, uint16_t* u, void* stream);
+
+/*
+ * Router top-K softmax gating (autoark.ai tier table: K of E routed experts;
+ * 2kiu.com config.json paragraph: the router gate is 8-bit).
+ *   logits[t][e] = sum_k u[t][k] * (q[e][k]*scale + bias) + router_bias[e]   (fp32)
+ *   idx[t][0..K-1] = the K largest logits, descending, equal values -> lower index
+ *   w[t][k]  = exp(l_k - l_0) / sum_j exp(l_j - l_0) over the K selected
+ * u [T][H] bf16; logits [T][E] fp32 (required output); idx [T][K] int32;
+ * w [T][K] fp32.  Two launches.
+ */
+moe_status moe_route_topk(const moe_layer* L, const uint16_t* u, int32_t T, int32_t K,
+                          float* logits, int32_t* idx, float* w, void* stream);
+
+/*
+ * Routed experts + shared expert + combine for T tokens with K experts each
+ * (2kiu.com bullets "SSD expert offload" and "Recover-LoRA"; the pool replaces
+ * the pages' SSD with HBM):
+ *   h_{t,k} = silu(Wg u_t) * (Wu u_t),  y_{t,k} = Wd h_{t,k} (+ routed down LoRA)
+ *   for expert e = idx[t][k]; shared expert likewise with its LoRA deltas;
+ *   g_t = sigmoid(shared_gate . u_t);
+ *   out_t = sum_{k=0}^{K-1} w[t][k] y_{t,k} + g_t y_shared,t   (k order fixed)
+ * u [T][H] bf16; idx [T][K] int32 in [0,E); w [T][K] fp32.
+ * out_mode 0: out [T][H] fp32 = result;  1: out [T][H] bf16 = result;
+ *          2: out [T][H] fp32 += result (residual stream).
+ * perm_out: if not NULL, receives the expert-sorted slot order [T*K] int32
+ *   (slot t*K+k; stable, ascending slot id within an expert).
+ * workspace: device scratch of at least moe_workspace_size(L, T, K) bytes,
+ *   256-byte aligned; its contents on entry do not matter.
+ */
+moe_status moe_expert_forward(const moe_layer* L, const uint16_t* u, int32_t T, int32_t K,
+                              const int32_t* idx, const float* w, void* out, int32_t out_mode,
+                              int32_t* perm_out, void* workspace, size_t ws_bytes, void* stream);
+
+/* Scratch bytes moe_expert_forward needs for (L, T, K) (host). */
+size_t moe_workspace_size(const moe_layer* L, int32_t T, int32_t K);
+
+/*
+ * Prerouter prediction (see moe_prerouter).  u [T][H] bf16; sel [T][K] int32
+ * = experts executed at this layer; pred [T][K_next] int32 (same ordering and
+ * tie rule as moe_route_topk); scores [T][E_next] fp32 (required output, the
+ * p vector); workspace >= prerouter_workspace_size(head, T) bytes.
+ */
+moe_status prerouter_predict(const moe_prerouter* head, const uint16_t* u, const int32_t* sel,
+                             int32_t T, int32_t K, int32_t K_next, int32_t* pred, float* scores,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+size_t prerouter_workspace_size(const moe_prerouter* head, int32_t T);
+
+/*
+ * A stack of n_layers routed-expert layers on a residual stream (attention is
+ * omitted, as in the pages' statement of the hot path; the norm between
+ * layers is the moe_rmsnorm_bf16 glue):
+ *   for l: u_l = bf16(rmsnorm(x)); route; x += MoE_l(u_l); pred_l = head_l(u_l, executed_l)
+ * With use_predicted_routing (2kiu.com "Prerouter" bullet: the prediction is
+ * used directly as the routing), layer l >= 1 executes pred_{l-1} with gating
+ * weights = softmax of its own logits at those indices; requires K_next == K.
+ * x [T][H] fp32 in/out.  Optional outputs (NULL = not written):
+ *   x_trace [n_layers][T][H] fp32 (x entering each layer), u_trace [n_layers][T][H] bf16, idx_all [n_layers][T][K] executed experts,
+ *   true_idx_all [n_layers][T][K] the router's own top-K,
+ *   pred_all [n_layers][T][K_next].
+ * heads may be NULL (no Prerouter) unless use_predicted_routing.
+ * All layers must share H, E, I and r; heads share P and E_next.
+ */
+moe_status moe_stack_decode(const moe_layer* layers, const moe_prerouter* heads, int32_t n_layers, int32_t T,
+                            int32_t K, int32_t K_next, float eps, float* x, float* x_trace, uint16_t* u_trace, int32_t* idx_all,
+                            int32_t* true_idx_all, int32_t* pred_all, int32_t use_predicted_routing,
+                            void* workspace, size_t ws_bytes, void* stream);
+
+size_t moe_stack_workspace_size(const moe_layer* layers, const moe_prerouter* heads, int32_t n_layers, int32_t T,
+                                int32_t K, int32_t K_next);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

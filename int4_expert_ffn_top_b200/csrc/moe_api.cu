@@ -1,0 +1,465 @@
+// C ABI of the routed-expert layer library: argument checks on the host, then
+// kernel launches on the caller's stream.  Nothing here allocates memory.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "../../include/moe.h"
+#include "layer_kernels.cuh"
+
+namespace {
+
+using namespace moe;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline bool pow2_in(int v, int lo, int hi) { return v >= lo && v <= hi && (v & (v - 1)) == 0; }
+
+// Supported hidden sizes and intermediate sizes (template instantiations).
+inline bool h_ok(int H) { return pow2_in(H, 256, 4096); }
+inline bool i_ok(int I) { return pow2_in(I, 128, 2048); }
+
+moe_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+bool qmat_ok(const moe_qmat& m, int out_dim, int in_dim, int bits) {
+  return m.q && m.scale && m.bias && m.out_dim == out_dim && m.in_dim == in_dim && m.bits == bits &&
+         aligned(m.q, 16) && aligned(m.scale, 2) && aligned(m.bias, 2);
+}
+
+moe_status check_layer(const moe_layer* L, int T, int K) {
+  if (!L) return MOE_ERR_INVALID_ARG;
+  if (T < 0 || K < 1 || K > 8) return MOE_ERR_UNSUPPORTED;
+  if (!h_ok(L->H) || !i_ok(L->I) || L->I_s != L->I) return MOE_ERR_UNSUPPORTED;
+  if (L->E < K || L->E > 256 || L->r < 0 || L->r > 32) return MOE_ERR_UNSUPPORTED;
+  if (!qmat_ok(L->router, L->E, L->H, 8)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+// Workspace carve-up of moe_expert_forward.
+struct Ws {
+  int32_t *idx, *count, *offset, *perm, *inv;
+  float *g, *t_gu, *t_ds, *t_ex;
+  uint16_t* h16;
+  size_t bytes;
+};
+
+Ws carve(void* base, int T, int K, int E, int I, int r) {
+  Ws w{};
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    const size_t o = off;
+    off = align_up(off + n, 256);
+    return base ? static_cast<char*>(base) + o : nullptr;
+  };
+  const size_t TK = static_cast<size_t>(T) * K;
+  w.idx = reinterpret_cast<int32_t*>(take(TK * 4));
+  w.count = reinterpret_cast<int32_t*>(take(static_cast<size_t>(E) * 4));
+  w.offset = reinterpret_cast<int32_t*>(take(static_cast<size_t>(E + 1) * 4));
+  w.perm = reinterpret_cast<int32_t*>(take(TK * 4));
+  w.inv = reinterpret_cast<int32_t*>(take(TK * 4));
+  w.g = reinterpret_cast<float*>(take(static_cast<size_t>(T) * 4));
+  w.t_gu = reinterpret_cast<float*>(take(static_cast<size_t>(T) * 2 * (r > 0 ? r : 1) * 4));
+  w.t_ds = reinterpret_cast<float*>(take(static_cast<size_t>(T) * (r > 0 ? r : 1) * 4));
+  w.t_ex = reinterpret_cast<float*>(take(TK * (r > 0 ? r : 1) * 4));
+  w.h16 = reinterpret_cast<uint16_t*>(take((TK + T) * static_cast<size_t>(I) * 2));
+  w.bytes = off;
+  return w;
+}
+
+size_t gemv_smem(int H, bool sum32, bool sum16) {
+  return static_cast<size_t>(TB) * H * 2 + (sum32 ? static_cast<size_t>(TB) * (H / 32) * 4 : 0) +
+         (sum16 ? static_cast<size_t>(TB) * (H / 16) * 4 : 0);
+}
+
+template <typename KernelT>
+void allow_smem(KernelT k, size_t bytes) {
+  if (bytes > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+}
+
+template <int H>
+moe_status route_h(const moe_layer* L, const uint16_t* u, int T, int K, float* logits, int32_t* idx, float* w,
+                   cudaStream_t st) {
+  constexpr int NCH = H / 16;
+  constexpr int SEG = NCH < 32 ? NCH : 32;
+  const int rows_per_cta = kWarps * (32 / SEG);
+  const size_t smem = gemv_smem(H, false, true);
+  allow_smem(router_kernel<NCH>, smem);
+  dim3 grid((L->E + rows_per_cta - 1) / rows_per_cta, (T + TB - 1) / TB);
+  router_kernel<NCH><<<grid, kThreads, smem, st>>>(u, T, L->router.q, L->router.scale, L->router.bias,
+                                                   L->router_bias, L->E, logits);
+  topk_kernel<<<(T + kWarps - 1) / kWarps, kThreads, 0, st>>>(logits, T, L->E, K, idx, w);
+  return launch_status();
+}
+
+template <int H, int I>
+moe_status expert_forward_hi(const moe_layer* L, const uint16_t* u, int T, int K, const int32_t* idx, const float* w,
+                             void* out, int out_mode, int32_t* perm_out, const Ws& ws, cudaStream_t st) {
+  const int TK = T * K;
+  // 1) buckets, shared gate, shared LoRA A u
+  PreArgs pa{};
+  pa.u = u;
+  pa.T = T;
+  pa.K = K;
+  pa.E = L->E;
+  pa.r = L->r;
+  pa.idx_in = idx;
+  pa.idx = ws.idx;
+  pa.perm_out = perm_out;
+  pa.count = ws.count;
+  pa.offset = ws.offset;
+  pa.perm = ws.perm;
+  pa.inv = ws.inv;
+  pa.sg_q = L->shared_gate.q;
+  pa.sg_s = L->shared_gate.scale;
+  pa.sg_b = L->shared_gate.bias;
+  pa.A_gate = L->r > 0 ? L->sh_lora_A[0] : nullptr;
+  pa.A_up = L->r > 0 ? L->sh_lora_A[1] : nullptr;
+  pa.g = ws.g;
+  pa.t_gu = ws.t_gu;
+  const int nrows = 1 + (pa.A_gate ? L->r : 0) + (pa.A_up ? L->r : 0);
+  const size_t smem_pre = gemv_smem(H, false, true);
+  allow_smem(pre_kernel<H / 8>, smem_pre);
+  pre_kernel<H / 8><<<1 + (nrows + kWarps - 1) / kWarps, kThreads, smem_pre, st>>>(pa);
+  // 2) gate/up + SwiGLU for every touched expert and the shared expert
+  GateUpArgs ga{};
+  ga.u = u;
+  ga.T = T;
+  ga.K = K;
+  ga.I = I;
+  ga.idx = ws.idx;
+  ga.perm = ws.perm;
+  ga.offset = ws.offset;
+  ga.pool = static_cast<const uint8_t*>(L->pool);
+  ga.stride = L->expert_stride;
+  ga.sh_q = L->sh_gate_up.q;
+  ga.sh_s = L->sh_gate_up.scale;
+  ga.sh_b = L->sh_gate_up.bias;
+  ga.sh_Bg = (L->r > 0 && L->sh_lora_A[0]) ? L->sh_lora_B[0] : nullptr;
+  ga.sh_Bu = (L->r > 0 && L->sh_lora_A[1]) ? L->sh_lora_B[1] : nullptr;
+  ga.t_gu = ws.t_gu;
+  ga.r = L->r;
+  ga.lora_scale = L->lora_scale;
+  ga.h16 = ws.h16;
+  {
+    constexpr int NCH = H / 32;
+    constexpr int SEG = NCH < 32 ? NCH : 32;
+    const int pairs_per_cta = kWarps * (32 / SEG);
+    const size_t smem = gemv_smem(H, true, false);
+    allow_smem(gate_up_kernel<NCH>, smem);
+    dim3 grid((I + pairs_per_cta - 1) / pairs_per_cta, TK + 1);
+    gate_up_kernel<NCH><<<grid, kThreads, smem, st>>>(ga);
+  }
+  // 3) LoRA A h for the shared down projection and routed down projections
+  MidArgs ma{};
+  ma.T = T;
+  ma.K = K;
+  ma.I = I;
+  ma.r = L->r;
+  ma.idx = ws.idx;
+  ma.h16 = ws.h16;
+  ma.A_sd = (L->r > 0) ? L->sh_lora_A[2] : nullptr;
+  ma.A_ex = (L->r > 0) ? L->ex_lora_A : nullptr;
+  ma.t_ds = ws.t_ds;
+  ma.t_ex = ws.t_ex;
+  const int n_mid = (ma.A_sd ? T * L->r : 0) + (ma.A_ex ? TK * L->r : 0);
+  if (n_mid > 0) lora_mid_kernel<<<(n_mid + kWarps - 1) / kWarps, kThreads, 0, st>>>(ma);
+  // 4) down projections + combine
+  DownArgs da{};
+  da.T = T;
+  da.K = K;
+  da.H = H;
+  da.I = I;
+  da.r = L->r;
+  da.idx = ws.idx;
+  da.w = w;
+  da.g = ws.g;
+  da.pool = static_cast<const uint8_t*>(L->pool);
+  da.stride = L->expert_stride;
+  da.sh_q = L->sh_down.q;
+  da.sh_s = L->sh_down.scale;
+  da.sh_b = L->sh_down.bias;
+  da.B_sd = ma.A_sd ? L->sh_lora_B[2] : nullptr;
+  da.B_ex = ma.A_ex ? L->ex_lora_B : nullptr;
+  da.t_ds = ws.t_ds;
+  da.t_ex = ws.t_ex;
+  da.lora_scale = L->lora_scale;
+  da.h16 = ws.h16;
+  da.out = out;
+  da.out_mode = out_mode;
+  down_kernel<I / 32><<<(H + kWarps - 1) / kWarps, kThreads, 0, st>>>(da);
+  return launch_status();
+}
+
+template <int H>
+moe_status expert_forward_h(const moe_layer* L, const uint16_t* u, int T, int K, const int32_t* idx, const float* w,
+                            void* out, int out_mode, int32_t* perm_out, const Ws& ws, cudaStream_t st) {
+  switch (L->I) {
+    case 128: return expert_forward_hi<H, 128>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
+    case 256: return expert_forward_hi<H, 256>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
+    case 512: return expert_forward_hi<H, 512>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
+    case 1024: return expert_forward_hi<H, 1024>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
+    case 2048: return expert_forward_hi<H, 2048>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
+    default: return MOE_ERR_UNSUPPORTED;
+  }
+}
+
+template <int H>
+moe_status prerouter_h(const moe_prerouter* P, const uint16_t* u, const int32_t* sel, int T, int K, int K_next,
+                       int32_t* pred, float* scores, float* z, cudaStream_t st) {
+  PreW1Args a{};
+  a.u = u;
+  a.T = T;
+  a.K = K;
+  a.E = P->E;
+  a.P = P->P;
+  a.sel = sel;
+  a.W1 = P->W1;
+  a.b1 = P->b1;
+  a.z = z;
+  const size_t smem = gemv_smem(H, false, false);
+  allow_smem(prerouter_w1_kernel<H / 8>, smem);
+  dim3 g1((P->P + kWarps - 1) / kWarps, (T + TB - 1) / TB);
+  prerouter_w1_kernel<H / 8><<<g1, kThreads, smem, st>>>(a);
+  prerouter_w2_kernel<<<(P->E_next + kWarps - 1) / kWarps, kThreads, 0, st>>>(z, T, P->P, P->W2, P->b2, P->E_next,
+                                                                               scores);
+  topk_kernel<<<(T + kWarps - 1) / kWarps, kThreads, 0, st>>>(scores, T, P->E_next, K_next, pred, nullptr);
+  return launch_status();
+}
+
+size_t prerouter_ws(const moe_prerouter* P, int T) {
+  return align_up(static_cast<size_t>(T) * P->P * 4, 256);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA launch failed";
+    case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+size_t moe_expert_block_bytes(int32_t H, int32_t I) {
+  if (H <= 0 || I <= 0 || H % 64 || I % 64) return 0;
+  const size_t gu = static_cast<size_t>(2 * I) * (H / 2 + 2 * 2 * (H / 64));
+  const size_t dn = static_cast<size_t>(H) * (I / 2 + 2 * 2 * (I / 64));
+  return gu + dn;
+}
+
+moe_status moe_rmsnorm_bf16(const float* x, int32_t T, int32_t H, float eps, uint16_t* u, void* stream) {
+  if (T < 0 || H <= 0 || !(eps >= 0.f)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !u) return MOE_ERR_INVALID_ARG;
+  rmsnorm_bf16_kernel<<<T, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(x, H, eps, u);
+  return launch_status();
+}
+
+moe_status moe_route_topk(const moe_layer* L, const uint16_t* u, int32_t T, int32_t K, float* logits, int32_t* idx,
+                          float* w, void* stream) {
+  const moe_status s = check_layer(L, T, K);
+  if (s != MOE_OK) return s;
+  if (T == 0) return MOE_OK;
+  if (!u || !logits || !idx || !w || !aligned(u, 16)) return MOE_ERR_INVALID_ARG;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (L->H) {
+    case 256: return route_h<256>(L, u, T, K, logits, idx, w, st);
+    case 512: return route_h<512>(L, u, T, K, logits, idx, w, st);
+    case 1024: return route_h<1024>(L, u, T, K, logits, idx, w, st);
+    case 2048: return route_h<2048>(L, u, T, K, logits, idx, w, st);
+    case 4096: return route_h<4096>(L, u, T, K, logits, idx, w, st);
+    default: return MOE_ERR_UNSUPPORTED;
+  }
+}
+
+size_t moe_workspace_size(const moe_layer* L, int32_t T, int32_t K) {
+  if (!L || T < 0 || K < 1) return 0;
+  return carve(nullptr, T, K, L->E, L->I, L->r).bytes;
+}
+
+moe_status moe_expert_forward(const moe_layer* L, const uint16_t* u, int32_t T, int32_t K, const int32_t* idx,
+                              const float* w, void* out, int32_t out_mode, int32_t* perm_out, void* workspace,
+                              size_t ws_bytes, void* stream) {
+  moe_status s = check_layer(L, T, K);
+  if (s != MOE_OK) return s;
+  if (out_mode < 0 || out_mode > 2) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!u || !idx || !w || !out || !L->pool || !aligned(u, 16) || !aligned(L->pool, 256) ||
+      L->expert_stride < static_cast<int64_t>(moe_expert_block_bytes(L->H, L->I)) || L->expert_stride % 256)
+    return MOE_ERR_INVALID_ARG;
+  if (!qmat_ok(L->shared_gate, 1, L->H, 8) || !qmat_ok(L->sh_gate_up, 2 * L->I_s, L->H, 4) ||
+      !qmat_ok(L->sh_down, L->H, L->I_s, 4))
+    return MOE_ERR_INVALID_ARG;
+  if (L->r > 0) {
+    for (int p = 0; p < 3; ++p)
+      if ((L->sh_lora_A[p] != nullptr) != (L->sh_lora_B[p] != nullptr)) return MOE_ERR_INVALID_ARG;
+    if ((L->ex_lora_A != nullptr) != (L->ex_lora_B != nullptr)) return MOE_ERR_INVALID_ARG;
+    const void* lp[8] = {L->sh_lora_A[0], L->sh_lora_A[1], L->sh_lora_A[2], L->ex_lora_A,
+                         L->sh_lora_B[0], L->sh_lora_B[1], L->sh_lora_B[2], L->ex_lora_B};
+    for (const void* p : lp)
+      if (p && !aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+  }
+  const Ws need = carve(nullptr, T, K, L->E, L->I, L->r);
+  if (!workspace || !aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < need.bytes) return MOE_ERR_WORKSPACE;
+  const Ws ws = carve(workspace, T, K, L->E, L->I, L->r);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (L->H) {
+    case 256: return expert_forward_h<256>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
+    case 512: return expert_forward_h<512>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
+    case 1024: return expert_forward_h<1024>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
+    case 2048: return expert_forward_h<2048>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
+    case 4096: return expert_forward_h<4096>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
+    default: return MOE_ERR_UNSUPPORTED;
+  }
+}
+
+size_t prerouter_workspace_size(const moe_prerouter* head, int32_t T) {
+  if (!head || T < 0) return 0;
+  return prerouter_ws(head, T);
+}
+
+moe_status prerouter_predict(const moe_prerouter* head, const uint16_t* u, const int32_t* sel, int32_t T, int32_t K,
+                             int32_t K_next, int32_t* pred, float* scores, void* workspace, size_t ws_bytes,
+                             void* stream) {
+  if (!head) return MOE_ERR_INVALID_ARG;
+  if (T < 0 || K < 1 || K > 8 || K_next < 1 || K_next > 8) return MOE_ERR_UNSUPPORTED;
+  if (!h_ok(head->H) || head->E < K || head->E > 256 || head->E % 8 || head->E_next < K_next ||
+      head->E_next > 256 || head->P < 8 || head->P % 8)
+    return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!u || !sel || !pred || !scores || !head->W1 || !head->b1 || !head->W2 || !head->b2 || !aligned(u, 16) ||
+      !aligned(head->W1, 16) || !aligned(head->W2, 16))
+    return MOE_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < prerouter_ws(head, T)) return MOE_ERR_WORKSPACE;
+  float* z = static_cast<float*>(workspace);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (head->H) {
+    case 256: return prerouter_h<256>(head, u, sel, T, K, K_next, pred, scores, z, st);
+    case 512: return prerouter_h<512>(head, u, sel, T, K, K_next, pred, scores, z, st);
+    case 1024: return prerouter_h<1024>(head, u, sel, T, K, K_next, pred, scores, z, st);
+    case 2048: return prerouter_h<2048>(head, u, sel, T, K, K_next, pred, scores, z, st);
+    case 4096: return prerouter_h<4096>(head, u, sel, T, K, K_next, pred, scores, z, st);
+    default: return MOE_ERR_UNSUPPORTED;
+  }
+}
+
+
+}  // extern "C"
+
+// ----------------------------------------------------------------------------- stacked decode
+namespace {
+struct StackWs {
+  uint16_t* u;
+  float *logits, *w, *scores;
+  int32_t *idx_true, *pred0, *pred1;
+  void* ews;
+  size_t ews_bytes;
+  void* pws;
+  size_t pws_bytes;
+  size_t bytes;
+};
+
+StackWs carve_stack(void* base, const moe_layer* L0, const moe_prerouter* P0, int T, int K, int K_next) {
+  StackWs w{};
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    const size_t o = off;
+    off = align_up(off + n, 256);
+    return base ? static_cast<char*>(base) + o : nullptr;
+  };
+  const int E_next = P0 ? P0->E_next : 1;
+  w.u = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(T) * L0->H * 2));
+  w.logits = reinterpret_cast<float*>(take(static_cast<size_t>(T) * L0->E * 4));
+  w.w = reinterpret_cast<float*>(take(static_cast<size_t>(T) * K * 4));
+  w.scores = reinterpret_cast<float*>(take(static_cast<size_t>(T) * E_next * 4));
+  w.idx_true = reinterpret_cast<int32_t*>(take(static_cast<size_t>(T) * K * 4));
+  w.pred0 = reinterpret_cast<int32_t*>(take(static_cast<size_t>(T) * K_next * 4));
+  w.pred1 = reinterpret_cast<int32_t*>(take(static_cast<size_t>(T) * K_next * 4));
+  w.ews_bytes = carve(nullptr, T, K, L0->E, L0->I, L0->r).bytes;
+  w.ews = take(w.ews_bytes);
+  w.pws_bytes = P0 ? prerouter_ws(P0, T) : 0;
+  w.pws = take(w.pws_bytes);
+  w.bytes = off;
+  return w;
+}
+}  // namespace
+
+extern "C" {
+
+size_t moe_stack_workspace_size(const moe_layer* layers, const moe_prerouter* heads, int32_t n_layers, int32_t T,
+                                int32_t K, int32_t K_next) {
+  if (!layers || n_layers < 1 || T < 0 || K < 1) return 0;
+  return carve_stack(nullptr, &layers[0], heads, T, K, K_next).bytes;
+}
+
+moe_status moe_stack_decode(const moe_layer* layers, const moe_prerouter* heads, int32_t n_layers, int32_t T,
+                            int32_t K, int32_t K_next, float eps, float* x, float* x_trace, uint16_t* u_trace, int32_t* idx_all,
+                            int32_t* true_idx_all, int32_t* pred_all, int32_t use_predicted_routing, void* workspace,
+                            size_t ws_bytes, void* stream) {
+  if (!layers || n_layers < 1 || !x) return MOE_ERR_INVALID_ARG;
+  if (use_predicted_routing && (!heads || K_next != K)) return MOE_ERR_INVALID_ARG;
+  for (int l = 0; l < n_layers; ++l) {
+    const moe_status s = check_layer(&layers[l], T, K);
+    if (s != MOE_OK) return s;
+    if (layers[l].H != layers[0].H || layers[l].E != layers[0].E || layers[l].I != layers[0].I ||
+        layers[l].r != layers[0].r)
+      return MOE_ERR_UNSUPPORTED;
+    if (heads && (heads[l].H != layers[0].H || heads[l].E != layers[0].E || heads[l].E_next != heads[0].E_next ||
+                  heads[l].P != heads[0].P))
+      return MOE_ERR_UNSUPPORTED;
+  }
+  if (T == 0) return MOE_OK;
+  const StackWs need = carve_stack(nullptr, &layers[0], heads, T, K, K_next);
+  if (!workspace || !aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < need.bytes) return MOE_ERR_WORKSPACE;
+  const StackWs ws = carve_stack(workspace, &layers[0], heads, T, K, K_next);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int H = layers[0].H, E = layers[0].E;
+  const size_t TK = static_cast<size_t>(T) * K, TKn = static_cast<size_t>(T) * K_next;
+  int32_t* pred_prev = nullptr;
+  for (int l = 0; l < n_layers; ++l) {
+    const moe_layer* L = &layers[l];
+    uint16_t* u = u_trace ? u_trace + static_cast<size_t>(l) * T * H : ws.u;
+    if (x_trace && cudaMemcpyAsync(x_trace + static_cast<size_t>(l) * T * H, x, static_cast<size_t>(T) * H * 4,
+                                   cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    moe_status s = moe_rmsnorm_bf16(x, T, H, eps, u, stream);
+    if (s != MOE_OK) return s;
+    int32_t* idx_true = true_idx_all ? true_idx_all + l * TK : (idx_all && !use_predicted_routing ? idx_all + l * TK
+                                                                                                    : ws.idx_true);
+    s = moe_route_topk(L, u, T, K, ws.logits, idx_true, ws.w, stream);
+    if (s != MOE_OK) return s;
+    const int32_t* idx_exec = idx_true;
+    if (use_predicted_routing && l > 0) {
+      gate_at_kernel<<<(T + kWarps - 1) / kWarps, kThreads, 0, st>>>(ws.logits, T, E, K, pred_prev, ws.w);
+      idx_exec = pred_prev;
+    }
+    if (idx_all && idx_all + l * TK != idx_exec &&
+        cudaMemcpyAsync(idx_all + l * TK, idx_exec, TK * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    s = moe_expert_forward(L, u, T, K, idx_exec, ws.w, x, 2, nullptr, ws.ews, ws.ews_bytes, stream);
+    if (s != MOE_OK) return s;
+    if (heads) {
+      int32_t* pred = pred_all ? pred_all + l * TKn : ((l & 1) ? ws.pred1 : ws.pred0);
+      s = prerouter_predict(&heads[l], u, idx_exec, T, K, K_next, pred, ws.scores, ws.pws, ws.pws_bytes, stream);
+      if (s != MOE_OK) return s;
+      pred_prev = pred;
+    }
+  }
+  return launch_status();
+}
+
+}  // extern "C"
+

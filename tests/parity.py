@@ -1,0 +1,82 @@
+"""Comparison rules between the CUDA path and the float64 oracle.
+
+* Floating-point outputs: ``max|gpu - ref| <= 2e-3 * max|ref|`` (bf16 activations,
+  fp32 accumulation).
+* Top-K indices: exact wherever the oracle's gap between the K-th and (K+1)-th
+  score exceeds twice a certified bound on the GPU's fp32 score error; inside
+  that margin ("certified near-ties") the GPU set must be one the margin admits.
+* bf16-rounded values (the RMSNorm glue): exact unless the float64 value lies
+  within the fp32 computation's relative error of a rounding midpoint.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from gen import inputs
+from oracle import moe_oracle as O
+
+EPS32 = 2.0 ** -24
+OUT_RTOL = 2e-3
+
+
+def assert_close_inf(gpu, ref, rtol=OUT_RTOL, what="output"):
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    scale = max(float(np.max(np.abs(ref))), 1e-30)
+    err = float(np.max(np.abs(gpu - ref))) if ref.size else 0.0
+    assert err <= rtol * scale, f"{what}: max|err| {err:.3e} > {rtol:g} * {scale:.3e}"
+    return err / scale
+
+
+def qmat_abs_terms(m: dict) -> np.ndarray:
+    """Per-element magnitudes |s (q - mid)| + |b + mid*s| of the GPU's split dequantisation."""
+    mid = 8 if m["bits"] == 4 else 128
+    q = O.unpack_codes(m["q"], m["bits"]).astype(np.float64)
+    s = np.repeat(m["s"].astype(np.float64), 64, 1)
+    b = np.repeat(m["b"].astype(np.float64), 64, 1)
+    return np.abs(q - mid) * s + np.abs(b + mid * s)
+
+
+def router_tau(u: np.ndarray, router: dict, n_round: int = 64) -> np.ndarray:
+    """Bound [T, E] on |fp32 GPU logit - exact logit| for inputs u (bf16 values)."""
+    beta = np.abs(np.asarray(router["beta"], np.float64))
+    return n_round * EPS32 * (np.abs(u) @ qmat_abs_terms(router).T) + 4 * EPS32 * beta
+
+
+def check_topk(gpu_idx, ref, tau_row, K: int, exact_order: bool = True) -> int:
+    """Check GPU top-K indices against float64 scores ``ref`` [T, E]; returns #certified near-tie rows."""
+    gpu_idx = np.asarray(gpu_idx)
+    T, E = ref.shape
+    near = 0
+    for t in range(T):
+        m = 2.0 * float(np.max(tau_row[t]) if np.ndim(tau_row) else tau_row)
+        order = np.lexsort((np.arange(E), -ref[t]))
+        kth = ref[t, order[K - 1]]
+        nxt = ref[t, order[K]] if K < E else -np.inf
+        g = [int(i) for i in gpu_idx[t]]
+        assert len(set(g)) == K and all(0 <= i < E for i in g), (t, g)
+        if kth - nxt > m:
+            assert set(g) == set(order[:K].tolist()), (t, g, order[:K])
+        else:
+            near += 1
+            chosen = np.zeros(E, bool)
+            chosen[g] = True
+            assert np.all(ref[t, chosen] >= kth - m) and np.all(ref[t, ~chosen] <= kth + m), (t, g)
+        vals = ref[t, g]
+        assert np.all(vals[:-1] >= vals[1:] - m), (t, g, vals)
+        if exact_order:
+            gaps = np.diff(np.sort(ref[t, order[:K + (1 if K < E else 0)]]))
+            if np.all(np.abs(gaps) > m):
+                assert g == order[:K].tolist(), (t, g, order[:K])
+    return near
+
+
+def check_bf16_rounding(gpu_bits, ref64, rel_err: float):
+    """GPU bf16 values equal round_bf16(ref) except where ref is within rel_err of a rounding midpoint."""
+    gpu = inputs.bf16_bits_to_f32(np.asarray(gpu_bits).view(np.uint16)).astype(np.float64)
+    want = O.round_bf16(ref64)
+    lo = O.round_bf16(ref64 * (1 - rel_err))
+    hi = O.round_bf16(ref64 * (1 + rel_err))
+    ok = (gpu == want) | ((lo != hi) & ((gpu == lo) | (gpu == hi)))
+    assert np.all(ok), f"{int((~ok).sum())} bf16 values off the certified rounding"
+    return int((gpu != want).sum())

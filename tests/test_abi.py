@@ -1,0 +1,99 @@
+"""CPU checks of the C ABI: the library loads, exports every declared symbol, and
+rejects bad arguments on the host before any launch (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from int4_expert_ffn_top_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    from int4_expert_ffn_top_b200 import _lib
+    return _lib.load()
+
+
+def declared_functions():
+    names = []
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", f)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^[A-Za-z_][\w\s\*]*?\b(\w+)\s*\(", src, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "while")))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert "moe_route_topk" in names and "moe_expert_forward" in names and "prerouter_predict" in names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_python_binding_mirrors_the_header():
+    import int4_expert_ffn_top_b200 as M
+    from int4_expert_ffn_top_b200 import _lib
+    for n in declared_functions():
+        assert n in _lib.SIGNATURES, n
+        assert hasattr(M, n), n
+
+
+def test_status_strings(lib):
+    from int4_expert_ffn_top_b200 import moe_status_string
+    assert moe_status_string(0) == "ok"
+    assert "workspace" in moe_status_string(3)
+    assert moe_status_string(99) == "unknown status"
+
+
+def test_expert_block_bytes(lib):
+    from int4_expert_ffn_top_b200 import moe_expert_block_bytes
+    from gen import CONFIGS
+    # gate/up 1024 x (1024 B codes + 64 B scales + 64 B biases) + down 2048 x (256 + 16 + 16)
+    assert moe_expert_block_bytes(2048, 512) == 1024 * 1152 + 2048 * 288 == 1769472
+    for c in CONFIGS:
+        assert moe_expert_block_bytes(c.H, c.I) == c.expert_block_bytes
+    assert moe_expert_block_bytes(2048, 100) == 0
+
+
+def test_host_side_rejections(lib):
+    from int4_expert_ffn_top_b200 import _lib
+    L = _lib.moe_layer()
+    # null layer / null pointers / bad shapes fail before any launch
+    assert lib.moe_route_topk(None, None, 1, 4, None, None, None, None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_rmsnorm_bf16(None, -1, 2048, 1e-6, None, None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_rmsnorm_bf16(None, 0, 2048, 1e-6, None, None) == _lib.MOE_OK
+    L.H, L.E, L.I, L.I_s, L.r = 2048, 256, 512, 512, 16
+    assert lib.moe_route_topk(ctypes.byref(L), None, 1, 9, None, None, None, None) == _lib.MOE_ERR_UNSUPPORTED
+    L.H = 2000
+    assert lib.moe_route_topk(ctypes.byref(L), None, 1, 4, None, None, None, None) == _lib.MOE_ERR_UNSUPPORTED
+    L.H = 2048
+    # router matrix missing
+    assert lib.moe_route_topk(ctypes.byref(L), None, 1, 4, None, None, None, None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_forward(ctypes.byref(L), None, 1, 4, None, None, None, 0, None, None, 0,
+                                  None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_forward(ctypes.byref(L), None, 1, 4, None, None, None, 7, None, None, 0,
+                                  None) == _lib.MOE_ERR_INVALID_ARG
+    P = _lib.moe_prerouter()
+    P.H, P.E, P.P, P.E_next = 2048, 256, 256, 256
+    assert lib.prerouter_predict(ctypes.byref(P), None, None, 1, 4, 9, None, None, None, 0,
+                                 None) == _lib.MOE_ERR_UNSUPPORTED
+    assert lib.prerouter_predict(ctypes.byref(P), None, None, 1, 4, 4, None, None, None, 0,
+                                 None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_stack_decode(None, None, 0, 1, 4, 4, 1e-6, None, None, None, None, None, None, 0, None, 0,
+                                None) == _lib.MOE_ERR_INVALID_ARG
+
+
+def test_workspace_sizes_grow_with_tokens(lib):
+    from int4_expert_ffn_top_b200 import _lib
+    L = _lib.moe_layer()
+    L.H, L.E, L.I, L.I_s, L.r = 2048, 256, 512, 512, 16
+    a = lib.moe_workspace_size(ctypes.byref(L), 1, 4)
+    b = lib.moe_workspace_size(ctypes.byref(L), 64, 4)
+    assert 0 < a < b and a % 256 == 0 and b % 256 == 0
+    # h for (T*K + T) slots x I fp16 dominates
+    assert b >= (64 * 4 + 64) * 512 * 2

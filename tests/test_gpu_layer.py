@@ -1,0 +1,336 @@
+"""GPU parity of the per-layer entry points against the float64 oracle.
+
+Every case feeds the same seeded inputs to both sides; expert-forward cases
+give both the same routing so that routing and expert math are checked
+separately; routing is checked with the certified near-tie rule.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from gen import CONFIGS, inputs
+from oracle import moe_oracle as O
+from parity import EPS32, assert_close_inf, check_bf16_rounding, check_topk, router_tau
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def M():
+    import int4_expert_ffn_top_b200 as mod
+    return mod
+
+
+def dev_bits(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(DEV)
+
+
+def u_vals(bits: np.ndarray) -> np.ndarray:
+    return inputs.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+class Layer:
+    def __init__(self, cfg, l=0, experts=None):
+        self.cfg = cfg
+        self.host = inputs.layer(cfg, l, experts)
+        self.dev = M().DeviceLayer(cfg, self.host)
+        self.head = M().DeviceHead(cfg, self.host["prerouter"])
+
+
+def route(layer: Layer, u_bits: np.ndarray, K: int):
+    T, E = u_bits.shape[0], layer.cfg.E
+    logits = torch.full((T, E), float("nan"), device=DEV)
+    idx = torch.full((T, K), -1, dtype=torch.int32, device=DEV)
+    w = torch.full((T, K), float("nan"), device=DEV)
+    M().moe_route_topk(layer.dev, dev_bits(u_bits), K, logits, idx, w)
+    torch.cuda.synchronize()
+    return logits.cpu().numpy().astype(np.float64), idx.cpu().numpy(), w.cpu().numpy().astype(np.float64)
+
+
+def expert_forward(layer: Layer, u_bits, K, idx, w, mode=0, x0=None, perm=False):
+    m = M()
+    T, H = u_bits.shape[0], layer.cfg.H
+    if mode == 1:
+        out = torch.zeros((T, H), dtype=torch.int16, device=DEV)
+    elif mode == 2:
+        out = torch.from_numpy(x0.astype(np.float32)).to(DEV)
+    else:
+        out = torch.full((T, H), float("nan"), device=DEV)
+    ws = m.workspace(m.moe_workspace_size(layer.dev, T, K))
+    ws.fill_(0xA5)  # contents on entry must not matter
+    perm_out = torch.full((T * K,), -1, dtype=torch.int32, device=DEV) if perm else None
+    m.moe_expert_forward(layer.dev, dev_bits(u_bits), K, torch.from_numpy(idx.astype(np.int32)).to(DEV),
+                         torch.from_numpy(w.astype(np.float32)).to(DEV), out, mode, ws, perm_out=perm_out)
+    torch.cuda.synchronize()
+    o = out.cpu().numpy()
+    if mode == 1:
+        o = inputs.bf16_bits_to_f32(o.view(np.uint16))
+    return (o.astype(np.float64), perm_out.cpu().numpy() if perm else None)
+
+
+def oracle_out(layer: Layer, u, idx, w):
+    L = layer.host
+    y = O.routed_outputs(u, L["experts"], idx)
+    return O.combine(w, y, O.shared_gate(u, L["shared"]), O.shared_expert(u, L["shared"]))
+
+
+def prerouter(layer: Layer, u_bits, sel, K_next):
+    m = M()
+    T = u_bits.shape[0]
+    pred = torch.full((T, K_next), -1, dtype=torch.int32, device=DEV)
+    scores = torch.full((T, layer.cfg.E_next), float("nan"), device=DEV)
+    ws = m.workspace(m.prerouter_workspace_size(layer.head, T))
+    m.prerouter_predict(layer.head, dev_bits(u_bits), torch.from_numpy(sel.astype(np.int32)).to(DEV), K_next, pred,
+                        scores, ws)
+    torch.cuda.synchronize()
+    return pred.cpu().numpy(), scores.cpu().numpy().astype(np.float64)
+
+
+def prerouter_tau(u, sel, head, E, n_round=128):
+    """Bound [T, E_next] on |fp32 GPU scores - exact| (first order through SiLU, |silu'| <= 1.1)."""
+    W1 = np.abs(head["W1"].astype(np.float64))
+    W2 = np.abs(head["W2"].astype(np.float64))
+    xin = np.concatenate([np.abs(u), O.multi_hot(sel, E)], axis=1)
+    a_err = n_round * EPS32 * (xin @ W1.T + np.abs(head["b1"].astype(np.float64)))
+    z = np.abs(O.silu(np.concatenate([u, O.multi_hot(sel, E)], 1) @ head["W1"].astype(np.float64).T
+                      + head["b1"].astype(np.float64)))
+    return (1.1 * a_err + 8 * EPS32 * z) @ W2.T + n_round * EPS32 * (z @ W2.T + np.abs(head["b2"].astype(np.float64)))
+
+
+@pytest.fixture(scope="module")
+def c0(cuda_ok):
+    return Layer(CONFIGS[0])
+
+
+# ----------------------------------------------------------------------------- glue
+@pytest.mark.parametrize("T,H", [(1, 256), (5, 2048), (3, 4096)])
+def test_rmsnorm_bf16_certified_rounding(cuda_ok, T, H):
+    m = M()
+    rng = np.random.default_rng(T * H)
+    x = (rng.standard_normal((T, H)) * rng.uniform(0.1, 50.0, size=(T, 1))).astype(np.float32)
+    u = torch.zeros((T, H), dtype=torch.int16, device=DEV)
+    m.moe_rmsnorm_bf16(torch.from_numpy(x).to(DEV), 1e-6, u)
+    torch.cuda.synchronize()
+    ref = O.rmsnorm(x.astype(np.float64), 1e-6)
+    check_bf16_rounding(u.cpu().numpy(), ref, rel_err=(H / 256 + 24) * EPS32)
+
+
+# ----------------------------------------------------------------------------- routing
+@pytest.mark.parametrize("T", [1, 4, 13])
+def test_route_topk_c0(c0, T):
+    cfg = c0.cfg
+    ub = inputs.activations(cfg, step=T, T=T)
+    u = u_vals(ub)
+    logits, idx, w = route(c0, ub, cfg.K)
+    ref = O.router_logits(u, c0.host["router"])
+    tau = router_tau(u, c0.host["router"])
+    assert np.all(np.abs(logits - ref) <= tau), float(np.max(np.abs(logits - ref) / tau))
+    check_topk(idx, ref, tau, cfg.K)
+    assert np.allclose(w, O.gating(ref, idx), atol=1e-6 + 4 * float(tau.max()), rtol=0)
+    assert np.allclose(w.sum(1), 1.0, atol=1e-6)
+
+
+@pytest.mark.parametrize("K", [1, 8])
+def test_route_topk_extreme_k(c0, K):
+    ub = inputs.activations(c0.cfg, step=100 + K, T=6)
+    u = u_vals(ub)
+    logits, idx, w = route(c0, ub, K)
+    ref = O.router_logits(u, c0.host["router"])
+    check_topk(idx, ref, router_tau(u, c0.host["router"]), K)
+    if K == 1:
+        assert np.all(w == 1.0)
+
+
+def test_route_topk_prefill_router_with_zipf_offsets(cuda_ok):
+    cfg = CONFIGS[3]
+    lay = Layer(cfg, 0, experts=[])
+    ub = inputs.activations(cfg, step=0, T=200)
+    u = u_vals(ub)
+    logits, idx, w = route(lay, ub, cfg.K)
+    ref = O.router_logits(u, lay.host["router"])
+    tau = router_tau(u, lay.host["router"])
+    assert np.all(np.abs(logits - ref) <= tau)
+    near = check_topk(idx, ref, tau, cfg.K)
+    assert near <= 10
+    # the offsets skew the load: the most popular expert gets far more than the mean share
+    counts = np.bincount(idx.reshape(-1), minlength=cfg.E)
+    assert counts.max() > 8 * idx.size / cfg.E
+
+
+# ----------------------------------------------------------------------------- experts + combine
+@pytest.mark.parametrize("T", [1, 4, 13])
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_expert_forward_c0(c0, T, mode):
+    cfg = c0.cfg
+    ub = inputs.activations(cfg, step=7 + T, T=T)
+    u = u_vals(ub)
+    ref_logits = O.router_logits(u, c0.host["router"])
+    idx = O.topk(ref_logits, cfg.K)
+    w = O.gating(ref_logits, idx)
+    x0 = np.random.default_rng(T).standard_normal((T, cfg.H)) * 4 if mode == 2 else None
+    out, _ = expert_forward(c0, ub, cfg.K, idx, w, mode=mode, x0=x0)
+    ref = oracle_out(c0, u, idx, w)
+    if mode == 2:
+        out = out - x0.astype(np.float32)
+    if mode == 1:
+        half_ulp = np.abs(O.round_bf16(ref) - ref)
+        assert np.all(np.abs(out - ref) <= 2e-3 * np.abs(ref).max() + half_ulp + 1e-30)
+    else:
+        assert_close_inf(out, ref)
+
+
+def test_expert_forward_duplicate_and_skewed_routing(c0):
+    cfg = c0.cfg
+    T = 11
+    ub = inputs.activations(cfg, step=3, T=T)
+    u = u_vals(ub)
+    idx = np.tile(np.array([[3, 5]]), (T, 1))
+    idx[2] = [7, 7]          # the same expert twice in one token
+    idx[9] = [15, 0]         # first and last experts
+    w = np.random.default_rng(0).dirichlet([1, 1], size=T)
+    out, perm = expert_forward(c0, ub, cfg.K, idx, w, perm=True)
+    assert_close_inf(out, oracle_out(c0, u, idx, w))
+    assert np.array_equal(perm, O.buckets(idx, cfg.E)["perm"])
+
+
+@pytest.mark.parametrize("T,K", [(13, 2), (64, 8), (1, 1)])
+def test_bucket_permutation_bit_exact(c0, T, K):
+    cfg = c0.cfg
+    rng = np.random.default_rng(T * 10 + K)
+    idx = np.stack([rng.choice(cfg.E, size=K, replace=False) for _ in range(T)])
+    ub = inputs.activations(cfg, step=50, T=T)
+    w = rng.dirichlet(np.ones(K), size=T)
+    out, perm = expert_forward(c0, ub, K, idx, w, perm=True)
+    assert np.array_equal(perm, O.buckets(idx, cfg.E)["perm"])
+    assert_close_inf(out, oracle_out(c0, u_vals(ub), idx, w))
+
+
+def test_zero_tokens_is_a_no_op(c0):
+    m = M()
+    out = torch.full((1, c0.cfg.H), 7.0, device=DEV)
+    ws = m.workspace(256)
+    empty = torch.zeros((0, c0.cfg.H), dtype=torch.int16, device=DEV)
+    m.moe_expert_forward(c0.dev, empty, 2, torch.zeros((0, 2), dtype=torch.int32, device=DEV),
+                         torch.zeros((0, 2), device=DEV), out, 0, ws)
+    torch.cuda.synchronize()
+    assert torch.all(out == 7.0)
+
+
+def test_workspace_too_small_is_rejected(c0):
+    m = M()
+    ub = dev_bits(inputs.activations(c0.cfg, T=4))
+    need = m.moe_workspace_size(c0.dev, 4, 2)
+    with pytest.raises(m.MoEError) as e:
+        m.moe_expert_forward(c0.dev, ub, 2, torch.zeros((4, 2), dtype=torch.int32, device=DEV),
+                             torch.zeros((4, 2), device=DEV), torch.zeros((4, c0.cfg.H), device=DEV), 0,
+                             m.workspace(need - 256))
+    assert e.value.code == 3
+
+
+# ----------------------------------------------------------------------------- Prerouter
+@pytest.mark.parametrize("T", [1, 4, 13])
+def test_prerouter_c0(c0, T):
+    cfg = c0.cfg
+    ub = inputs.activations(cfg, step=20 + T, T=T)
+    u = u_vals(ub)
+    sel = O.topk(O.router_logits(u, c0.host["router"]), cfg.K)
+    pred, scores = prerouter(c0, ub, sel, cfg.K)
+    ref = O.prerouter_scores(u, sel, c0.host["prerouter"], cfg.E)
+    tau = prerouter_tau(u, sel, c0.host["prerouter"], cfg.E)
+    assert np.all(np.abs(scores - ref) <= tau), float(np.max(np.abs(scores - ref) / tau))
+    check_topk(pred, ref, tau, cfg.K)
+
+
+# ----------------------------------------------------------------------------- full-size layers
+@pytest.mark.parametrize("cfg_id,l,T", [(1, 0, 1), (1, 39, 1), (2, 5, 1), (1, 3, 3)])
+def test_full_size_layer(cuda_ok, cfg_id, l, T):
+    cfg = CONFIGS[cfg_id]
+    lay = Layer(cfg, l)
+    ub = inputs.activations(cfg, step=1000 + l, T=T)
+    u = u_vals(ub)
+    logits, idx, w = route(lay, ub, cfg.K)
+    ref_logits = O.router_logits(u, lay.host["router"])
+    tau = router_tau(u, lay.host["router"])
+    assert np.all(np.abs(logits - ref_logits) <= tau)
+    check_topk(idx, ref_logits, tau, cfg.K)
+    out, _ = expert_forward(lay, ub, cfg.K, idx, w.astype(np.float64))
+    assert_close_inf(out, oracle_out(lay, u, idx, w))
+    pred, scores = prerouter(lay, ub, idx, cfg.K)
+    ref_p = O.prerouter_scores(u, idx, lay.host["prerouter"], cfg.E)
+    tau_p = prerouter_tau(u, idx, lay.host["prerouter"], cfg.E)
+    assert np.all(np.abs(scores - ref_p) <= tau_p)
+    check_topk(pred, ref_p, tau_p, cfg.K)
+
+
+# ----------------------------------------------------------------------------- stacks
+def _check_stack(cfg, stack_layers, T, res, x0, sample):
+    """Teacher-forced per-layer parity on the sampled layers of a stack run."""
+    xs = res["x_trace"]
+    for l in sample:
+        L = stack_layers(l)
+        ub = res["u_trace"][l]
+        u = u_vals(ub)
+        if l == 0:
+            check_bf16_rounding(ub, O.rmsnorm(x0.astype(np.float64), 1e-6), rel_err=(cfg.H / 256 + 24) * EPS32)
+        ref_logits = O.router_logits(u, L["router"])
+        tau = router_tau(u, L["router"])
+        check_topk(res["true_idx"][l], ref_logits, tau, cfg.K)
+        executed = res["idx"][l]
+        if cfg.predicted_routing and l > 0:
+            assert np.array_equal(executed, res["pred"][l - 1])
+        else:
+            assert np.array_equal(executed, res["true_idx"][l])
+        w = O.gating(ref_logits, executed)
+        y = O.routed_outputs(u, L["experts"], executed)
+        ref_out = O.combine(w, y, O.shared_gate(u, L["shared"]), O.shared_expert(u, L["shared"]))
+        x_next = xs[l + 1] if l + 1 < len(xs) else res["x"]
+        assert_close_inf(x_next.astype(np.float64) - xs[l].astype(np.float64), ref_out, what=f"layer {l} output")
+        ref_p = O.prerouter_scores(u, executed, L["prerouter"], cfg.E)
+        check_topk(res["pred"][l], ref_p, prerouter_tau(u, executed, L["prerouter"], cfg.E), cfg.K)
+
+
+def run_stack(stack, cfg, T, x0, predicted):
+    m = M()
+    n = stack.n
+    x = torch.from_numpy(x0.astype(np.float32)).to(DEV)
+    tr = dict(x_trace=torch.zeros((n, T, cfg.H), device=DEV),
+              u_trace=torch.zeros((n, T, cfg.H), dtype=torch.int16, device=DEV),
+              idx_all=torch.full((n, T, cfg.K), -1, dtype=torch.int32, device=DEV),
+              true_idx_all=torch.full((n, T, cfg.K), -1, dtype=torch.int32, device=DEV),
+              pred_all=torch.full((n, T, cfg.K), -1, dtype=torch.int32, device=DEV))
+    st = m.StackStructs(stack)
+    ws = m.workspace(m.moe_stack_workspace_size(st, T, cfg.K, cfg.K))
+    m.moe_stack_decode(st, x, cfg.K, cfg.K, 1e-6, ws, use_predicted_routing=predicted, **tr)
+    torch.cuda.synchronize()
+    return dict(x=x.cpu().numpy(), x_trace=tr["x_trace"].cpu().numpy(),
+                u_trace=tr["u_trace"].cpu().numpy().view(np.uint16), idx=tr["idx_all"].cpu().numpy(),
+                true_idx=tr["true_idx_all"].cpu().numpy(), pred=tr["pred_all"].cpu().numpy())
+
+
+@pytest.mark.parametrize("predicted", [False, True])
+def test_small_stack(cuda_ok, predicted):
+    cfg = dataclasses.replace(CONFIGS[0], layers=4, lora_routed_down=predicted, predicted_routing=predicted)
+    layer_fn = lambda l: inputs.layer(cfg, l)  # noqa: E731
+    stack = M().DeviceStack(cfg, layer_fn)
+    T = 5
+    x0 = inputs.bf16_bits_to_f32(inputs.activations(cfg, step=9, T=T)) * 3.0
+    res = run_stack(stack, cfg, T, x0, predicted)
+    _check_stack(cfg, layer_fn, T, res, x0, range(cfg.layers))
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("cfg_id", [1, 2])
+def test_full_size_stack_sampled_layers(cuda_ok, cfg_id):
+    """The whole 35B-/8B-shaped stack at batch 1, checked on sampled layers."""
+    cfg = CONFIGS[cfg_id]
+    stack = M().DeviceStack(cfg, lambda l: inputs.layer(cfg, l))
+    T = 1
+    x0 = inputs.bf16_bits_to_f32(inputs.activations(cfg, step=77, T=T))
+    res = run_stack(stack, cfg, T, x0, False)
+    del stack
+    torch.cuda.empty_cache()
+    sample = [0, 1, cfg.layers // 2, cfg.layers - 1]
+    needed = {l: sorted(set(res["idx"][l].reshape(-1).tolist())) for l in sample}
+    _check_stack(cfg, lambda l: inputs.layer(cfg, l, experts=needed[l]), T, res, x0, sample)
