@@ -198,6 +198,40 @@ moe_status moe_stack_decode(const moe_layer* layers, const moe_prerouter* heads,
 size_t moe_stack_workspace_size(const moe_layer* layers, const moe_prerouter* heads, int32_t n_layers, int32_t T,
                                 int32_t K, int32_t K_next);
 
+/*
+ * Allocation-free variant of moe_expert_forward.  The pages have no
+ * counterpart: this exists for callers that cannot allocate device memory for
+ * a workspace -- e.g. a host framework that owns every device allocation and
+ * hands a custom operator only its inputs and outputs, or a process whose
+ * caching allocator has already reserved nearly all of HBM so that a fresh
+ * cudaMalloc would fail.
+ *
+ * Same computation, arguments and output modes as moe_expert_forward, but the
+ * scratch comes from a fixed array of MOE_NOALLOC_SCRATCH_BYTES (4 MiB) in the
+ * library's device memory, which every GPU that loads the library reserves
+ * until the process exits.  This call itself allocates nothing (no cudaMalloc,
+ * no library allocator).
+ * Errors: MOE_ERR_WORKSPACE when moe_workspace_size(L, T, K) exceeds
+ *   MOE_NOALLOC_SCRATCH_BYTES (nothing is enqueued); otherwise as
+ *   moe_expert_forward.
+ * Set-up: the first call on a device (with that device current) looks up the
+ *   array's device address once; make that first call before any stream
+ *   capture on that device.
+ * Sharing: all calls in the process share the one array per device and it
+ *   keeps the previous call's contents.  Every scratch word the kernels read
+ *   is written earlier in the same call, so nothing needs clearing; but calls
+ *   that overlap on the GPU (different streams, or different host threads
+ *   without ordering) race on the array and must be serialised by the caller.
+ */
+#define MOE_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+
+moe_status moe_expert_forward_noalloc(const moe_layer* L, const uint16_t* u, int32_t T, int32_t K,
+                                      const int32_t* idx, const float* w, void* out, int32_t out_mode,
+                                      int32_t* perm_out, void* stream);
+
+/* MOE_NOALLOC_SCRATCH_BYTES as compiled into the library (host). */
+size_t moe_noalloc_scratch_bytes(void);
+
 #ifdef __cplusplus
 }
 #endif

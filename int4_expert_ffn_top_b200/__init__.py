@@ -75,6 +75,23 @@ def moe_expert_forward(layer: DeviceLayer, u: torch.Tensor, K: int, idx: torch.T
         workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+def moe_noalloc_scratch_bytes() -> int:
+    return lib().moe_noalloc_scratch_bytes()
+
+
+def moe_expert_forward_noalloc(layer: DeviceLayer, u: torch.Tensor, K: int, idx: torch.Tensor, w: torch.Tensor,
+                               out: torch.Tensor, out_mode: int, perm_out: torch.Tensor | None = None, stream=None):
+    """moe_expert_forward without a workspace: scratch is the library's fixed per-device array.
+
+    For callers that cannot allocate device memory.  Calls share that array, so
+    calls that overlap on the GPU race; the first call on a device should come
+    before any stream capture on it.
+    """
+    T = u.shape[0]
+    _check("moe_expert_forward_noalloc", lib().moe_expert_forward_noalloc(
+        ctypes.byref(layer.struct), _p(u), T, K, _p(idx), _p(w), _p(out), out_mode, _p(perm_out), _stream(stream)))
+
+
 def prerouter_workspace_size(head: DeviceHead, T: int) -> int:
     return lib().prerouter_workspace_size(ctypes.byref(head.struct), T)
 

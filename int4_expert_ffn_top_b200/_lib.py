@@ -46,6 +46,9 @@ SIGNATURES = {
                                    c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int32,
                                    c_void_p,
                                    c_size_t, c_void_p]),
+    "moe_expert_forward_noalloc": (c_int32, [POINTER(moe_layer), c_void_p, c_int32, c_int32, c_void_p, c_void_p,
+                                             c_void_p, c_int32, c_void_p, c_void_p]),
+    "moe_noalloc_scratch_bytes": (c_size_t, []),
     "moe_stack_workspace_size": (c_size_t, [POINTER(moe_layer), POINTER(moe_prerouter), c_int32, c_int32, c_int32,
                                             c_int32]),
 }

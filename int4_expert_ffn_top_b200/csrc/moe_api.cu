@@ -4,6 +4,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "../../include/moe.h"
 #include "layer_kernels.cuh"
@@ -459,6 +460,58 @@ moe_status moe_stack_decode(const moe_layer* layers, const moe_prerouter* heads,
     }
   }
   return launch_status();
+}
+
+}  // extern "C"
+
+// ----------------------------------------------------------------------------- allocation-free variant
+// Scratch for moe_expert_forward_noalloc lives in this fixed device array
+// instead of a caller-provided workspace.  Every GPU that loads the library
+// reserves it until the process exits.  In host code the name is only a
+// host-side stand-in: its device address is fetched once per device with
+// cudaGetSymbolAddress and passed to the kernels.
+namespace {
+
+constexpr size_t kStaticScratchBytes = MOE_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::once_flag g_scratch_once[kMaxDevices];
+void* g_scratch_ptr[kMaxDevices];
+cudaError_t g_scratch_err[kMaxDevices];
+
+// Device address of the scratch array on the current device (set up on first use).
+moe_status static_scratch(void** ptr) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  std::call_once(g_scratch_once[dev], [dev] {
+    void* p = nullptr;
+    g_scratch_err[dev] = cudaGetSymbolAddress(&p, g_static_scratch);
+    g_scratch_ptr[dev] = p;
+  });
+  if (g_scratch_err[dev] != cudaSuccess || !g_scratch_ptr[dev]) return MOE_ERR_CUDA;
+  *ptr = g_scratch_ptr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_noalloc_scratch_bytes(void) { return kStaticScratchBytes; }
+
+moe_status moe_expert_forward_noalloc(const moe_layer* L, const uint16_t* u, int32_t T, int32_t K,
+                                      const int32_t* idx, const float* w, void* out, int32_t out_mode,
+                                      int32_t* perm_out, void* stream) {
+  moe_status s = check_layer(L, T, K);
+  if (s != MOE_OK) return s;
+  if (out_mode < 0 || out_mode > 2) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (moe_workspace_size(L, T, K) > kStaticScratchBytes) return MOE_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  s = static_scratch(&scratch);
+  if (s != MOE_OK) return s;
+  return moe_expert_forward(L, u, T, K, idx, w, out, out_mode, perm_out, scratch, kStaticScratchBytes, stream);
 }
 
 }  // extern "C"
