@@ -44,8 +44,10 @@ def peaks():
 
 def token_layer_bytes(cfg) -> int:
     """Algorithmic HBM bytes one token reads in one layer (batch-1 decode)."""
-    blk = cfg.expert_block_bytes
-    shared = 2 * cfg.I_s * (cfg.H // 2 + 4 * (cfg.H // 64)) + cfg.H * (cfg.I_s // 2 + 4 * (cfg.I_s // 64))
+    def mat(out, inp):  # int4 codes + fp16 scale and bias per 64 inputs
+        return out * (inp // 2 + 4 * (inp // 64))
+    blk = mat(2 * cfg.I, cfg.H) + mat(cfg.H, cfg.I)
+    shared = mat(2 * cfg.I_s, cfg.H) + mat(cfg.H, cfg.I_s)
     lora = 2 * (cfg.r * cfg.H * 2 + cfg.I_s * cfg.r * 2) + cfg.r * cfg.I_s * 2 + cfg.H * cfg.r * 2
     router = cfg.E * (cfg.H + 4 * (cfg.H // 64))
     sgate = cfg.H + 4 * (cfg.H // 64)

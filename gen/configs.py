@@ -41,13 +41,6 @@ class MoEConfig:
         # every head predicts a layer of the same stack
         return self.E
 
-    @property
-    def expert_block_bytes(self) -> int:
-        """Bytes of one routed expert: gate/up and down, codes + fp16 scales + biases."""
-        gu = 2 * self.I * (self.H // 2 + 2 * 2 * (self.H // 64))
-        dn = self.H * (self.I // 2 + 2 * 2 * (self.I // 64))
-        return gu + dn
-
 
 CONFIGS = [
     MoEConfig(0, "tiny layer", T=4, layers=1, H=256, E=16, K=2, I=128, I_s=128, r=8, P=64),

@@ -29,13 +29,19 @@
  * Determinism: results are bitwise reproducible for fixed inputs and launch
  *             shapes; no atomics accumulate into outputs.
  * Formats:    bf16/fp16 values are passed as their 16-bit patterns.
- *   int4 matrix [out][in]: codes q[out][in/8] uint32; element k of a row sits at
- *     bits 4*(k%8) of word k/8 (low nibble first); scale[out][in/64] and
- *     bias[out][in/64] fp16; w[o][k] = q*scale + bias  (affine, group 64).
- *   8-bit matrix [out][in]: q[out][in/4] uint32, element k at bits 8*(k%4) of
- *     word k/4; same fp16 scale/bias per 64 inputs.
- * Supported shapes: H % 64 == 0, I % 64 == 0, I_s % 64 == 0, 1 <= K <= 8,
- *   K <= E <= 256, LoRA rank r <= 32, Prerouter P % 64 == 0.
+ *   Row record (one row of a quantised matrix with in_dim inputs, `bits` 4 or
+ *     8): the codes (in_dim*bits/8 bytes; a 4-bit element k sits at bits
+ *     4*(k%8) of little-endian 32-bit word k/8, an 8-bit element k at byte k),
+ *     then in_dim/64 fp16 scales, then in_dim/64 fp16 biases, zero-padded to a
+ *     multiple of 16 bytes (moe_qrow_bytes).  w[o][k] = q*scale[k/64] +
+ *     bias[k/64]  (affine, group 64).
+ *   Expert block (moe_expert_block_bytes(H, I)): 2I gate/up records of H
+ *     inputs interleaved gate_0, up_0, gate_1, up_1, ..., then H down records
+ *     of I inputs.  Every row, and every run of rows one unit of work needs,
+ *     is one contiguous span (one bulk copy / one coalesced warp read).
+ * Supported shapes: H a power of two in [256, 4096], I a power of two in
+ *   [128, 2048], I_s == I, 1 <= K <= 8, K <= E <= 256, LoRA rank r <= 32,
+ *   Prerouter E % 8 == 0 and P % 8 == 0.
  */
 #ifndef MOE_H
 #define MOE_H
@@ -56,28 +62,18 @@ typedef enum {
   MOE_ERR_TIMEOUT = 5       /* a device-side bounded wait gave up */
 } moe_status;
 
-/* A packed affine group-64 matrix (see Formats). `bits` is 4 or 8. */
+/* A quantised matrix stored as out_dim row records (see Formats), 16-byte aligned. */
 typedef struct {
-  const uint32_t* q;
-  const uint16_t* scale;
-  const uint16_t* bias;
+  const void* rows;
   int32_t out_dim, in_dim, bits;
-} moe_qmat;
+} moe_qrows;
 
 /*
  * One routed-expert layer.
  *
- * Routed experts live in one HBM pool: expert e is the block at
- * pool + e*expert_stride with the layout (offsets in bytes, I = expert
- * intermediate size):
- *   gate_up codes  [2I][H/8]  uint32   (rows 0..I-1 gate, I..2I-1 up)
- *   gate_up scale  [2I][H/64] fp16
- *   gate_up bias   [2I][H/64] fp16
- *   down codes     [H][I/8]   uint32
- *   down scale     [H][I/64]  fp16
- *   down bias      [H][I/64]  fp16
- * moe_expert_block_bytes(H, I) gives the block size; expert_stride must be at
- * least that and a multiple of 256.
+ * Routed experts live in one HBM pool: expert e is the expert block at
+ * pool + e*expert_stride (expert_stride >= moe_expert_block_bytes(H, I), a
+ * multiple of 256).  The shared expert is one more expert block.
  *
  * LoRA (unmerged, 2kiu.com "Recover-LoRA" bullet): the delta on a projection
  * with input x is lora_scale * B (A x), added before the activation; A is
@@ -87,11 +83,10 @@ typedef struct {
  */
 typedef struct {
   int32_t H, E, I, I_s, r;
-  moe_qmat router;             /* 8-bit [E][H] */
+  moe_qrows router;            /* 8-bit [E][H] */
   const float* router_bias;    /* [E] fp32 added to the logits, or NULL */
-  moe_qmat shared_gate;        /* 8-bit [1][H]; g = sigmoid(w . u) */
-  moe_qmat sh_gate_up;         /* int4 [2*I_s][H], gate rows first */
-  moe_qmat sh_down;            /* int4 [H][I_s] */
+  moe_qrows shared_gate;       /* 8-bit [1][H]; g = sigmoid(w . u) */
+  const void* shared_block;    /* shared expert, one expert block (I_s == I) */
   const uint16_t* sh_lora_A[3];
   const uint16_t* sh_lora_B[3];
   float lora_scale;
@@ -118,7 +113,10 @@ typedef struct {
 /* Human-readable name of a status code (static string, host). */
 const char* moe_status_string(moe_status s);
 
-/* Bytes of one routed-expert block in the pool layout above (host). */
+/* Bytes of one row record of in_dim inputs at `bits` (4 or 8); 0 if unsupported (host). */
+size_t moe_qrow_bytes(int32_t in_dim, int32_t bits);
+
+/* Bytes of one expert block (host). */
 size_t moe_expert_block_bytes(int32_t H, int32_t I);
 
 /*
@@ -131,7 +129,7 @@ moe_status moe_rmsnorm_bf16(const float* x, int32_t T, int32_t H, float eps, uin
 /*
  * Router top-K softmax gating (autoark.ai tier table: K of E routed experts;
  * 2kiu.com config.json paragraph: the router gate is 8-bit).
- *   logits[t][e] = sum_k u[t][k] * (q[e][k]*scale + bias) + router_bias[e]   (fp32)
+ *   logits[t][e] = sum_k u[t][k] * W_r[e][k] + router_bias[e]   (fp32)
  *   idx[t][0..K-1] = the K largest logits, descending, equal values -> lower index
  *   w[t][k]  = exp(l_k - l_0) / sum_j exp(l_j - l_0) over the K selected
  * u [T][H] bf16; logits [T][E] fp32 (required output); idx [T][K] int32;

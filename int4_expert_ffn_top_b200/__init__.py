@@ -12,7 +12,7 @@ import ctypes
 import torch
 
 from . import _lib
-from .weights import DeviceHead, DeviceLayer, DeviceStack, block_bytes, block_stride  # noqa: F401
+from .weights import DeviceHead, DeviceLayer, DeviceStack, block_bytes, block_stride, qrow_bytes  # noqa: F401
 
 OUT_F32, OUT_BF16, OUT_ADD_F32 = 0, 1, 2
 
@@ -44,6 +44,10 @@ def _check(fn: str, code: int):
 
 def moe_status_string(code: int) -> str:
     return lib().moe_status_string(code).decode()
+
+
+def moe_qrow_bytes(in_dim: int, bits: int) -> int:
+    return lib().moe_qrow_bytes(in_dim, bits)
 
 
 def moe_expert_block_bytes(H: int, I: int) -> int:

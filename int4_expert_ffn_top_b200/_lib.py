@@ -11,15 +11,14 @@ LIB_PATH = os.path.join(HERE, "libmoe.so")
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = range(6)
 
 
-class moe_qmat(ctypes.Structure):
-    _fields_ = [("q", c_void_p), ("scale", c_void_p), ("bias", c_void_p),
-                ("out_dim", c_int32), ("in_dim", c_int32), ("bits", c_int32)]
+class moe_qrows(ctypes.Structure):
+    _fields_ = [("rows", c_void_p), ("out_dim", c_int32), ("in_dim", c_int32), ("bits", c_int32)]
 
 
 class moe_layer(ctypes.Structure):
     _fields_ = [("H", c_int32), ("E", c_int32), ("I", c_int32), ("I_s", c_int32), ("r", c_int32),
-                ("router", moe_qmat), ("router_bias", c_void_p), ("shared_gate", moe_qmat),
-                ("sh_gate_up", moe_qmat), ("sh_down", moe_qmat),
+                ("router", moe_qrows), ("router_bias", c_void_p), ("shared_gate", moe_qrows),
+                ("shared_block", c_void_p),
                 ("sh_lora_A", c_void_p * 3), ("sh_lora_B", c_void_p * 3), ("lora_scale", c_float),
                 ("pool", c_void_p), ("expert_stride", c_int64), ("ex_lora_A", c_void_p), ("ex_lora_B", c_void_p)]
 
@@ -32,6 +31,7 @@ class moe_prerouter(ctypes.Structure):
 # name -> (restype, argtypes); mirrors include/moe.h
 SIGNATURES = {
     "moe_status_string": (c_char_p, [c_int32]),
+    "moe_qrow_bytes": (c_size_t, [c_int32, c_int32]),
     "moe_expert_block_bytes": (c_size_t, [c_int32, c_int32]),
     "moe_rmsnorm_bf16": (c_int32, [c_void_p, c_int32, c_int32, c_float, c_void_p, c_void_p]),
     "moe_route_topk": (c_int32, [POINTER(moe_layer), c_void_p, c_int32, c_int32, c_void_p, c_void_p, c_void_p,

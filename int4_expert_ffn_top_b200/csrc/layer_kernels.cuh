@@ -17,6 +17,9 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int TB = 8;  // tokens per pass of a GEMV kernel
 
+// Bytes of one row record: codes, then in/64 fp16 scales, then in/64 fp16 biases, padded to 16.
+__host__ __device__ constexpr int qrow_bytes(int in, int bits) { return (in * bits / 8 + 4 * (in / 64) + 15) / 16 * 16; }
+
 // ----------------------------------------------------------------------------- activation staging
 // Stage tokens tok[0..nt) of u (bf16 [.][H]) into shared memory as fp16:
 // natural order (8 consecutive values per uint4) or pair order (per 8-block:
@@ -113,12 +116,12 @@ MOE_DEV void row_int8(const uint32_t* __restrict__ q, const uint16_t* __restrict
 // Router logits: logits[t][e] = W_r[e] . u[t] + bias[e].  grid (ceil(E / rows per CTA), ceil(T / TB)).
 template <int NCH>  // H / 16
 __global__ void __launch_bounds__(kThreads) router_kernel(const uint16_t* __restrict__ u, int T,
-                                                          const uint32_t* __restrict__ q, const uint16_t* __restrict__ sc,
-                                                          const uint16_t* __restrict__ bi, const float* __restrict__ rbias,
+                                                          const uint8_t* __restrict__ rows, const float* __restrict__ rbias,
                                                           int E, float* __restrict__ logits) {
   constexpr int SEG = NCH < 32 ? NCH : 32;
   constexpr int RPW = 32 / SEG;
   constexpr int H = NCH * 16;
+  constexpr int R = qrow_bytes(H, 8);
   extern __shared__ uint4 smem[];
   uint4* us = smem;
   float* sum16 = reinterpret_cast<float*>(us + TB * (H / 8));
@@ -133,9 +136,11 @@ __global__ void __launch_bounds__(kThreads) router_kernel(const uint16_t* __rest
   float acc[TB];
 #pragma unroll
   for (int t = 0; t < TB; ++t) acc[t] = 0.f;
-  if (e < E)
-    row_int8<NCH, SEG>(q + static_cast<size_t>(e) * (H / 4), sc + static_cast<size_t>(e) * (H / 64),
-                       bi + static_cast<size_t>(e) * (H / 64), us, sum16, nt, sl, acc);
+  if (e < E) {
+    const uint8_t* rec = rows + static_cast<size_t>(e) * R;
+    const uint16_t* sc = reinterpret_cast<const uint16_t*>(rec + H);
+    row_int8<NCH, SEG>(reinterpret_cast<const uint32_t*>(rec), sc, sc + H / 64, us, sum16, nt, sl, acc);
+  }
 #pragma unroll
   for (int t = 0; t < TB; ++t) acc[t] = seg_reduce<SEG>(acc[t]);
   if (e < E && sl == 0) {
@@ -305,8 +310,7 @@ struct PreArgs {
   const int32_t* idx_in;  // caller's indices
   int32_t* idx;           // clamped copy used by every later kernel
   int32_t *count, *offset, *perm, *inv, *perm_out;
-  const uint32_t* sg_q;
-  const uint16_t *sg_s, *sg_b;
+  const uint8_t* sg_rec;   // shared-gate row record (8-bit, H inputs)
   const uint16_t* A_gate;  // [r][H] or null
   const uint16_t* A_up;
   float* g;     // [T]
@@ -346,8 +350,9 @@ __global__ void __launch_bounds__(kThreads) pre_kernel(PreArgs a) {
 #pragma unroll
     for (int t = 0; t < TB; ++t) acc[t] = 0.f;
     if (row == 0) {
-      row_int8<H / 16, 32 < H / 16 ? 32 : H / 16>(a.sg_q, a.sg_s, a.sg_b, us, sum16, nt,
-                                                   lane % (32 < H / 16 ? 32 : H / 16), acc);
+      const uint16_t* sc = reinterpret_cast<const uint16_t*>(a.sg_rec + H);
+      row_int8<H / 16, 32 < H / 16 ? 32 : H / 16>(reinterpret_cast<const uint32_t*>(a.sg_rec), sc, sc + H / 64, us,
+                                                   sum16, nt, lane % (32 < H / 16 ? 32 : H / 16), acc);
       constexpr int SEG = 32 < H / 16 ? 32 : H / 16;
 #pragma unroll
       for (int t = 0; t < TB; ++t) acc[t] = seg_reduce<SEG>(acc[t]);
@@ -375,8 +380,7 @@ struct GateUpArgs {
   const int32_t *idx, *perm, *offset;
   const uint8_t* pool;
   int64_t stride;
-  const uint32_t* sh_q;
-  const uint16_t *sh_s, *sh_b;
+  const uint8_t* sh_block;        // shared expert block
   const uint16_t *sh_Bg, *sh_Bu;  // [I][r] or null
   const float* t_gu;              // [T][2][r]
   int r;
@@ -394,6 +398,7 @@ __global__ void __launch_bounds__(kThreads) gate_up_kernel(GateUpArgs a) {
   constexpr int PPW = 32 / SEG;
   constexpr int H = NCH * 32;
   constexpr int G = H / 64;
+  constexpr int RGU = qrow_bytes(H, 4);
   extern __shared__ uint4 smem[];
   uint4* up = smem;
   float* sum32 = reinterpret_cast<float*>(up + TB * (H / 8));
@@ -403,17 +408,13 @@ __global__ void __launch_bounds__(kThreads) gate_up_kernel(GateUpArgs a) {
   const int unit = blockIdx.y;
   const bool shared = unit == TK;
   int start = 0, n = a.T;
-  const uint32_t* q = a.sh_q;
-  const uint16_t *sc = a.sh_s, *bi = a.sh_b;
+  const uint8_t* blk = a.sh_block;
   if (!shared) {
     const int e = a.idx[a.perm[unit]];
     if (a.offset[e] != unit) return;
     start = unit;
     n = a.offset[e + 1] - unit;
-    const uint8_t* blk = a.pool + static_cast<int64_t>(e) * a.stride;
-    q = reinterpret_cast<const uint32_t*>(blk);
-    sc = reinterpret_cast<const uint16_t*>(blk + static_cast<size_t>(2 * a.I) * (H / 2));
-    bi = sc + static_cast<size_t>(2 * a.I) * G;
+    blk = a.pool + static_cast<int64_t>(e) * a.stride;
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, sl = lane % SEG;
   const int j = (blockIdx.x * kWarps + warp) * PPW + lane / SEG;
@@ -435,8 +436,12 @@ __global__ void __launch_bounds__(kThreads) gate_up_kernel(GateUpArgs a) {
 #pragma unroll
     for (int t = 0; t < TB; ++t) ag[t] = au[t] = 0.f;
     if (valid) {
-      const uint4* qg = reinterpret_cast<const uint4*>(q + static_cast<size_t>(j) * (H / 8));
-      const uint4* qu = reinterpret_cast<const uint4*>(q + static_cast<size_t>(j + a.I) * (H / 8));
+      const uint8_t* rg = blk + static_cast<size_t>(2 * j) * RGU;  // gate row j, then up row j
+      const uint8_t* ru = rg + RGU;
+      const uint4* qg = reinterpret_cast<const uint4*>(rg);
+      const uint4* qu = reinterpret_cast<const uint4*>(ru);
+      const uint16_t* sgp = reinterpret_cast<const uint16_t*>(rg + H / 2);
+      const uint16_t* sup = reinterpret_cast<const uint16_t*>(ru + H / 2);
       uint4 wg[CPL], wu[CPL];
 #pragma unroll
       for (int c = 0; c < CPL; ++c) {
@@ -446,10 +451,10 @@ __global__ void __launch_bounds__(kThreads) gate_up_kernel(GateUpArgs a) {
 #pragma unroll
       for (int c = 0; c < CPL; ++c) {
         const int ch = sl + c * SEG, g = ch >> 1;
-        const float sg = half_bits_to_float(sc[static_cast<size_t>(j) * G + g]);
-        const float bg = half_bits_to_float(bi[static_cast<size_t>(j) * G + g]) + 8.0f * sg;
-        const float su = half_bits_to_float(sc[static_cast<size_t>(j + a.I) * G + g]);
-        const float bu = half_bits_to_float(bi[static_cast<size_t>(j + a.I) * G + g]) + 8.0f * su;
+        const float sg = half_bits_to_float(sgp[g]);
+        const float bg = half_bits_to_float(sgp[G + g]) + 8.0f * sg;
+        const float su = half_bits_to_float(sup[g]);
+        const float bu = half_bits_to_float(sup[G + g]) + 8.0f * su;
 #pragma unroll
         for (int t = 0; t < TB; ++t) {
           if (t < nt) {
@@ -547,8 +552,7 @@ struct DownArgs {
   const float* g;
   const uint8_t* pool;
   int64_t stride;
-  const uint32_t* sh_q;
-  const uint16_t *sh_s, *sh_b;
+  const uint8_t* sh_block;
   const uint16_t* B_sd;  // [H][r] or null
   const uint16_t* B_ex;  // [E][H][r] or null
   const float* t_ds;
@@ -572,7 +576,8 @@ __global__ void __launch_bounds__(kThreads) down_kernel(DownArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, sl = lane % SEG, sub = lane / SEG;
   const int o = blockIdx.x * kWarps + warp;
   if (o >= a.H) return;
-  const size_t dn_off = static_cast<size_t>(2 * I) * (a.H / 2 + 2 * 2 * (a.H / 64));
+  constexpr int RDN = qrow_bytes(I, 4);
+  const size_t dn_off = static_cast<size_t>(2 * I) * qrow_bytes(a.H, 4) + static_cast<size_t>(o) * RDN;
   const int TK = a.T * a.K;
   for (int t = 0; t < a.T; ++t) {
     float acc = 0.f;
@@ -581,22 +586,19 @@ __global__ void __launch_bounds__(kThreads) down_kernel(DownArgs a) {
       float y = 0.f;
       int e = -1;
       if (k <= a.K) {
-        const uint32_t* q;
-        const uint16_t *sc, *bi;
+        const uint8_t* rec;
         const uint16_t* h;
         if (k < a.K) {
           e = a.idx[t * a.K + k];
-          const uint8_t* blk = a.pool + static_cast<int64_t>(e) * a.stride + dn_off;
-          q = reinterpret_cast<const uint32_t*>(blk) + static_cast<size_t>(o) * (I / 8);
-          sc = reinterpret_cast<const uint16_t*>(blk + static_cast<size_t>(a.H) * (I / 2)) + static_cast<size_t>(o) * G;
-          bi = sc + static_cast<size_t>(a.H) * G;
+          rec = a.pool + static_cast<int64_t>(e) * a.stride + dn_off;
           h = a.h16 + static_cast<size_t>(t * a.K + k) * I;
         } else {
-          q = a.sh_q + static_cast<size_t>(o) * (I / 8);
-          sc = a.sh_s + static_cast<size_t>(o) * G;
-          bi = a.sh_b + static_cast<size_t>(o) * G;
+          rec = a.sh_block + dn_off;
           h = a.h16 + static_cast<size_t>(TK + t) * I;
         }
+        const uint32_t* q = reinterpret_cast<const uint32_t*>(rec);
+        const uint16_t* sc = reinterpret_cast<const uint16_t*>(rec + I / 2);
+        const uint16_t* bi = sc + G;
         uint4 wv[CPL];
 #pragma unroll
         for (int c = 0; c < CPL; ++c) wv[c] = ldg_stream(reinterpret_cast<const uint4*>(q) + sl + c * SEG);

@@ -26,9 +26,8 @@ moe_status launch_status() {
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-bool qmat_ok(const moe_qmat& m, int out_dim, int in_dim, int bits) {
-  return m.q && m.scale && m.bias && m.out_dim == out_dim && m.in_dim == in_dim && m.bits == bits &&
-         aligned(m.q, 16) && aligned(m.scale, 2) && aligned(m.bias, 2);
+bool qrows_ok(const moe_qrows& m, int out_dim, int in_dim, int bits) {
+  return m.rows && m.out_dim == out_dim && m.in_dim == in_dim && m.bits == bits && aligned(m.rows, 16);
 }
 
 moe_status check_layer(const moe_layer* L, int T, int K) {
@@ -36,7 +35,7 @@ moe_status check_layer(const moe_layer* L, int T, int K) {
   if (T < 0 || K < 1 || K > 8) return MOE_ERR_UNSUPPORTED;
   if (!h_ok(L->H) || !i_ok(L->I) || L->I_s != L->I) return MOE_ERR_UNSUPPORTED;
   if (L->E < K || L->E > 256 || L->r < 0 || L->r > 32) return MOE_ERR_UNSUPPORTED;
-  if (!qmat_ok(L->router, L->E, L->H, 8)) return MOE_ERR_INVALID_ARG;
+  if (!qrows_ok(L->router, L->E, L->H, 8)) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -90,7 +89,7 @@ moe_status route_h(const moe_layer* L, const uint16_t* u, int T, int K, float* l
   const size_t smem = gemv_smem(H, false, true);
   allow_smem(router_kernel<NCH>, smem);
   dim3 grid((L->E + rows_per_cta - 1) / rows_per_cta, (T + TB - 1) / TB);
-  router_kernel<NCH><<<grid, kThreads, smem, st>>>(u, T, L->router.q, L->router.scale, L->router.bias,
+  router_kernel<NCH><<<grid, kThreads, smem, st>>>(u, T, static_cast<const uint8_t*>(L->router.rows),
                                                    L->router_bias, L->E, logits);
   topk_kernel<<<(T + kWarps - 1) / kWarps, kThreads, 0, st>>>(logits, T, L->E, K, idx, w);
   return launch_status();
@@ -114,9 +113,7 @@ moe_status expert_forward_hi(const moe_layer* L, const uint16_t* u, int T, int K
   pa.offset = ws.offset;
   pa.perm = ws.perm;
   pa.inv = ws.inv;
-  pa.sg_q = L->shared_gate.q;
-  pa.sg_s = L->shared_gate.scale;
-  pa.sg_b = L->shared_gate.bias;
+  pa.sg_rec = static_cast<const uint8_t*>(L->shared_gate.rows);
   pa.A_gate = L->r > 0 ? L->sh_lora_A[0] : nullptr;
   pa.A_up = L->r > 0 ? L->sh_lora_A[1] : nullptr;
   pa.g = ws.g;
@@ -136,9 +133,7 @@ moe_status expert_forward_hi(const moe_layer* L, const uint16_t* u, int T, int K
   ga.offset = ws.offset;
   ga.pool = static_cast<const uint8_t*>(L->pool);
   ga.stride = L->expert_stride;
-  ga.sh_q = L->sh_gate_up.q;
-  ga.sh_s = L->sh_gate_up.scale;
-  ga.sh_b = L->sh_gate_up.bias;
+  ga.sh_block = static_cast<const uint8_t*>(L->shared_block);
   ga.sh_Bg = (L->r > 0 && L->sh_lora_A[0]) ? L->sh_lora_B[0] : nullptr;
   ga.sh_Bu = (L->r > 0 && L->sh_lora_A[1]) ? L->sh_lora_B[1] : nullptr;
   ga.t_gu = ws.t_gu;
@@ -180,9 +175,7 @@ moe_status expert_forward_hi(const moe_layer* L, const uint16_t* u, int T, int K
   da.g = ws.g;
   da.pool = static_cast<const uint8_t*>(L->pool);
   da.stride = L->expert_stride;
-  da.sh_q = L->sh_down.q;
-  da.sh_s = L->sh_down.scale;
-  da.sh_b = L->sh_down.bias;
+  da.sh_block = static_cast<const uint8_t*>(L->shared_block);
   da.B_sd = ma.A_sd ? L->sh_lora_B[2] : nullptr;
   da.B_ex = ma.A_ex ? L->ex_lora_B : nullptr;
   da.t_ds = ws.t_ds;
@@ -251,11 +244,14 @@ const char* moe_status_string(moe_status s) {
   return "unknown status";
 }
 
+size_t moe_qrow_bytes(int32_t in_dim, int32_t bits) {
+  if (in_dim <= 0 || in_dim % 64 || (bits != 4 && bits != 8)) return 0;
+  return static_cast<size_t>(qrow_bytes(in_dim, bits));
+}
+
 size_t moe_expert_block_bytes(int32_t H, int32_t I) {
   if (H <= 0 || I <= 0 || H % 64 || I % 64) return 0;
-  const size_t gu = static_cast<size_t>(2 * I) * (H / 2 + 2 * 2 * (H / 64));
-  const size_t dn = static_cast<size_t>(H) * (I / 2 + 2 * 2 * (I / 64));
-  return gu + dn;
+  return static_cast<size_t>(2 * I) * qrow_bytes(H, 4) + static_cast<size_t>(H) * qrow_bytes(I, 4);
 }
 
 moe_status moe_rmsnorm_bf16(const float* x, int32_t T, int32_t H, float eps, uint16_t* u, void* stream) {
@@ -298,8 +294,7 @@ moe_status moe_expert_forward(const moe_layer* L, const uint16_t* u, int32_t T, 
   if (!u || !idx || !w || !out || !L->pool || !aligned(u, 16) || !aligned(L->pool, 256) ||
       L->expert_stride < static_cast<int64_t>(moe_expert_block_bytes(L->H, L->I)) || L->expert_stride % 256)
     return MOE_ERR_INVALID_ARG;
-  if (!qmat_ok(L->shared_gate, 1, L->H, 8) || !qmat_ok(L->sh_gate_up, 2 * L->I_s, L->H, 4) ||
-      !qmat_ok(L->sh_down, L->H, L->I_s, 4))
+  if (!qrows_ok(L->shared_gate, 1, L->H, 8) || !L->shared_block || !aligned(L->shared_block, 16))
     return MOE_ERR_INVALID_ARG;
   if (L->r > 0) {
     for (int p = 0; p < 3; ++p)

@@ -14,19 +14,38 @@ import torch
 from . import _lib
 
 
+def qrow_bytes(in_dim: int, bits: int) -> int:
+    """Bytes of one row record: codes, in/64 fp16 scales, in/64 fp16 biases, padded to 16."""
+    return (in_dim * bits // 8 + 4 * (in_dim // 64) + 15) // 16 * 16
+
+
 def block_bytes(H: int, I: int) -> int:
-    return 2 * I * (H // 2 + 4 * (H // 64)) + H * (I // 2 + 4 * (I // 64))
+    return 2 * I * qrow_bytes(H, 4) + H * qrow_bytes(I, 4)
 
 
 def block_stride(H: int, I: int) -> int:
     return (block_bytes(H, I) + 255) // 256 * 256
 
 
+def qrows(m: dict) -> np.ndarray:
+    """Row records ``[out, qrow_bytes]`` (uint8) of a matrix given as codes / scales / biases."""
+    out = m["q"].shape[0]
+    in_dim = m["q"].shape[1] * 32 // m["bits"]
+    cb, G = in_dim * m["bits"] // 8, in_dim // 64
+    rec = np.zeros((out, qrow_bytes(in_dim, m["bits"])), np.uint8)
+    rec[:, :cb] = np.ascontiguousarray(m["q"]).view(np.uint8).reshape(out, cb)
+    rec[:, cb:cb + 2 * G] = np.ascontiguousarray(m["s"]).view(np.uint8).reshape(out, 2 * G)
+    rec[:, cb + 2 * G:cb + 4 * G] = np.ascontiguousarray(m["b"]).view(np.uint8).reshape(out, 2 * G)
+    return rec
+
+
 def expert_block(ex: dict) -> np.ndarray:
-    """One expert's bytes in pool order."""
-    parts = [ex["gate_up"]["q"], ex["gate_up"]["s"], ex["gate_up"]["b"],
-             ex["down"]["q"], ex["down"]["s"], ex["down"]["b"]]
-    return np.concatenate([np.ascontiguousarray(p).view(np.uint8).reshape(-1) for p in parts])
+    """One expert's bytes: gate/up records interleaved (gate_0, up_0, gate_1, ...), then down records."""
+    gu = qrows(ex["gate_up"])
+    I = gu.shape[0] // 2
+    inter = np.empty_like(gu)
+    inter[0::2], inter[1::2] = gu[:I], gu[I:]
+    return np.concatenate([inter.reshape(-1), qrows(ex["down"]).reshape(-1)])
 
 
 def _dev(a: np.ndarray, device) -> torch.Tensor:
@@ -58,11 +77,10 @@ class DeviceLayer:
         R, S = host["router"], host["shared"]
         self.t = {}
         t = self.t
-        t["router_q"], t["router_s"], t["router_b"] = (_dev(R["q"], device), _dev(R["s"], device),
-                                                       _dev(R["b"], device))
+        t["router"] = _dev(qrows(R), device)
         t["router_bias"] = _dev(R["beta"].astype(np.float32), device)
-        for name, m in (("sg", S["gate"]), ("sgu", S["gate_up"]), ("sdn", S["down"])):
-            t[name + "_q"], t[name + "_s"], t[name + "_b"] = _dev(m["q"], device), _dev(m["s"], device), _dev(m["b"], device)
+        t["sgate"] = _dev(qrows(S["gate"]), device)
+        t["shared"] = _dev(expert_block(S), device)
         for i, p in enumerate(("gate", "up", "down")):
             lo = S.get("lora_" + p)
             t[f"A{i}"] = None if lo is None else _dev(lo["A"], device)
@@ -105,11 +123,10 @@ class DeviceLayer:
         c, t = self.cfg, self.t
         L = _lib.moe_layer()
         L.H, L.E, L.I, L.I_s, L.r = c.H, c.E, c.I, c.I_s, c.r
-        L.router = _lib.moe_qmat(_ptr(t["router_q"]), _ptr(t["router_s"]), _ptr(t["router_b"]), c.E, c.H, 8)
+        L.router = _lib.moe_qrows(_ptr(t["router"]), c.E, c.H, 8)
         L.router_bias = _ptr(t["router_bias"])
-        L.shared_gate = _lib.moe_qmat(_ptr(t["sg_q"]), _ptr(t["sg_s"]), _ptr(t["sg_b"]), 1, c.H, 8)
-        L.sh_gate_up = _lib.moe_qmat(_ptr(t["sgu_q"]), _ptr(t["sgu_s"]), _ptr(t["sgu_b"]), 2 * c.I_s, c.H, 4)
-        L.sh_down = _lib.moe_qmat(_ptr(t["sdn_q"]), _ptr(t["sdn_s"]), _ptr(t["sdn_b"]), c.H, c.I_s, 4)
+        L.shared_gate = _lib.moe_qrows(_ptr(t["sgate"]), 1, c.H, 8)
+        L.shared_block = _ptr(t["shared"])
         for i in range(3):
             L.sh_lora_A[i] = _ptr(t[f"A{i}"])
             L.sh_lora_B[i] = _ptr(t[f"B{i}"])

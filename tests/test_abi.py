@@ -51,13 +51,15 @@ def test_status_strings(lib):
 
 
 def test_expert_block_bytes(lib):
-    from int4_expert_ffn_top_b200 import moe_expert_block_bytes
-    from gen import CONFIGS
+    from int4_expert_ffn_top_b200 import block_bytes, moe_expert_block_bytes, moe_qrow_bytes, qrow_bytes
     # gate/up 1024 x (1024 B codes + 64 B scales + 64 B biases) + down 2048 x (256 + 16 + 16)
     assert moe_expert_block_bytes(2048, 512) == 1024 * 1152 + 2048 * 288 == 1769472
-    for c in CONFIGS:
-        assert moe_expert_block_bytes(c.H, c.I) == c.expert_block_bytes
-    assert moe_expert_block_bytes(2048, 100) == 0
+    # records pad to 16 bytes: 64 + 4 + 4 -> 80
+    assert moe_qrow_bytes(128, 4) == 80 and moe_qrow_bytes(2048, 8) == 2048 + 128
+    for H, I in ((256, 128), (2048, 512), (4096, 1024)):
+        assert moe_expert_block_bytes(H, I) == block_bytes(H, I)
+        assert moe_qrow_bytes(H, 4) == qrow_bytes(H, 4)
+    assert moe_expert_block_bytes(2048, 100) == 0 and moe_qrow_bytes(100, 4) == 0
 
 
 def test_host_side_rejections(lib):
