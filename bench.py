@@ -55,33 +55,41 @@ def token_layer_bytes(cfg) -> int:
     return cfg.K * blk + shared + lora + router + sgate + pre
 
 
-def launches_per_step(cfg, predicted=False) -> int:
+def launches_per_step(cfg, single: bool, predicted=False) -> int:
+    if single:
+        return 1  # the whole stack is one cooperative launch (plus two cudaMemsetAsync, not kernels)
     per_layer = 1 + 2 + 1 + 1 + 1 + 1 + 3  # rmsnorm, router+topk, pre, gate/up, lora-mid, down, prerouter x3
     return cfg.layers * per_layer + (cfg.layers - 1 if predicted else 0)
 
 
 class Clocks:
-    """nvidia-smi samples (SM clock, throttle reasons) during the timed region."""
+    """nvidia-smi samples (SM clock, throttle reasons), started before the warm-up so that
+    its start-up does not fall in the timed region; samples are kept by their own timestamp."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
+        self.lines = []
+        self.window = None
 
-    def __enter__(self):
+    def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True, bufsize=1)
+            self.proc.stdout.readline()  # first sample: nvidia-smi is up
         except Exception:
             self.proc = None
         return self
 
-    def __exit__(self, *a):
-        self.lines = []
+    def mark(self, t0: float, t1: float):
+        self.window = (t0, t1)
+
+    def stop(self):
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -92,20 +100,37 @@ class Clocks:
             self.lines = [l for l in out.splitlines() if l.strip()]
 
     def summary(self):
+        import datetime
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for l in self.lines:
             f = [x.strip() for x in l.split(",")]
             try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                if self.window and not (self.window[0] - 0.05 <= ts <= self.window[1] + 0.05):
+                    continue
+                sm.append(float(f[2]))
+                mx = float(f[3])
             except (ValueError, IndexError):
                 continue
-            for n, v in zip(names, f[5:9]):
+            for n, v in zip(names, f[6:10]):
                 if v.lower() == "active":
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+def measured_traffic(layers: int):
+    """DRAM bytes per stack-kernel launch from the committed ncu record, or None if the kernel changed since."""
+    import hashlib
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "stack_decode_traffic.json")))
+        src = b"".join(open(os.path.join(ROOT, f), "rb").read() for f in rec["source_files"])
+        if hashlib.sha256(src).hexdigest() != rec["source_sha256"]:
+            return None
+        return (rec["dram_bytes_read"] + rec["dram_bytes_write"]) * layers / rec["captured_layers"]
+    except Exception:
+        return None
 
 
 def cpu_baseline(cfg, budget_s: float = 20.0):
@@ -161,6 +186,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", type=int, default=0, help="0 auto, 1 per-layer launches, 2 single launch")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -194,10 +220,15 @@ def main():
     x = torch.empty((T, cfg.H), device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    opts = M.stack_opts(path=args.path)
+    err = torch.zeros((1,), dtype=torch.int32, device=dev)
+    single = args.path != 1 and T == 1
+
     def step(i):
         x.copy_(xpool[i % N_TOKENS])
-        M.moe_stack_decode(st, x, cfg.K, cfg.K, EPS, ws)
+        M.moe_stack_decode(st, x, cfg.K, cfg.K, EPS, ws, err_word=err, opts=opts)
 
+    clk = Clocks(local).start()
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize(dev)
@@ -205,13 +236,17 @@ def main():
         dist.barrier()
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with Clocks(local) as clk:
-        e0.record(stream)
-        for i in range(args.steps):
-            step(i)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
+    t0 = time.time()
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk.mark(t0, time.time())
+    clk.stop()
     ms = e0.elapsed_time(e1)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device-side wait timed out (status {int(err.item())})")
     if dist is not None:
         dist.barrier()
         t = torch.tensor([ms], device=dev)
@@ -226,7 +261,7 @@ def main():
     e2e_steps = max(args.steps // 4, 10)
     for i in range(3):
         x.copy_(xh[i], non_blocking=True)
-        M.moe_stack_decode(st, x, cfg.K, cfg.K, EPS, ws)
+        M.moe_stack_decode(st, x, cfg.K, cfg.K, EPS, ws, err_word=err, opts=opts)
         outh.copy_(x, non_blocking=True)
     torch.cuda.synchronize(dev)
     if dist is not None:
@@ -234,7 +269,7 @@ def main():
     e0.record(stream)
     for i in range(e2e_steps):
         x.copy_(xh[i % N_TOKENS], non_blocking=True)
-        M.moe_stack_decode(st, x, cfg.K, cfg.K, EPS, ws)
+        M.moe_stack_decode(st, x, cfg.K, cfg.K, EPS, ws, err_word=err, opts=opts)
         outh.copy_(x, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize(dev)
@@ -256,13 +291,15 @@ def main():
                                "I 512, shared expert I 512 + LoRA r16, Prerouter P 256)",
                    "tokens_per_step": T, "layers": cfg.layers, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2: 433 MB of weights read per step, a distinct token per step",
-                   "path": "moe_stack_decode"},
+                   "path": "moe_stack_decode, " + ("one cooperative launch per token" if single
+                                                     else "per-layer launches")},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": None, "peak_kind": peak_kind, "scope": "whole step (all launches)",
+                     "traffic": measured_traffic(cfg.layers) if single else None, "peak_kind": peak_kind,
+                     "scope": "stack kernel (the whole step)" if single else "whole step (all launches)",
                      "algorithmic_bytes_per_step": bytes_step},
         "e2e": {"value": e2e_value, "unit": "tok/s", "h2d_bytes_per_step": T * cfg.H * 4,
                 "d2h_bytes_per_step": T * cfg.H * 4},
-        "gpu_launches": launches_per_step(cfg) * args.steps,
+        "gpu_launches": launches_per_step(cfg, single) * args.steps,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -173,6 +173,27 @@ moe_status prerouter_predict(const moe_prerouter* head, const uint16_t* u, const
 
 size_t prerouter_workspace_size(const moe_prerouter* head, int32_t T);
 
+/* Options of moe_stack_decode (NULL = all defaults). */
+typedef struct {
+  int64_t timeout_ns;  /* bound on every device-side wait of the single-launch path; <= 0: 1 s */
+  int32_t path;        /* 0: automatic; 1: per-layer launches; 2: single-launch kernel (MOE_ERR_UNSUPPORTED if
+                          the shapes are not eligible) */
+  int32_t test_drop_layer;  /* test hook for the timeout path, 0 = off; L > 0: CTA test_drop_cta of the */
+  int32_t test_drop_cta;    /*   single-launch kernel never publishes its residual rows of layer L-1, so the
+                                 other CTAs' bounded waits run out and err_word reports MOE_ERR_TIMEOUT */
+  int64_t* trace;           /* optional device buffer [n_layers][moe_stack_grid()][16] of int64 %globaltimer
+                               stamps (ns) per CTA of the single-launch kernel, written by its thread 0:
+                               0 residual received, 1 router rows published, 2 logits received, 3 routed
+                               copies issued (after the block barrier), 4 hidden vector published, 5 hidden
+                               vector received, 6 residual rows published, 7 layer end, 8 RMSNorm done,
+                               9 token-independent weights landed, 10 top-K done, 11 copy barriers armed,
+                               12 copies issued, 13 first routed pair landed (if thread 0 waits for it),
+                               14 down prologue done, 15 routed down rows landed */
+} moe_stack_opts;
+
+/* Grid size (CTAs) the single-launch stack kernel uses on the current device (host). */
+int32_t moe_stack_grid(void);
+
 /*
  * A stack of n_layers routed-expert layers on a residual stream (attention is
  * omitted, as in the pages' statement of the hot path; the norm between
@@ -182,15 +203,28 @@ size_t prerouter_workspace_size(const moe_prerouter* head, int32_t T);
  * used directly as the routing), layer l >= 1 executes pred_{l-1} with gating
  * weights = softmax of its own logits at those indices; requires K_next == K.
  * x [T][H] fp32 in/out.  Optional outputs (NULL = not written):
- *   x_trace [n_layers][T][H] fp32 (x entering each layer), u_trace [n_layers][T][H] bf16, idx_all [n_layers][T][K] executed experts,
+ *   x_trace [n_layers][T][H] fp32 (x entering each layer),
+ *   u_trace [n_layers][T][H] bf16, idx_all [n_layers][T][K] executed experts,
  *   true_idx_all [n_layers][T][K] the router's own top-K,
  *   pred_all [n_layers][T][K_next].
  * heads may be NULL (no Prerouter) unless use_predicted_routing.
  * All layers must share H, E, I and r; heads share P and E_next.
+ *
+ * Paths: for one token (T == 1) without predicted routing, H 1024 or 2048,
+ * I 512, shared LoRA on all three projections or none, no routed LoRA and
+ * K_next == K, the whole stack runs as ONE cooperative kernel launch (one CTA
+ * per SM; layer-internal exchanges through device memory with bounded waits);
+ * otherwise as per-layer launches of the kernels behind the per-layer entry
+ * points.  err_word (device, optional): set to 0 at the start of the call and
+ * to MOE_ERR_TIMEOUT if a wait of the single-launch kernel gave up (its
+ * outputs are then undefined); read it after synchronising the stream.
+ * workspace >= moe_stack_workspace_size(...) bytes, 256-byte aligned; contents
+ * on entry do not matter.
  */
 moe_status moe_stack_decode(const moe_layer* layers, const moe_prerouter* heads, int32_t n_layers, int32_t T,
-                            int32_t K, int32_t K_next, float eps, float* x, float* x_trace, uint16_t* u_trace, int32_t* idx_all,
-                            int32_t* true_idx_all, int32_t* pred_all, int32_t use_predicted_routing,
+                            int32_t K, int32_t K_next, float eps, float* x, float* x_trace, uint16_t* u_trace,
+                            int32_t* idx_all, int32_t* true_idx_all, int32_t* pred_all,
+                            int32_t use_predicted_routing, int32_t* err_word, const moe_stack_opts* opts,
                             void* workspace, size_t ws_bytes, void* stream);
 
 size_t moe_stack_workspace_size(const moe_layer* layers, const moe_prerouter* heads, int32_t n_layers, int32_t T,

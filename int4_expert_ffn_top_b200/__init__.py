@@ -127,14 +127,28 @@ def moe_stack_workspace_size(stack: StackStructs, T: int, K: int, K_next: int) -
     return lib().moe_stack_workspace_size(stack.layers, stack.heads_ptr(), stack.n, T, K, K_next)
 
 
+PATH_AUTO, PATH_LAYERS, PATH_SINGLE = 0, 1, 2
+
+
+def stack_opts(timeout_ns: int = 0, path: int = PATH_AUTO, drop_layer: int = -1, drop_cta: int = -1,
+               trace: torch.Tensor | None = None):
+    """moe_stack_opts; drop_layer/drop_cta (>= 0) arm the timeout-path test hook; trace: int64 device tensor."""
+    return _lib.moe_stack_opts(timeout_ns, path, drop_layer + 1 if drop_layer >= 0 else 0, drop_cta, _p(trace))
+
+
+def moe_stack_grid() -> int:
+    return lib().moe_stack_grid()
+
+
 def moe_stack_decode(stack: StackStructs, x: torch.Tensor, K: int, K_next: int, eps: float, workspace: torch.Tensor,
-                     x_trace=None, u_trace=None, idx_all=None, true_idx_all=None, pred_all=None, use_predicted_routing=False,
-                     stream=None):
+                     x_trace=None, u_trace=None, idx_all=None, true_idx_all=None, pred_all=None,
+                     use_predicted_routing=False, err_word=None, opts=None, stream=None):
     T = x.shape[0]
     _check("moe_stack_decode", lib().moe_stack_decode(
         stack.layers, stack.heads_ptr(), stack.n, T, K, K_next, eps, _p(x), _p(x_trace), _p(u_trace), _p(idx_all),
-        _p(true_idx_all), _p(pred_all), int(bool(use_predicted_routing)), _p(workspace),
-        workspace.numel() * workspace.element_size(), _stream(stream)))
+        _p(true_idx_all), _p(pred_all), int(bool(use_predicted_routing)), _p(err_word),
+        None if opts is None else ctypes.byref(opts), _p(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
 
 
 def workspace(nbytes: int, device="cuda") -> torch.Tensor:

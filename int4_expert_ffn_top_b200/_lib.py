@@ -23,6 +23,11 @@ class moe_layer(ctypes.Structure):
                 ("pool", c_void_p), ("expert_stride", c_int64), ("ex_lora_A", c_void_p), ("ex_lora_B", c_void_p)]
 
 
+class moe_stack_opts(ctypes.Structure):
+    _fields_ = [("timeout_ns", c_int64), ("path", c_int32), ("test_drop_layer", c_int32), ("test_drop_cta", c_int32),
+                ("trace", c_void_p)]
+
+
 class moe_prerouter(ctypes.Structure):
     _fields_ = [("W1", c_void_p), ("b1", c_void_p), ("W2", c_void_p), ("b2", c_void_p),
                 ("H", c_int32), ("E", c_int32), ("P", c_int32), ("E_next", c_int32)]
@@ -44,11 +49,12 @@ SIGNATURES = {
     "prerouter_workspace_size": (c_size_t, [POINTER(moe_prerouter), c_int32]),
     "moe_stack_decode": (c_int32, [POINTER(moe_layer), POINTER(moe_prerouter), c_int32, c_int32, c_int32, c_int32,
                                    c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int32,
-                                   c_void_p,
+                                   c_void_p, POINTER(moe_stack_opts), c_void_p,
                                    c_size_t, c_void_p]),
     "moe_expert_forward_noalloc": (c_int32, [POINTER(moe_layer), c_void_p, c_int32, c_int32, c_void_p, c_void_p,
                                              c_void_p, c_int32, c_void_p, c_void_p]),
     "moe_noalloc_scratch_bytes": (c_size_t, []),
+    "moe_stack_grid": (c_int32, []),
     "moe_stack_workspace_size": (c_size_t, [POINTER(moe_layer), POINTER(moe_prerouter), c_int32, c_int32, c_int32,
                                             c_int32]),
 }

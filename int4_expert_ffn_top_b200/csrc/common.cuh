@@ -11,6 +11,12 @@ namespace moe {
 
 constexpr int kGroup = 64;
 
+// Bytes of one row record: codes, then in/64 fp16 scales, then in/64 fp16 biases, padded to 16.
+__host__ __device__ constexpr int qrow_bytes(int in, int bits) { return (in * bits / 8 + 4 * (in / 64) + 15) / 16 * 16; }
+
+// Position of element j of an fp16 vector stored in pair order (per 8-block: (v_j, v_{j+4})).
+MOE_DEV int pair_pos(int j) { return (j & ~7) + ((j & 3) << 1) + ((j >> 2) & 1); }
+
 MOE_DEV uint32_t lop_and_or(uint32_t a, uint32_t b, uint32_t c) {
   // (a & b) | c in one LOP3
   uint32_t d;
@@ -130,8 +136,10 @@ MOE_DEV uint16_t bf16_to_f16_bits(uint16_t b) {
   return __half_as_ushort(__float2half_rn(bf16_bits_to_float(b)));
 }
 
-MOE_DEV float silu(float x) { return x / (1.0f + expf(-x)); }
-MOE_DEV float sigmoid(float x) { return 1.0f / (1.0f + expf(-x)); }
+// SiLU and sigmoid through the hardware reciprocal (__fdividef, <= 2 ulp): the
+// IEEE division would inline a long slow path at every call site.
+MOE_DEV float silu(float x) { return __fdividef(x, 1.0f + expf(-x)); }
+MOE_DEV float sigmoid(float x) { return __fdividef(1.0f, 1.0f + expf(-x)); }
 
 template <int SEG>
 MOE_DEV float seg_reduce(float v) {

@@ -17,8 +17,6 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int TB = 8;  // tokens per pass of a GEMV kernel
 
-// Bytes of one row record: codes, then in/64 fp16 scales, then in/64 fp16 biases, padded to 16.
-__host__ __device__ constexpr int qrow_bytes(int in, int bits) { return (in * bits / 8 + 4 * (in / 64) + 15) / 16 * 16; }
 
 // ----------------------------------------------------------------------------- activation staging
 // Stage tokens tok[0..nt) of u (bf16 [.][H]) into shared memory as fp16:
@@ -67,8 +65,6 @@ MOE_DEV void stage_tokens(const uint16_t* __restrict__ u, int H, const int* tok,
   }
 }
 
-// Position of element j of an fp16 vector stored in pair order.
-MOE_DEV int pair_pos(int j) { return (j & ~7) + ((j & 3) << 1) + ((j >> 2) & 1); }
 
 // ----------------------------------------------------------------------------- glue: RMSNorm -> bf16
 __global__ void __launch_bounds__(kThreads) rmsnorm_bf16_kernel(const float* __restrict__ x, int H, float eps,
@@ -83,7 +79,7 @@ __global__ void __launch_bounds__(kThreads) rmsnorm_bf16_kernel(const float* __r
   float tot = 0.f;
 #pragma unroll
   for (int w = 0; w < kWarps; ++w) tot += red[w];
-  const float rs = 1.0f / sqrtf(tot / static_cast<float>(H) + eps);
+  const float rs = rsqrtf(tot / static_cast<float>(H) + eps);
   uint16_t* ur = u + static_cast<size_t>(blockIdx.x) * H;
   for (int i = threadIdx.x; i < H; i += kThreads) ur[i] = __bfloat16_as_ushort(__float2bfloat16_rn(xr[i] * rs));
 }
@@ -208,7 +204,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict_
     for (int k = 0; k < 8; ++k) {
       if (k < K) {
         idx[static_cast<size_t>(t) * K + k] = seli[k];
-        if (w) w[static_cast<size_t>(t) * K + k] = ex[k] / sum;
+        if (w) w[static_cast<size_t>(t) * K + k] = __fdividef(ex[k], sum);
       }
     }
   }
@@ -221,18 +217,23 @@ __global__ void __launch_bounds__(kThreads) gate_at_kernel(const float* __restri
   const int t = blockIdx.x * kWarps + (threadIdx.x >> 5);
   if (t >= T || (threadIdx.x & 31) != 0) return;
   float l[8], ex[8], sum = 0.f;
+#pragma unroll 1
   for (int k = 0; k < K; ++k) {
     int e = idx[static_cast<size_t>(t) * K + k];
     e = e < 0 ? 0 : (e >= E ? E - 1 : e);
     l[k] = logits[static_cast<size_t>(t) * E + e];
   }
   float m = l[0];
+#pragma unroll 1
   for (int k = 1; k < K; ++k) m = fmaxf(m, l[k]);
+#pragma unroll 1
   for (int k = 0; k < K; ++k) {
     ex[k] = expf(l[k] - m);
     sum += ex[k];
   }
-  for (int k = 0; k < K; ++k) w[static_cast<size_t>(t) * K + k] = ex[k] / sum;
+  const float inv = __fdividef(1.0f, sum);
+#pragma unroll 1
+  for (int k = 0; k < K; ++k) w[static_cast<size_t>(t) * K + k] = ex[k] * inv;
 }
 
 // ----------------------------------------------------------------------------- buckets

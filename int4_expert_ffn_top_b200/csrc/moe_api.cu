@@ -8,6 +8,7 @@
 
 #include "../../include/moe.h"
 #include "layer_kernels.cuh"
+#include "stack_kernel.cuh"
 
 namespace {
 
@@ -356,10 +357,179 @@ moe_status prerouter_predict(const moe_prerouter* head, const uint16_t* u, const
 
 // ----------------------------------------------------------------------------- stacked decode
 namespace {
+
+inline uint32_t al128(size_t x) { return static_cast<uint32_t>(align_up(x, 128)); }
+
+// Layout and eligibility of the persistent single-launch path.
+struct Persist {
+  bool ok = false;
+  stk::Smem sm{};
+  int NA = 0, grid = 0;
+  int ll_x = 0, ll_a = 0, ll_h = 0, ll_z = 0, ll_p = 0, ll_stride = 0;
+  size_t ll_bytes = 0;
+};
+
+Persist plan_persistent(const moe_layer* Ls, const moe_prerouter* Ps, int n, int T, int K, int K_next, int use_pred) {
+  Persist pl;
+  const moe_layer& L0 = Ls[0];
+  const int H = L0.H, E = L0.E, I = L0.I, r = L0.r;
+  if (T != 1 || use_pred || n > stk::kMaxLayers || (H != 1024 && H != 2048) || I != 512 || E % 8) return pl;
+  const bool lora = r > 0 && L0.sh_lora_A[0];
+  if (lora && (r % 8 || r > 32)) return pl;
+  for (int l = 0; l < n; ++l) {
+    const moe_layer& L = Ls[l];
+    if (L.ex_lora_A) return pl;
+    for (int q = 0; q < 3; ++q)
+      if ((L.sh_lora_A[q] != nullptr) != lora || (L.sh_lora_B[q] != nullptr) != lora) return pl;
+    if (!L.shared_block || !aligned(L.shared_block, 16) || !qrows_ok(L.shared_gate, 1, H, 8)) return pl;
+    if (!L.pool || !aligned(L.pool, 256) || L.expert_stride != L0.expert_stride || L.expert_stride % 256) return pl;
+    if (Ps && (!Ps[l].W1 || !Ps[l].b1 || !Ps[l].W2 || !Ps[l].b2 || !aligned(Ps[l].W1, 16) || !aligned(Ps[l].W2, 16)))
+      return pl;
+  }
+  const int P = Ps ? Ps[0].P : 0, En = Ps ? Ps[0].E_next : 0;
+  if (Ps && (P % 8 || P > 2048 || En > 256 || En < K || K_next != K)) return pl;
+  int dev = 0, nsm = 0, optin = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess || nsm <= 0)
+    return pl;
+  const int N = nsm;
+  const int NA = E + 1 + (lora ? 2 * r : 0);
+  auto cdiv = [](int a, int b) { return (a + b - 1) / b; };
+  stk::Smem& S = pl.sm;
+  S.maxA = cdiv(NA, N);
+  S.maxS = cdiv(I / 2, N);
+  S.maxR = cdiv(K * I / 2, N);
+  S.maxD = cdiv(H, N);
+  S.maxZ = P ? cdiv(P, N) : 0;
+  S.maxP = En ? cdiv(En, N) : 0;
+  const int RGU = qrow_bytes(H, 4), RDN = qrow_bytes(I, 4), R8 = qrow_bytes(H, 8), UNIT = 4 * RGU;
+  S.item_bytes = static_cast<int>(align_up(static_cast<size_t>(R8 > 2 * H ? R8 : 2 * H), 16));
+  size_t o = 0;
+  auto put = [&](size_t bytes) {
+    const uint32_t at = al128(o);
+    o = at + bytes;
+    return at;
+  };
+  S.o_items = put(static_cast<size_t>(S.maxA) * S.item_bytes);
+  S.o_shu = put(static_cast<size_t>(S.maxS) * UNIT);
+  S.o_shB = put(static_cast<size_t>(S.maxS) * 8 * r);
+  S.o_sdn = put(static_cast<size_t>(S.maxD) * RDN);
+  S.o_Bd = put(static_cast<size_t>(S.maxD) * 2 * r);
+  S.o_Ad = put(static_cast<size_t>(r) * I * 2);
+  S.o_W1 = put(static_cast<size_t>(S.maxZ) * 2 * H);
+  const uint32_t st_bytes = al128(o);
+  o = 0;
+  S.st[0] = put(st_bytes);
+  S.st[1] = put(st_bytes);
+  S.units = put(static_cast<size_t>(S.maxR) * UNIT);
+  S.down = put(static_cast<size_t>(K) * S.maxD * RDN);
+  S.xs = put(4 * H);
+  S.un = put(2 * H);
+  S.up = put(2 * H);
+  S.s16 = put(4 * H / 16);
+  S.s32 = put(4 * H / 32);
+  S.hs = put(2 * (K + 1) * I);
+  S.hsum = put(4 * (K + 1) * I / 32);
+  S.hraw = put(4 * (K + 1) * I / 2);
+  S.logit = put(4 * ((E > En ? E : En) + 1 + 2 * r));
+  S.td = put(4 * (r + 1));
+  S.yd = put(4 * S.maxD * (K + 1));
+  S.red = put(4 * 64);
+  S.z = put(4 * (P + 1));
+  S.hloc = put(4 * 2 * (S.maxS + S.maxR));
+  S.bar = put(8 * (3 + S.maxR));
+  S.sent = put(4 * 6 * N);
+  S.total = al128(o);
+  if (static_cast<int>(S.total) > optin) return pl;
+  pl.NA = NA;
+  pl.ll_x = 0;
+  pl.ll_a = H;
+  pl.ll_h = pl.ll_a + NA;
+  pl.ll_z = pl.ll_h + (K + 1) * I / 2;
+  pl.ll_stride = (pl.ll_z + P + 31) / 32 * 32;
+  pl.ll_p = 2 * pl.ll_stride;
+  pl.ll_bytes = (static_cast<size_t>(pl.ll_p) + static_cast<size_t>(n) * En) * 8;
+  pl.grid = N;
+  pl.ok = true;
+  return pl;
+}
+
+template <int H>
+cudaError_t launch_persistent(const Persist& pl, const moe_layer* Ls, const moe_prerouter* Ps, int n, int K, float eps,
+                              float* x, float* x_trace, uint16_t* u_trace, int32_t* idx_all, int32_t* true_idx_all,
+                              int32_t* pred_all, int32_t* err, unsigned long long* ll, const moe_stack_opts* opts,
+                              cudaStream_t st) {
+  auto kern = stk::stack_decode_kernel<H, 512>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(pl.sm.total));
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, stk::kThreads, pl.sm.total);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorCooperativeLaunchTooLarge;
+  stk::Params p{};
+  const moe_layer& L0 = Ls[0];
+  p.n_layers = n;
+  p.E = L0.E;
+  p.K = K;
+  p.r = (L0.r > 0 && L0.sh_lora_A[0]) ? L0.r : 0;
+  p.P = Ps ? Ps[0].P : 0;
+  p.En = Ps ? Ps[0].E_next : 0;
+  p.NA = pl.NA;
+  p.stride = L0.expert_stride;
+  p.eps = eps;
+  p.lora_scale = L0.lora_scale;
+  p.x = x;
+  p.x_trace = x_trace;
+  p.u_trace = u_trace;
+  p.idx_all = idx_all;
+  p.true_idx_all = true_idx_all;
+  p.pred_all = pred_all;
+  p.err = err;
+  p.ll = ll;
+  p.ll_x = pl.ll_x;
+  p.ll_a = pl.ll_a;
+  p.ll_h = pl.ll_h;
+  p.ll_z = pl.ll_z;
+  p.ll_p = pl.ll_p;
+  p.ll_stride = pl.ll_stride;
+  p.timeout_ns = (opts && opts->timeout_ns > 0) ? opts->timeout_ns : 1000000000LL;
+  p.drop_layer = (opts && opts->test_drop_layer > 0) ? opts->test_drop_layer - 1 : -1;
+  p.drop_cta = opts ? opts->test_drop_cta : -1;
+  p.trace = opts ? reinterpret_cast<long long*>(opts->trace) : nullptr;
+  p.sm = pl.sm;
+  for (int l = 0; l < n; ++l) {
+    const moe_layer& L = Ls[l];
+    stk::LayerPtrs& d = p.L[l];
+    d.router = static_cast<const uint8_t*>(L.router.rows);
+    d.rbias = L.router_bias;
+    d.sgate = static_cast<const uint8_t*>(L.shared_gate.rows);
+    d.shared = static_cast<const uint8_t*>(L.shared_block);
+    if (p.r) {
+      d.Ag = L.sh_lora_A[0];
+      d.Bg = L.sh_lora_B[0];
+      d.Au = L.sh_lora_A[1];
+      d.Bu = L.sh_lora_B[1];
+      d.Ad = L.sh_lora_A[2];
+      d.Bd = L.sh_lora_B[2];
+    }
+    d.pool = static_cast<const uint8_t*>(L.pool);
+    if (Ps) {
+      d.W1 = Ps[l].W1;
+      d.b1 = Ps[l].b1;
+      d.W2 = Ps[l].W2;
+      d.b2 = Ps[l].b2;
+    }
+  }
+  void* args[] = {&p};
+  return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(kern), dim3(pl.grid), dim3(stk::kThreads), args,
+                                    pl.sm.total, st);
+}
+
 struct StackWs {
   uint16_t* u;
   float *logits, *w, *scores;
-  int32_t *idx_true, *pred0, *pred1;
+  int32_t *idx_true, *pred0, *pred1, *err;
+  unsigned long long* ll;
   void* ews;
   size_t ews_bytes;
   void* pws;
@@ -367,7 +537,7 @@ struct StackWs {
   size_t bytes;
 };
 
-StackWs carve_stack(void* base, const moe_layer* L0, const moe_prerouter* P0, int T, int K, int K_next) {
+StackWs carve_stack(void* base, const moe_layer* L0, const moe_prerouter* P0, int T, int K, int K_next, size_t ll_bytes) {
   StackWs w{};
   size_t off = 0;
   auto take = [&](size_t n) {
@@ -383,6 +553,8 @@ StackWs carve_stack(void* base, const moe_layer* L0, const moe_prerouter* P0, in
   w.idx_true = reinterpret_cast<int32_t*>(take(static_cast<size_t>(T) * K * 4));
   w.pred0 = reinterpret_cast<int32_t*>(take(static_cast<size_t>(T) * K_next * 4));
   w.pred1 = reinterpret_cast<int32_t*>(take(static_cast<size_t>(T) * K_next * 4));
+  w.err = reinterpret_cast<int32_t*>(take(4));
+  w.ll = reinterpret_cast<unsigned long long*>(take(ll_bytes));
   w.ews_bytes = carve(nullptr, T, K, L0->E, L0->I, L0->r).bytes;
   w.ews = take(w.ews_bytes);
   w.pws_bytes = P0 ? prerouter_ws(P0, T) : 0;
@@ -390,22 +562,39 @@ StackWs carve_stack(void* base, const moe_layer* L0, const moe_prerouter* P0, in
   w.bytes = off;
   return w;
 }
+
+// Upper bound of the epoch-word region (two parity halves + one score vector per layer).
+size_t ll_bound(const moe_layer* L0, const moe_prerouter* P0, int K, int n_layers) {
+  const int NA = L0->E + 1 + 2 * (L0->r > 0 ? L0->r : 0);
+  const size_t words = L0->H + NA + static_cast<size_t>(K + 1) * L0->I / 2 + (P0 ? P0->P : 0) + 32;
+  return (2 * words + static_cast<size_t>(n_layers) * (P0 ? P0->E_next : 0)) * 8;
+}
+
 }  // namespace
 
 extern "C" {
 
+int32_t moe_stack_grid(void) {
+  int dev = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return nsm;
+}
+
 size_t moe_stack_workspace_size(const moe_layer* layers, const moe_prerouter* heads, int32_t n_layers, int32_t T,
                                 int32_t K, int32_t K_next) {
   if (!layers || n_layers < 1 || T < 0 || K < 1) return 0;
-  return carve_stack(nullptr, &layers[0], heads, T, K, K_next).bytes;
+  return carve_stack(nullptr, &layers[0], heads, T, K, K_next, ll_bound(&layers[0], heads, K, n_layers)).bytes;
 }
 
 moe_status moe_stack_decode(const moe_layer* layers, const moe_prerouter* heads, int32_t n_layers, int32_t T,
-                            int32_t K, int32_t K_next, float eps, float* x, float* x_trace, uint16_t* u_trace, int32_t* idx_all,
-                            int32_t* true_idx_all, int32_t* pred_all, int32_t use_predicted_routing, void* workspace,
-                            size_t ws_bytes, void* stream) {
+                            int32_t K, int32_t K_next, float eps, float* x, float* x_trace, uint16_t* u_trace,
+                            int32_t* idx_all, int32_t* true_idx_all, int32_t* pred_all, int32_t use_predicted_routing,
+                            int32_t* err_word, const moe_stack_opts* opts, void* workspace, size_t ws_bytes,
+                            void* stream) {
   if (!layers || n_layers < 1 || !x) return MOE_ERR_INVALID_ARG;
   if (use_predicted_routing && (!heads || K_next != K)) return MOE_ERR_INVALID_ARG;
+  if (opts && (opts->path < 0 || opts->path > 2)) return MOE_ERR_INVALID_ARG;
   for (int l = 0; l < n_layers; ++l) {
     const moe_status s = check_layer(&layers[l], T, K);
     if (s != MOE_OK) return s;
@@ -417,12 +606,31 @@ moe_status moe_stack_decode(const moe_layer* layers, const moe_prerouter* heads,
       return MOE_ERR_UNSUPPORTED;
   }
   if (T == 0) return MOE_OK;
-  const StackWs need = carve_stack(nullptr, &layers[0], heads, T, K, K_next);
+  const size_t llb = ll_bound(&layers[0], heads, K, n_layers);
+  const StackWs need = carve_stack(nullptr, &layers[0], heads, T, K, K_next, llb);
   if (!workspace || !aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < need.bytes) return MOE_ERR_WORKSPACE;
-  const StackWs ws = carve_stack(workspace, &layers[0], heads, T, K, K_next);
+  const StackWs ws = carve_stack(workspace, &layers[0], heads, T, K, K_next, llb);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int H = layers[0].H, E = layers[0].E;
+  int32_t* err = err_word ? err_word : ws.err;
+  if (cudaMemsetAsync(err, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  const int want = opts ? opts->path : 0;
+  if (want != 1) {
+    const Persist pl = plan_persistent(layers, heads, n_layers, T, K, K_next, use_predicted_routing);
+    if (pl.ok && pl.ll_bytes <= llb) {
+      if (cudaMemsetAsync(ws.ll, 0, pl.ll_bytes, st) != cudaSuccess) return MOE_ERR_CUDA;
+      const cudaError_t e =
+          H == 2048 ? launch_persistent<2048>(pl, layers, heads, n_layers, K, eps, x, x_trace, u_trace, idx_all,
+                                              true_idx_all, pred_all, err, ws.ll, opts, st)
+                    : launch_persistent<1024>(pl, layers, heads, n_layers, K, eps, x, x_trace, u_trace, idx_all,
+                                              true_idx_all, pred_all, err, ws.ll, opts, st);
+      return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    }
+    if (want == 2) return MOE_ERR_UNSUPPORTED;
+  }
+
   const size_t TK = static_cast<size_t>(T) * K, TKn = static_cast<size_t>(T) * K_next;
   int32_t* pred_prev = nullptr;
   for (int l = 0; l < n_layers; ++l) {

@@ -86,8 +86,8 @@ def test_host_side_rejections(lib):
                                  None) == _lib.MOE_ERR_UNSUPPORTED
     assert lib.prerouter_predict(ctypes.byref(P), None, None, 1, 4, 4, None, None, None, 0,
                                  None) == _lib.MOE_ERR_INVALID_ARG
-    assert lib.moe_stack_decode(None, None, 0, 1, 4, 4, 1e-6, None, None, None, None, None, None, 0, None, 0,
-                                None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_stack_decode(None, None, 0, 1, 4, 4, 1e-6, None, None, None, None, None, None, 0, None, None,
+                                None, 0, None) == _lib.MOE_ERR_INVALID_ARG
 
 
 def test_workspace_sizes_grow_with_tokens(lib):

@@ -291,10 +291,11 @@ def _check_stack(cfg, stack_layers, T, res, x0, sample):
         check_topk(res["pred"][l], ref_p, prerouter_tau(u, executed, L["prerouter"], cfg.E), cfg.K)
 
 
-def run_stack(stack, cfg, T, x0, predicted):
+def run_stack(stack, cfg, T, x0, predicted, opts=None):
     m = M()
     n = stack.n
     x = torch.from_numpy(x0.astype(np.float32)).to(DEV)
+    err = torch.full((1,), -7, dtype=torch.int32, device=DEV)
     tr = dict(x_trace=torch.zeros((n, T, cfg.H), device=DEV),
               u_trace=torch.zeros((n, T, cfg.H), dtype=torch.int16, device=DEV),
               idx_all=torch.full((n, T, cfg.K), -1, dtype=torch.int32, device=DEV),
@@ -302,9 +303,9 @@ def run_stack(stack, cfg, T, x0, predicted):
               pred_all=torch.full((n, T, cfg.K), -1, dtype=torch.int32, device=DEV))
     st = m.StackStructs(stack)
     ws = m.workspace(m.moe_stack_workspace_size(st, T, cfg.K, cfg.K))
-    m.moe_stack_decode(st, x, cfg.K, cfg.K, 1e-6, ws, use_predicted_routing=predicted, **tr)
+    m.moe_stack_decode(st, x, cfg.K, cfg.K, 1e-6, ws, use_predicted_routing=predicted, err_word=err, opts=opts, **tr)
     torch.cuda.synchronize()
-    return dict(x=x.cpu().numpy(), x_trace=tr["x_trace"].cpu().numpy(),
+    return dict(err=int(err.item()), x=x.cpu().numpy(), x_trace=tr["x_trace"].cpu().numpy(),
                 u_trace=tr["u_trace"].cpu().numpy().view(np.uint16), idx=tr["idx_all"].cpu().numpy(),
                 true_idx=tr["true_idx_all"].cpu().numpy(), pred=tr["pred_all"].cpu().numpy())
 
@@ -320,6 +321,51 @@ def test_small_stack(cuda_ok, predicted):
     _check_stack(cfg, layer_fn, T, res, x0, range(cfg.layers))
 
 
+SMALL_SINGLE = [dict(H=1024, E=32, K=4, P=128), dict(H=1024, E=64, K=8, P=64), dict(H=2048, E=16, K=2, P=256)]
+
+
+@pytest.mark.parametrize("shape", SMALL_SINGLE)
+def test_single_launch_stack(cuda_ok, shape):
+    """The one-launch stack kernel on small stacks, against the oracle and the per-layer path."""
+    m = M()
+    cfg = dataclasses.replace(CONFIGS[1], layers=5, I=512, I_s=512, r=16, **shape)
+    layer_fn = lambda l: inputs.layer(cfg, l)  # noqa: E731
+    stack = m.DeviceStack(cfg, layer_fn)
+    x0 = inputs.bf16_bits_to_f32(inputs.activations(cfg, step=11, T=1))
+    res = run_stack(stack, cfg, 1, x0, False, opts=m.stack_opts(path=m.PATH_SINGLE))
+    assert res["err"] == 0
+    _check_stack(cfg, layer_fn, 1, res, x0, range(cfg.layers))
+    ref = run_stack(stack, cfg, 1, x0, False, opts=m.stack_opts(path=m.PATH_LAYERS))
+    assert ref["err"] == 0
+    # both paths agree wherever routing agrees (it does unless a certified near-tie flips)
+    if all(np.array_equal(a, b) for a, b in zip(res["idx"], ref["idx"])):
+        assert_close_inf(res["x"], ref["x"], what="single launch vs per-layer launches")
+
+
+def test_single_launch_bounded_wait_reports_timeout(cuda_ok):
+    """A residual publication that never arrives: the waits give up and the status says so."""
+    m = M()
+    cfg = dataclasses.replace(CONFIGS[1], layers=3, H=1024, E=32, K=4, P=128)
+    stack = m.DeviceStack(cfg, lambda l: inputs.layer(cfg, l))
+    x0 = inputs.bf16_bits_to_f32(inputs.activations(cfg, step=12, T=1))
+    res = run_stack(stack, cfg, 1, x0, False,
+                    opts=m.stack_opts(path=m.PATH_SINGLE, timeout_ns=20_000_000, drop_layer=1, drop_cta=3))
+    assert res["err"] == 5
+    # the context stays usable: the next call succeeds
+    res2 = run_stack(stack, cfg, 1, x0, False, opts=m.stack_opts(path=m.PATH_SINGLE))
+    assert res2["err"] == 0 and np.all(np.isfinite(res2["x"]))
+
+
+def test_single_launch_rejects_ineligible_shapes(cuda_ok, c0):
+    m = M()
+    st = m.StackStructs([c0.dev], [c0.head])
+    ws = m.workspace(m.moe_stack_workspace_size(st, 1, 2, 2))
+    x = torch.zeros((1, c0.cfg.H), device=DEV)
+    with pytest.raises(m.MoEError) as e:
+        m.moe_stack_decode(st, x, 2, 2, 1e-6, ws, opts=m.stack_opts(path=m.PATH_SINGLE))
+    assert e.value.code == 2
+
+
 @pytest.mark.slow
 @pytest.mark.parametrize("cfg_id", [1, 2])
 def test_full_size_stack_sampled_layers(cuda_ok, cfg_id):
@@ -329,6 +375,7 @@ def test_full_size_stack_sampled_layers(cuda_ok, cfg_id):
     T = 1
     x0 = inputs.bf16_bits_to_f32(inputs.activations(cfg, step=77, T=T))
     res = run_stack(stack, cfg, T, x0, False)
+    assert res["err"] == 0
     del stack
     torch.cuda.empty_cache()
     sample = [0, 1, cfg.layers // 2, cfg.layers - 1]
