@@ -8,6 +8,7 @@
 
 #include "../../include/moe.h"
 #include "layer_kernels.cuh"
+#include "prefill_kernels.cuh"
 #include "stack_kernel.cuh"
 
 namespace {
@@ -42,6 +43,7 @@ moe_status check_layer(const moe_layer* L, int T, int K) {
 
 // Workspace carve-up of moe_expert_forward.
 struct Ws {
+  void* base;
   int32_t *idx, *count, *offset, *perm, *inv;
   float *g, *t_gu, *t_ds, *t_ex;
   uint16_t* h16;
@@ -50,6 +52,7 @@ struct Ws {
 
 Ws carve(void* base, int T, int K, int E, int I, int r) {
   Ws w{};
+  w.base = base;
   size_t off = 0;
   auto take = [&](size_t n) {
     const size_t o = off;
@@ -189,9 +192,181 @@ moe_status expert_forward_hi(const moe_layer* L, const uint16_t* u, int T, int K
   return launch_status();
 }
 
+// ----------------------------------------------------------------------------- grouped-GEMM path (many slots)
+constexpr int kGemmMinSlots = 128;  // T*K from which moe_expert_forward uses the tensor-core path
+
+struct GWs {
+  int32_t *idx, *count, *offset, *perm, *inv, *blockhist;
+  float *w_pos, *t1, *t2, *g;
+  uint16_t *X, *Hh, *Y;
+  gg::Tile *tiles_gu, *tiles_dn;
+  int* n_tiles;
+  int* err;
+  int max_gu, max_dn, nblk;
+  size_t bytes;
+};
+
+GWs carve_gemm(void* base, int T, int K, int E, int H, int I, int r) {
+  GWs w{};
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    const size_t o = off;
+    off = align_up(off + n, 256);
+    return base ? static_cast<char*>(base) + o : nullptr;
+  };
+  const size_t TK = static_cast<size_t>(T) * K, R = TK + T;
+  const int rr = r > 0 ? r : 1;
+  w.nblk = static_cast<int>((TK + pf::kChunk - 1) / pf::kChunk);
+  const int nt_max = static_cast<int>((TK + static_cast<size_t>(E) * (gg::BN - 1)) / gg::BN) + (T + gg::BN - 1) / gg::BN + 1;
+  w.max_gu = nt_max * (2 * I / gg::BM);
+  w.max_dn = nt_max * (H / gg::BM);
+  w.idx = reinterpret_cast<int32_t*>(take(TK * 4));
+  w.count = reinterpret_cast<int32_t*>(take(static_cast<size_t>(E) * 4));
+  w.offset = reinterpret_cast<int32_t*>(take(static_cast<size_t>(E + 1) * 4));
+  w.perm = reinterpret_cast<int32_t*>(take(TK * 4));
+  w.inv = reinterpret_cast<int32_t*>(take(TK * 4));
+  w.blockhist = reinterpret_cast<int32_t*>(take(static_cast<size_t>(w.nblk) * E * 4));
+  w.w_pos = reinterpret_cast<float*>(take(TK * 4));
+  w.t1 = reinterpret_cast<float*>(take(R * rr * 4));
+  w.t2 = reinterpret_cast<float*>(take(R * rr * 4));
+  w.g = reinterpret_cast<float*>(take(static_cast<size_t>(T) * 4));
+  w.X = reinterpret_cast<uint16_t*>(take(R * H * 2));
+  w.Hh = reinterpret_cast<uint16_t*>(take(R * I * 2));
+  w.Y = reinterpret_cast<uint16_t*>(take(R * H * 2));
+  w.tiles_gu = reinterpret_cast<gg::Tile*>(take(static_cast<size_t>(w.max_gu) * sizeof(gg::Tile)));
+  w.tiles_dn = reinterpret_cast<gg::Tile*>(take(static_cast<size_t>(w.max_dn) * sizeof(gg::Tile)));
+  w.n_tiles = reinterpret_cast<int*>(take(2 * 4));
+  w.err = reinterpret_cast<int*>(take(4));
+  w.bytes = off;
+  return w;
+}
+
+bool gemm_path(const moe_layer* L, int T, int K) {
+  return static_cast<long long>(T) * K >= kGemmMinSlots && L->H % gg::BM == 0 && (2 * L->I) % gg::BM == 0 &&
+         L->I % gg::BK == 0;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// Row-major fp16 matrix [rows][cols] as a TMA source of [128 rows x 64 cols] boxes, 128-byte swizzle.
+bool token_map(CUtensorMap* m, const uint16_t* X, int cols, int rows) {
+  const EncodeTiledFn f = encode_tiled();
+  if (!f) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(gg::BK), static_cast<cuuint32_t>(gg::BN)};
+  const cuuint32_t estr[2] = {1, 1};
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(X), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int H>
+moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int K, const int32_t* idx, const float* w,
+                               void* out, int out_mode, int32_t* perm_out, void* workspace, cudaStream_t st) {
+  const int E = L->E, I = L->I, TK = T * K, R = TK + T;
+  const bool lora = L->r > 0 && L->sh_lora_A[0];
+  const int r = L->r > 0 ? L->r : 0;
+  const GWs ws = carve_gemm(workspace, T, K, E, H, I, L->r);
+  if (cudaMemsetAsync(ws.err, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+  pf::bucket_count_kernel<<<ws.nblk, pf::kChunk, 0, st>>>(idx, TK, E, ws.idx, ws.blockhist);
+  pf::bucket_scan_kernel<<<1, 256, 0, st>>>(ws.nblk, E, ws.blockhist, ws.count, ws.offset);
+  pf::bucket_place_kernel<<<ws.nblk, pf::kChunk, 0, st>>>(ws.idx, TK, E, ws.blockhist, ws.perm, ws.inv, perm_out);
+  pf::permute_kernel<<<R, 256, 0, st>>>(u, T, K, H, ws.perm, w, ws.X, ws.w_pos);
+  pf::tile_list_kernel<<<1, 288, 0, st>>>(ws.count, ws.offset, E, T, K, 2 * I / gg::BM, H / gg::BM, ws.tiles_gu,
+                                          ws.tiles_dn, ws.n_tiles);
+  // The GEMMs trust the device-built tile list: stop here if any launch so far failed.
+  if (launch_status() != MOE_OK) return MOE_ERR_CUDA;
+  {
+    const int nrows = 1 + (lora ? 2 * r : 0);
+    const size_t smem = gemv_smem(H, false, true);
+    allow_smem(pf::lora_a_tokens_kernel<H / 8>, smem);
+    dim3 grid((T + TB - 1) / TB, (nrows + kWarps - 1) / kWarps);
+    pf::lora_a_tokens_kernel<H / 8><<<grid, kThreads, smem, st>>>(
+        u, T, TK, r, static_cast<const uint8_t*>(L->shared_gate.rows), lora ? L->sh_lora_A[0] : nullptr,
+        lora ? L->sh_lora_A[1] : nullptr, ws.g, ws.t1, ws.t2);
+  }
+  CUtensorMap mx, mh;
+  if (!token_map(&mx, ws.X, H, R) || !token_map(&mh, ws.Hh, I, R)) return MOE_ERR_CUDA;
+  const int RGU = qrow_bytes(H, 4), RDN = qrow_bytes(I, 4);
+  auto base_args = [&]() {
+    gg::Args a{};
+    a.n_tiles = ws.n_tiles;
+    a.pool = static_cast<const uint8_t*>(L->pool);
+    a.stride = L->expert_stride;
+    a.shared_block = static_cast<const uint8_t*>(L->shared_block);
+    a.E = E;
+    a.lora_r = r;
+    a.lora_scale = L->lora_scale;
+    a.err = ws.err;
+    a.timeout_ns = 2000000000LL;
+    return a;
+  };
+  if (cudaFuncSetAttribute(gg::grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gg::SMEM_BYTES) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  {  // gate/up + SwiGLU for every bucket and the shared expert
+    gg::Args a = base_args();
+    a.tiles = ws.tiles_gu;
+    a.K = H;
+    a.a_off = 0;
+    a.a_rec = RGU;
+    a.epi = gg::EPI_SWIGLU;
+    a.out = ws.Hh;
+    a.out_ld = I;
+    if (lora) {
+      a.lora_B1 = L->sh_lora_B[0];
+      a.lora_t1 = ws.t1;
+      a.lora_B2 = L->sh_lora_B[1];
+      a.lora_t2 = ws.t2;
+    }
+    gg::grouped_gemm_kernel<<<ws.max_gu, gg::kThreads, gg::SMEM_BYTES, st>>>(mx, a);
+  }
+  const bool ex = r > 0 && L->ex_lora_A;
+  if (lora || ex) {  // LoRA A products on the SwiGLU output (shared down, routed down)
+    const int row_begin = ex ? 0 : TK, nrows = ex ? (lora ? R : TK) : T;
+    pf::lora_a_rows_kernel<<<(nrows * r + kWarps - 1) / kWarps, kThreads, 0, st>>>(
+        ws.Hh, I, TK, nrows, row_begin, r, lora ? L->sh_lora_A[2] : nullptr, ex ? L->ex_lora_A : nullptr, ws.idx,
+        ws.perm, ws.t1);
+  }
+  {  // down (+ LoRA), routed rows scaled by their gating weight
+    gg::Args a = base_args();
+    a.tiles = ws.tiles_dn;
+    a.n_tiles = ws.n_tiles + 1;
+    a.K = I;
+    a.a_off = static_cast<int64_t>(2 * I) * RGU;
+    a.a_rec = RDN;
+    a.epi = gg::EPI_DOWN;
+    a.out = ws.Y;
+    a.out_ld = H;
+    a.row_scale = ws.w_pos;
+    a.lora_B1 = lora ? L->sh_lora_B[2] : nullptr;
+    a.lora_t1 = ws.t1;
+    a.lora_Bex = ex ? L->ex_lora_B : nullptr;
+    gg::grouped_gemm_kernel<<<ws.max_dn, gg::kThreads, gg::SMEM_BYTES, st>>>(mh, a);
+  }
+  pf::combine_kernel<<<T, 256, 0, st>>>(ws.Y, T, K, H, ws.inv, ws.g, out, out_mode);
+  return launch_status();
+}
+
 template <int H>
 moe_status expert_forward_h(const moe_layer* L, const uint16_t* u, int T, int K, const int32_t* idx, const float* w,
                             void* out, int out_mode, int32_t* perm_out, const Ws& ws, cudaStream_t st) {
+  if (gemm_path(L, T, K)) return expert_forward_gemm<H>(L, u, T, K, idx, w, out, out_mode, perm_out, ws.base, st);
   switch (L->I) {
     case 128: return expert_forward_hi<H, 128>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
     case 256: return expert_forward_hi<H, 256>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
@@ -280,9 +455,18 @@ moe_status moe_route_topk(const moe_layer* L, const uint16_t* u, int32_t T, int3
   }
 }
 
+static size_t ws_bytes_for(const moe_layer* L, int T, int K) {
+  size_t b = carve(nullptr, T, K, L->E, L->I, L->r).bytes;
+  if (gemm_path(L, T, K)) {
+    const size_t g = carve_gemm(nullptr, T, K, L->E, L->H, L->I, L->r).bytes;
+    if (g > b) b = g;
+  }
+  return b;
+}
+
 size_t moe_workspace_size(const moe_layer* L, int32_t T, int32_t K) {
   if (!L || T < 0 || K < 1) return 0;
-  return carve(nullptr, T, K, L->E, L->I, L->r).bytes;
+  return ws_bytes_for(L, T, K);
 }
 
 moe_status moe_expert_forward(const moe_layer* L, const uint16_t* u, int32_t T, int32_t K, const int32_t* idx,
@@ -306,9 +490,8 @@ moe_status moe_expert_forward(const moe_layer* L, const uint16_t* u, int32_t T, 
     for (const void* p : lp)
       if (p && !aligned(p, 16)) return MOE_ERR_INVALID_ARG;
   }
-  const Ws need = carve(nullptr, T, K, L->E, L->I, L->r);
   if (!workspace || !aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
-  if (ws_bytes < need.bytes) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < ws_bytes_for(L, T, K)) return MOE_ERR_WORKSPACE;
   const Ws ws = carve(workspace, T, K, L->E, L->I, L->r);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (L->H) {

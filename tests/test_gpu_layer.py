@@ -381,3 +381,62 @@ def test_full_size_stack_sampled_layers(cuda_ok, cfg_id):
     sample = [0, 1, cfg.layers // 2, cfg.layers - 1]
     needed = {l: sorted(set(res["idx"][l].reshape(-1).tolist())) for l in sample}
     _check_stack(cfg, lambda l: inputs.layer(cfg, l, experts=needed[l]), T, res, x0, sample)
+
+
+# ----------------------------------------------------------------------------- many-token (tensor-core) path
+@pytest.mark.parametrize("T", [64, 200])
+@pytest.mark.parametrize("routed_lora", [False, True])
+def test_expert_forward_grouped_gemm_small(cuda_ok, T, routed_lora):
+    """T*K >= 128 slots take the tcgen05 grouped-GEMM path; same definition as the decode path."""
+    _grouped_gemm_case(dataclasses.replace(CONFIGS[0], lora_routed_down=routed_lora), T)
+
+
+# (H, I): gate/up and down with different m-tile counts; K/64 above the pipeline depth of 4
+@pytest.mark.parametrize("H,I", [(256, 256), (512, 128), (1024, 512)])
+def test_expert_forward_grouped_gemm_shapes(cuda_ok, H, I):
+    _grouped_gemm_case(dataclasses.replace(CONFIGS[0], H=H, I=I, I_s=I, lora_routed_down=True), 96)
+
+
+def _grouped_gemm_case(cfg, T):
+    lay = Layer(cfg, 0)
+    ub = inputs.activations(cfg, step=500 + T, T=T)
+    u = u_vals(ub)
+    logits = O.router_logits(u, lay.host["router"])
+    idx = O.topk(logits, cfg.K)
+    w = O.gating(logits, idx)
+    out, perm = expert_forward(lay, ub, cfg.K, idx, w, perm=True)
+    assert np.array_equal(perm, O.buckets(idx, cfg.E)["perm"])
+    assert_close_inf(out, oracle_out(lay, u, idx, w))
+    x0 = np.random.default_rng(T).standard_normal((T, cfg.H))
+    out2, _ = expert_forward(lay, ub, cfg.K, idx, w, mode=2, x0=x0)
+    assert_close_inf(out2 - x0.astype(np.float32), oracle_out(lay, u, idx, w))
+
+
+def test_expert_forward_grouped_gemm_skewed_buckets(cuda_ok):
+    """One expert takes most slots (several 128-token tiles), others one or none."""
+    cfg = CONFIGS[0]
+    lay = Layer(cfg, 0)
+    T = 300
+    ub = inputs.activations(cfg, step=77, T=T)
+    u = u_vals(ub)
+    rng = np.random.default_rng(5)
+    idx = np.stack([[3, int(rng.integers(4, 16))] if t % 7 else [int(rng.integers(0, 3)), 3] for t in range(T)])
+    w = rng.dirichlet([1, 1], size=T)
+    out, perm = expert_forward(lay, ub, cfg.K, idx, w, perm=True)
+    assert np.array_equal(perm, O.buckets(idx, cfg.E)["perm"])
+    assert_close_inf(out, oracle_out(lay, u, idx, w))
+
+
+def test_expert_forward_grouped_gemm_full_size_layer(cuda_ok):
+    """35B-shaped prefill layer (Zipf-offset router) on 512 tokens, sampled tokens checked."""
+    cfg = CONFIGS[3]
+    lay = Layer(cfg, 1)
+    T = 512
+    ub = inputs.activations(cfg, step=9, T=T)
+    u = u_vals(ub)
+    logits, idx, w = route(lay, ub, cfg.K)
+    out, perm = expert_forward(lay, ub, cfg.K, idx, w, perm=True)
+    assert np.array_equal(perm, O.buckets(idx, cfg.E)["perm"])
+    sample = np.arange(0, T, 37)
+    ref = oracle_out(lay, u[sample], idx[sample], w[sample])
+    assert_close_inf(out[sample], ref)
