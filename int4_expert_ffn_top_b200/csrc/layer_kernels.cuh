@@ -705,31 +705,59 @@ __global__ void __launch_bounds__(kThreads) prerouter_w1_kernel(PreW1Args a) {
   }
 }
 
-// scores[t][e] = W2[e] . z[t] + b2[e]; z fp32, W2 fp16 widened to fp32.  One row per warp.
+// Second Prerouter layer: scores[t][e] = b2[e] + sum_p W2[e][p] * z[t][p].
+// A CTA takes 32 tokens x 32 rows; z of its tokens is staged in shared memory
+// 256 inputs at a time (rows padded by one float against bank conflicts); lane
+// = token, each warp 4 rows, whose W2 values are warp-uniform (broadcast) loads.
+constexpr int kW2Tok = 32, kW2Rows = 32, kW2Chunk = 256;
 __global__ void __launch_bounds__(kThreads) prerouter_w2_kernel(const float* __restrict__ z, int T, int P,
                                                                 const uint16_t* __restrict__ W2,
                                                                 const uint16_t* __restrict__ b2, int En,
                                                                 float* __restrict__ scores) {
+  __shared__ float zs[kW2Tok * (kW2Chunk + 1)];
+  const int t0 = blockIdx.y * kW2Tok, e0 = blockIdx.x * kW2Rows;
+  const int nt = min(kW2Tok, T - t0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e = blockIdx.x * kWarps + warp;
-  if (e >= En) return;
-  const uint16_t* row = W2 + static_cast<size_t>(e) * P;
-  const float b = half_bits_to_float(b2[e]);
-  for (int t = 0; t < T; ++t) {
-    const float* zt = z + static_cast<size_t>(t) * P;
-    float acc = 0.f;
-    for (int c = lane; c < P / 8; c += 32) {
-      const uint4 w = ldg_stream(reinterpret_cast<const uint4*>(row) + c);
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+  constexpr int RPW = kW2Rows / kWarps;  // rows per warp
+  float acc[RPW];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const float2 f = __half22float2(as_h2(ws[m]));
-        acc = fmaf(f.x, zt[c * 8 + 2 * m], acc);
-        acc = fmaf(f.y, zt[c * 8 + 2 * m + 1], acc);
+  for (int j = 0; j < RPW; ++j) acc[j] = 0.f;
+  for (int p0 = 0; p0 < P; p0 += kW2Chunk) {
+    const int pc = min(kW2Chunk, P - p0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < kW2Tok * pc; i += blockDim.x) {
+      const int tt = i / pc, pp = i - tt * pc;
+      zs[tt * (kW2Chunk + 1) + pp] = tt < nt ? z[static_cast<size_t>(t0 + tt) * P + p0 + pp] : 0.f;
+    }
+    __syncthreads();
+    const float* zr = zs + lane * (kW2Chunk + 1);
+#pragma unroll 1
+    for (int pp = 0; pp < pc; pp += 8) {
+      float zv[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) zv[m] = zr[pp + m];
+#pragma unroll
+      for (int j = 0; j < RPW; ++j) {
+        const int e = e0 + warp * RPW + j;
+        if (e < En) {
+          const uint4 w = *reinterpret_cast<const uint4*>(W2 + static_cast<size_t>(e) * P + p0 + pp);
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const float2 f = __half22float2(as_h2(ws[m]));
+            acc[j] = fmaf(f.x, zv[2 * m], acc[j]);
+            acc[j] = fmaf(f.y, zv[2 * m + 1], acc[j]);
+          }
+        }
       }
     }
-    acc = warp_reduce(acc);
-    if (lane == 0) scores[static_cast<size_t>(t) * En + e] = acc + b;
+  }
+  if (lane < nt) {
+#pragma unroll
+    for (int j = 0; j < RPW; ++j) {
+      const int e = e0 + warp * RPW + j;
+      if (e < En) scores[static_cast<size_t>(t0 + lane) * En + e] = acc[j] + half_bits_to_float(b2[e]);
+    }
   }
 }
 

@@ -394,8 +394,8 @@ moe_status prerouter_h(const moe_prerouter* P, const uint16_t* u, const int32_t*
   allow_smem(prerouter_w1_kernel<H / 8>, smem);
   dim3 g1((P->P + kWarps - 1) / kWarps, (T + TB - 1) / TB);
   prerouter_w1_kernel<H / 8><<<g1, kThreads, smem, st>>>(a);
-  prerouter_w2_kernel<<<(P->E_next + kWarps - 1) / kWarps, kThreads, 0, st>>>(z, T, P->P, P->W2, P->b2, P->E_next,
-                                                                               scores);
+  dim3 g2((P->E_next + kW2Rows - 1) / kW2Rows, (T + kW2Tok - 1) / kW2Tok);
+  prerouter_w2_kernel<<<g2, kThreads, 0, st>>>(z, T, P->P, P->W2, P->b2, P->E_next, scores);
   topk_kernel<<<(T + kWarps - 1) / kWarps, kThreads, 0, st>>>(scores, T, P->E_next, K_next, pred, nullptr);
   return launch_status();
 }
@@ -738,7 +738,7 @@ StackWs carve_stack(void* base, const moe_layer* L0, const moe_prerouter* P0, in
   w.pred1 = reinterpret_cast<int32_t*>(take(static_cast<size_t>(T) * K_next * 4));
   w.err = reinterpret_cast<int32_t*>(take(4));
   w.ll = reinterpret_cast<unsigned long long*>(take(ll_bytes));
-  w.ews_bytes = carve(nullptr, T, K, L0->E, L0->I, L0->r).bytes;
+  w.ews_bytes = ws_bytes_for(L0, T, K);
   w.ews = take(w.ews_bytes);
   w.pws_bytes = P0 ? prerouter_ws(P0, T) : 0;
   w.pws = take(w.pws_bytes);
