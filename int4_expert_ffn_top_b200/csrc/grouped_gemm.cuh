@@ -5,7 +5,7 @@
 // weight rows never are).
 //
 // Per CTA one tile: 128 weight rows x up to 128 tokens, K in steps of 64 (one
-// quantisation group per step), 4-stage shared-memory pipeline:
+// quantisation group per step), 2-stage shared-memory pipeline:
 //  * warps 0-3 dequantise the int4 row records of the tile (w = q*s + b, one
 //    fp16 rounding) straight into the 128-byte-swizzled K-major layout the MMA
 //    reads, one row per thread;
@@ -28,7 +28,11 @@ namespace gg {
 constexpr int BM = 128;
 constexpr int BN = 128;
 constexpr int BK = 64;
-constexpr int STAGES = 4;
+// Two stages keep a CTA at 66 KB of shared memory, so two CTAs share an SM:
+// twice the dequantising warps in flight per SM, which the weight stream needs
+// more than a deeper per-CTA pipeline (one layer's expert forward at 3,328
+// tokens: 1.53 ms with four stages and one CTA per SM, 0.98 ms with this).
+constexpr int STAGES = 2;
 constexpr int kThreads = 192;
 constexpr int A_STAGE = BM * BK * 2;  // 16 KB
 constexpr int B_STAGE = BN * BK * 2;  // 16 KB
