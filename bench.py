@@ -56,6 +56,21 @@ def token_layer_bytes(cfg) -> int:
     return cfg.K * blk + shared + lora + router + sgate + pre
 
 
+def max_over_ranks(v: float, dist, device) -> float:
+    """The largest of every rank's value (the whole job waits for the slowest replica)."""
+    if dist is None:
+        return v
+    import torch
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms: float) -> float:
+    """Units per second processed by all ranks together over the (max-over-ranks) time ms."""
+    return units_per_rank * world / (ms / 1000.0)
+
+
 def expert_flops(cfg, T: int) -> float:
     """Algorithmic tensor-core work of one layer's experts: T*K routed slots and T shared-expert rows,
     each 2*(2I*H) for gate/up plus 2*(H*I) for down."""
@@ -336,11 +351,8 @@ def main():
         raise RuntimeError(f"device-side wait timed out (status {int(err.item())})")
     if dist is not None:
         dist.barrier()
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    tokens_total = T * args.steps * world
-    value = tokens_total / (ms / 1000.0)
+    ms = max_over_ranks(ms, dist, dev)
+    value = whole_job_rate(T * args.steps, world, ms)
 
     # end to end through the public API with host buffers: H2D of the token, D2H of the result
     xh = torch.from_numpy(toks).pin_memory()
@@ -361,11 +373,8 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize(dev)
     ms_e2e = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([ms_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
-    e2e_value = T * e2e_steps * world / (ms_e2e / 1000.0)
+    ms_e2e = max_over_ranks(ms_e2e, dist, dev)
+    e2e_value = whole_job_rate(T * e2e_steps, world, ms_e2e)
 
     peak, peak_kind = peaks()
     bytes_step = token_layer_bytes(cfg) * cfg.layers * T
@@ -393,11 +402,8 @@ def main():
         del stack, st, ws, xpool
         torch.cuda.empty_cache()
         pre = prefill_leg(dev, M)
-        if dist is not None:
-            t = torch.tensor([pre["ms_per_pass"]], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            pre["ms_per_pass"] = float(t.item())
-            pre["value"] = CONFIGS[PREFILL_CFG_ID].T * world / (pre["ms_per_pass"] / 1000.0)
+        pre["ms_per_pass"] = max_over_ranks(pre["ms_per_pass"], dist, dev)
+        pre["value"] = whole_job_rate(CONFIGS[PREFILL_CFG_ID].T, world, pre["ms_per_pass"])
         out["prefill"] = pre
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(cfg)
