@@ -30,6 +30,8 @@ from gen import CONFIGS, inputs  # noqa: E402
 METRIC = "MoE-stack decode tok/s (35B-shape, bs=1) & HBM GB/s vs peak; prefill tok/s"
 CFG_ID = 1
 PREFILL_CFG_ID = 3
+DECODE_8B_CFG_ID = 2
+BATCHED_CFG_ID = 4
 EPS = 1e-6
 N_TOKENS = 64  # distinct tokens cycled through the steps
 
@@ -154,6 +156,105 @@ def prefill_leg(dev, M, passes: int = 5):
                                         "scope": "every kernel of one layer's moe_expert_forward (the two grouped "
                                                  "GEMMs dominate), timed alone"}},
     }
+
+
+def decode_leg(dev, M, cfg_id: int, steps: int):
+    """Batch-1 decode of another stack shape (per token: all layers, one launch when eligible)."""
+    import torch
+    cfg = CONFIGS[cfg_id]
+    stack = M.DeviceStack(cfg, lambda l: inputs.layer(cfg, l), device=dev)
+    st = M.StackStructs(stack)
+    ws = M.workspace(M.moe_stack_workspace_size(st, 1, cfg.K, cfg.K), device=dev)
+    xs = torch.from_numpy(np.stack([inputs.bf16_bits_to_f32(inputs.activations(cfg, step=1 + i, T=1))
+                                    for i in range(N_TOKENS)])).to(dev)
+    x = torch.empty((1, cfg.H), device=dev)
+    err = torch.zeros((1,), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        x.copy_(xs[i % N_TOKENS])
+        M.moe_stack_decode(st, x, cfg.K, cfg.K, EPS, ws, err_word=err)
+
+    for i in range(10):
+        step(i)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device-side wait timed out (status {int(err.item())})")
+    ms = e0.elapsed_time(e1) / steps
+    del stack, st, ws
+    torch.cuda.empty_cache()
+    peak, kind = peaks()
+    bytes_tok = token_layer_bytes(cfg) * cfg.layers
+    gbs = bytes_tok / (ms / 1000.0) / 1e9
+    return {"workload": f"{cfg.name}: {cfg.layers} layers, {cfg.E} experts, top-{cfg.K}, H {cfg.H}, I {cfg.I}, batch 1",
+            "value": 1000.0 / ms, "unit": "tok/s", "ms_per_token": ms, "steps": steps,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "peak_kind": kind, "algorithmic_bytes_per_token": bytes_tok}}
+
+
+def batched_decode_leg(dev, M, steps: int = 20):
+    """35B-shaped batched decode: 64 tokens per step, layers >= 1 executing the previous head's prediction,
+    LoRA on every routed down projection.  Reports tok/s, the bytes of the experts actually touched per step
+    over the step time, and the Prerouter hit rate (|pred_{l-1} & true_l| / K)."""
+    import torch
+    cfg = CONFIGS[BATCHED_CFG_ID]
+    T, K = cfg.T, cfg.K
+    stack = M.DeviceStack(cfg, lambda l: inputs.layer(cfg, l), device=dev)
+    st = M.StackStructs(stack)
+    ws = M.workspace(M.moe_stack_workspace_size(st, T, K, K), device=dev)
+    x0 = torch.from_numpy(inputs.bf16_bits_to_f32(inputs.activations(cfg, step=5, T=T))).to(dev)
+    x = torch.empty_like(x0)
+    err = torch.zeros((1,), dtype=torch.int32, device=dev)
+    n = cfg.layers
+    idx_all = torch.full((n, T, K), -1, dtype=torch.int32, device=dev)
+    true_all = torch.full((n, T, K), -1, dtype=torch.int32, device=dev)
+    pred_all = torch.full((n, T, K), -1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(trace):
+        x.copy_(x0)
+        kw = dict(idx_all=idx_all, true_idx_all=true_all, pred_all=pred_all) if trace else {}
+        M.moe_stack_decode(st, x, K, K, EPS, ws, use_predicted_routing=True, err_word=err, **kw)
+
+    step(True)
+    torch.cuda.synchronize(dev)
+    idx_h, true_h, pred_h = idx_all.cpu().numpy(), true_all.cpu().numpy(), pred_all.cpu().numpy()
+    for _ in range(3):
+        step(False)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step(False)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device-side wait timed out (status {int(err.item())})")
+    ms = e0.elapsed_time(e1) / steps
+    del stack, st, ws
+    torch.cuda.empty_cache()
+    hits = [np.mean([len(set(pred_h[l - 1, t]) & set(true_h[l, t])) / K for t in range(T)]) for l in range(1, n)]
+    touched = [len(np.unique(idx_h[l])) for l in range(n)]
+    mat = lambda out, inp: out * (inp // 2 + 4 * (inp // 64))
+    blk = mat(2 * cfg.I, cfg.H) + mat(cfg.H, cfg.I)
+    down_lora = cfg.r * cfg.I * 2 + cfg.H * cfg.r * 2
+    per_layer_fixed = token_layer_bytes(cfg) - K * blk  # shared expert, its LoRA, router, gate, Prerouter
+    step_bytes = sum(t * (blk + down_lora) for t in touched) + n * per_layer_fixed
+    peak, kind = peaks()
+    gbs = step_bytes / (ms / 1000.0) / 1e9
+    return {"workload": "35B-shaped batched decode: 64 tokens per step, 40 layers, predicted routing for layers >= 1, "
+                        "LoRA r16 on every routed down projection",
+            "value": T / (ms / 1000.0), "unit": "tok/s", "ms_per_step": ms, "steps": steps,
+            "touched_experts_per_layer": float(np.mean(touched)), "prerouter_hit_rate": float(np.mean(hits)),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "peak_kind": kind, "bytes_per_step": step_bytes,
+                         "scope": "whole step; bytes = experts touched (with their down LoRA) + per-layer fixed weights"}}
 
 
 def launches_per_step(cfg, single: bool, predicted=False) -> int:
@@ -288,6 +389,7 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the 3,328-token prefill leg")
+    ap.add_argument("--no-extra", action="store_true", help="skip the 8B-shaped and batched decode legs")
     ap.add_argument("--path", type=int, default=0, help="0 auto, 1 per-layer launches, 2 single launch")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -405,6 +507,19 @@ def main():
         pre["ms_per_pass"] = max_over_ranks(pre["ms_per_pass"], dist, dev)
         pre["value"] = whole_job_rate(CONFIGS[PREFILL_CFG_ID].T, world, pre["ms_per_pass"])
         out["prefill"] = pre
+    if not args.no_extra:
+        for key, fn in (("decode_8b", lambda: decode_leg(dev, M, DECODE_8B_CFG_ID, steps=500)),
+                        ("batched_decode", lambda: batched_decode_leg(dev, M))):
+            try:
+                leg = fn()
+                ms_leg = leg.get("ms_per_token", leg.get("ms_per_step"))
+            except Exception as exc:  # a failing extra leg must not lose the headline line
+                leg, ms_leg = {"error": f"{type(exc).__name__}: {exc}"}, -1.0
+            # every rank takes this collective, on the error path too
+            ms_leg = max_over_ranks(ms_leg, dist, dev)
+            if "error" not in leg:
+                leg["ms_max_over_ranks"] = ms_leg
+            out[key] = leg
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(cfg)
     if rank == 0:

@@ -383,6 +383,23 @@ def test_full_size_stack_sampled_layers(cuda_ok, cfg_id):
     _check_stack(cfg, lambda l: inputs.layer(cfg, l, experts=needed[l]), T, res, x0, sample)
 
 
+@pytest.mark.slow
+def test_batched_decode_stack_with_predicted_routing(cuda_ok):
+    """35B-shaped stack at 64 tokens per step: layers >= 1 execute the previous head's prediction, every
+    routed expert carries a down-projection LoRA; the experts take the grouped-GEMM path (64*4 slots)."""
+    cfg = CONFIGS[4]
+    stack = M().DeviceStack(cfg, lambda l: inputs.layer(cfg, l))
+    T = cfg.T
+    x0 = inputs.bf16_bits_to_f32(inputs.activations(cfg, step=123, T=T))
+    res = run_stack(stack, cfg, T, x0, True)
+    assert res["err"] == 0
+    del stack
+    torch.cuda.empty_cache()
+    sample = [0, 1, cfg.layers // 2, cfg.layers - 1]
+    needed = {l: sorted(set(res["idx"][l].reshape(-1).tolist())) for l in sample}
+    _check_stack(cfg, lambda l: inputs.layer(cfg, l, experts=needed[l]), T, res, x0, sample)
+
+
 # ----------------------------------------------------------------------------- many-token (tensor-core) path
 @pytest.mark.parametrize("T", [64, 200])
 @pytest.mark.parametrize("routed_lora", [False, True])
