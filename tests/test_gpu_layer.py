@@ -400,6 +400,41 @@ def test_batched_decode_stack_with_predicted_routing(cuda_ok):
     _check_stack(cfg, lambda l: inputs.layer(cfg, l, experts=needed[l]), T, res, x0, sample)
 
 
+@pytest.mark.slow
+def test_prefill_stack_full_size_sampled(cuda_ok):
+    """35B-shaped prefill exactly as the benchmark runs it: 3,328 tokens through all 40 layers (per-layer
+    launches, grouped-GEMM experts), checked on sampled layers for every 52nd token."""
+    cfg = CONFIGS[3]
+    stack = M().DeviceStack(cfg, lambda l: inputs.layer(cfg, l))
+    T = cfg.T
+    x0 = inputs.bf16_bits_to_f32(inputs.activations(cfg, step=1, T=T))
+    res = run_stack(stack, cfg, T, x0, False, opts=M().stack_opts(path=M().PATH_LAYERS))
+    assert res["err"] == 0
+    del stack
+    torch.cuda.empty_cache()
+    toks = np.arange(0, T, 52)
+    sub = {k: (v[:, toks] if k in ("x_trace", "u_trace", "idx", "true_idx", "pred") else v[toks]) for k, v in res.items()
+           if k != "err"}
+    sample = [0, 1, cfg.layers // 2, cfg.layers - 1]
+    needed = {l: sorted(set(sub["idx"][l].reshape(-1).tolist())) for l in sample}
+    _check_stack(cfg, lambda l: inputs.layer(cfg, l, experts=needed[l]), len(toks), sub, x0[toks], sample)
+
+
+# Largest supported shapes (H 4096, I 2048) on both expert paths: 4 tokens (GEMV), 64 tokens (grouped GEMM).
+@pytest.mark.parametrize("T", [4, 64])
+def test_expert_forward_max_shapes(cuda_ok, T):
+    cfg = dataclasses.replace(CONFIGS[0], H=4096, I=2048, I_s=2048, r=32, lora_routed_down=True)
+    lay = Layer(cfg, 0)
+    ub = inputs.activations(cfg, step=31 + T, T=T)
+    u = u_vals(ub)
+    logits = O.router_logits(u, lay.host["router"])
+    idx = O.topk(logits, cfg.K)
+    w = O.gating(logits, idx)
+    out, perm = expert_forward(lay, ub, cfg.K, idx, w, perm=True)
+    assert np.array_equal(perm, O.buckets(idx, cfg.E)["perm"])
+    assert_close_inf(out, oracle_out(lay, u, idx, w))
+
+
 # ----------------------------------------------------------------------------- many-token (tensor-core) path
 @pytest.mark.parametrize("T", [64, 200])
 @pytest.mark.parametrize("routed_lora", [False, True])
