@@ -397,11 +397,16 @@ def test_planted_mistakes_are_caught(monkeypatch):
         "top-k tie to higher index": lambda: monkeypatch.setattr(
             O, "topk", lambda s, K: np.stack([np.lexsort((-np.arange(s.shape[1]), -row))[:K] for row in s])),
         "silu sign flipped": lambda: monkeypatch.setattr(O, "sigmoid", lambda a: 0.5 * (1.0 - np.tanh(0.5 * a))),
+        "predicted routing ignored": lambda: monkeypatch.setattr(
+            O, "layer_forward", lambda u, L, K, routing=None, K_next=None, _f=O.layer_forward: _f(u, L, K, None, K_next)),
+        "layer input not rounded to bf16": lambda: monkeypatch.setattr(
+            O, "layer_input", lambda x, eps=1e-6: O.rmsnorm(x, eps)),
     }
     pins = [test_hand_built_words, lambda: test_dequant_exhaustive_codes_exact(4), test_dequant_group_boundaries,
             test_expert_ffn_closed_form_on_selection_weights, test_topk_brute_force_with_ties,
             test_topk_all_equal_gives_lowest_indices, test_activation_closed_forms,
-            test_router_closed_form_on_one_hot_weights]
+            test_router_closed_form_on_one_hot_weights, test_stack_forward_with_zero_experts_keeps_the_residual,
+            test_stack_forward_predicted_routing_executes_the_previous_prediction]
     for name, plant in planted.items():
         plant()
         failed = False
@@ -413,3 +418,53 @@ def test_planted_mistakes_are_caught(monkeypatch):
                 break
         monkeypatch.undo()
         assert failed, f"no pin caught: {name}"
+
+
+# ----------------------------------------------------------------------------- stack glue and predicted routing
+def _zeroed_layer(cfg, l):
+    """A c0-shaped layer whose routed experts, shared expert and LoRA deltas are all exactly zero."""
+    L = inputs.layer(cfg, l)
+    for m in [*(ex[k] for ex in L["experts"].values() for k in ("gate_up", "down")),
+              L["shared"]["gate_up"], L["shared"]["down"]]:
+        m["s"] = np.zeros_like(m["s"])
+        m["b"] = np.zeros_like(m["b"])
+    for k in ("lora_gate", "lora_up", "lora_down"):
+        if L["shared"].get(k):
+            L["shared"][k]["B"] = np.zeros_like(L["shared"][k]["B"])
+    return L
+
+
+def test_stack_forward_with_zero_experts_keeps_the_residual():
+    """x_{l+1} = x_l + MoE_l(...) with every expert weight zero: x never changes, so every layer sees
+    the same normed input bf16(rmsnorm(x0))."""
+    cfg = CONFIGS[0]
+    x0 = np.random.default_rng(3).standard_normal((cfg.T, cfg.H))
+    res = O.stack_forward(x0, [_zeroed_layer(cfg, l) for l in range(3)], cfg.K)
+    assert np.array_equal(res["x"], x0)
+    u0 = O.round_bf16(O.rmsnorm(x0))
+    for tr in res["trace"]:
+        assert np.array_equal(tr["u"], u0)
+
+
+def test_stack_forward_predicted_routing_executes_the_previous_prediction():
+    """With zero Prerouter weights the prediction is the ranking of b2 (a permutation here); with
+    predicted routing every layer after the first executes exactly that prediction, layer 0 its own top-K."""
+    cfg = CONFIGS[0]
+    rng = np.random.default_rng(11)
+    b2 = rng.permutation(cfg.E).astype(np.float16)
+    want = list(np.argsort(-b2.astype(float), kind="stable")[:cfg.K])
+    layers = []
+    for l in range(3):
+        L = inputs.layer(cfg, l)
+        hd = L["prerouter"]
+        L["prerouter"] = dict(W1=np.zeros_like(hd["W1"]), b1=np.zeros_like(hd["b1"]),
+                              W2=np.zeros_like(hd["W2"]), b2=b2)
+        layers.append(L)
+    x0 = rng.standard_normal((cfg.T, cfg.H))
+    res = O.stack_forward(x0, layers, cfg.K, predicted_routing=True)
+    tr = res["trace"]
+    assert np.array_equal(tr[0]["idx"], tr[0]["true_idx"])
+    for l in range(3):
+        assert all(list(tr[l]["pred"][t]) == want for t in range(cfg.T))
+    for l in (1, 2):
+        assert all(list(tr[l]["idx"][t]) == want for t in range(cfg.T))
