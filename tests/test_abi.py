@@ -99,3 +99,13 @@ def test_workspace_sizes_grow_with_tokens(lib):
     assert 0 < a < b and a % 256 == 0 and b % 256 == 0
     # h for (T*K + T) slots x I fp16 dominates
     assert b >= (64 * 4 + 64) * 512 * 2
+
+
+def test_stack_probe_tool_parses_its_arguments():
+    """The profiling/tracing driver named in profiles/ is importable and parses its options without a GPU."""
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, "-m", "int4_expert_ffn_top_b200.stack_probe", "--help"],
+                       cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))), capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0 and "--trace" in r.stdout
