@@ -109,3 +109,37 @@ def test_stack_probe_tool_parses_its_arguments():
                        cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))), capture_output=True, text=True,
                        timeout=300)
     assert r.returncode == 0 and "--trace" in r.stdout
+
+
+def test_expert_block_layout_decodes_back_to_the_expert():
+    """The HBM expert block: gate/up records interleaved (gate_j, up_j), then down records; each record is
+    codes (nibble k at bits 4(k%2) of byte k/2), then in/64 fp16 scales, then in/64 fp16 biases."""
+    import numpy as np
+
+    from gen import CONFIGS, inputs
+    from int4_expert_ffn_top_b200.weights import expert_block, qrow_bytes
+    from oracle import moe_oracle as O
+
+    cfg = CONFIGS[0]
+    ex = inputs.layer(cfg, 0, experts=[5])["experts"][5]
+    blk = expert_block(ex)
+    H, I = cfg.H, cfg.I
+
+    def decode(rec, in_dim):
+        cb, G = in_dim // 2, in_dim // 64
+        q = np.empty(in_dim)
+        q[0::2], q[1::2] = rec[:cb] & 15, rec[:cb] >> 4
+        s = rec[cb:cb + 2 * G].view(np.float16).astype(np.float64)
+        b = rec[cb + 2 * G:cb + 4 * G].view(np.float16).astype(np.float64)
+        return q * np.repeat(s, 64) + np.repeat(b, 64)
+
+    rgu, rdn = qrow_bytes(H, 4), qrow_bytes(I, 4)
+    assert blk.size == 2 * I * rgu + H * rdn
+    gu = O.dequant(ex["gate_up"])
+    dn = O.dequant(ex["down"])
+    for j in (0, 1, I // 2, I - 1):
+        assert np.array_equal(decode(blk[(2 * j) * rgu:(2 * j + 1) * rgu], H), gu[j])          # gate row j
+        assert np.array_equal(decode(blk[(2 * j + 1) * rgu:(2 * j + 2) * rgu], H), gu[I + j])  # up row j
+    off = 2 * I * rgu
+    for o in (0, 7, H - 1):
+        assert np.array_equal(decode(blk[off + o * rdn:off + (o + 1) * rdn], I), dn[o])
