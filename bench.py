@@ -335,48 +335,130 @@ def measured_traffic(layers: int):
         return None
 
 
+class OracleTokenPass:
+    """Batch-1 tokens through the stack on the float64 oracle, one work item at a time.
+
+    A layer is K + 3 items, taken in the order of the oracle's own layer pass:
+    ``route`` (layer input, router logits, top-K, gating weights), ``expert``
+    once per routed slot, ``shared`` (shared expert and its sigmoid gate) and
+    ``tail`` (weighted combine, residual add, Prerouter prediction).  Every item
+    calls the oracle's functions as they stand; ``step`` returns the item's kind
+    and its seconds of oracle work.  Inputs are drawn outside the clock: each
+    layer's router, shared expert and Prerouter once (then kept), and per layer
+    only the experts the token is routed to.  After the last layer the next
+    token (a new seeded activation) starts at layer 0.
+    """
+
+    KINDS = ("route", "expert", "shared", "tail")
+
+    def __init__(self, cfg, eps: float = EPS):
+        from oracle import moe_oracle as O
+        self.O, self.cfg, self.eps = O, cfg, eps
+        self.static = {}
+        self.token, self.layer, self.i = 0, 0, 0
+        self.finished = []  # residual streams of completed tokens
+        self._new_token()
+
+    def _new_token(self):
+        self.x = inputs.bf16_bits_to_f32(inputs.activations(self.cfg, step=self.token, T=1)).astype(np.float64)
+
+    def _layer_static(self, l: int):
+        if l not in self.static:
+            self.static[l] = (inputs.router(self.cfg, l), inputs.shared(self.cfg, l), inputs.prerouter(self.cfg, l))
+        return self.static[l]
+
+    def step(self) -> tuple[str, float]:
+        O, cfg, K = self.O, self.cfg, self.cfg.K
+        R, S, P = self._layer_static(self.layer)
+        i = self.i
+        if i == 0:
+            kind, t0 = "route", time.perf_counter()
+            self.u = O.layer_input(self.x, self.eps)
+            logits = O.router_logits(self.u, R)
+            self.idx = O.topk(logits, K)
+            self.w = O.gating(logits, self.idx)
+            dt = time.perf_counter() - t0
+            self.experts = {int(e): inputs.expert(cfg, self.layer, int(e)) for e in self.idx[0]}
+            self.y = np.zeros((1, K, cfg.H), dtype=np.float64)
+        elif i <= K:
+            kind, t0 = "expert", time.perf_counter()
+            self.y[:, i - 1] = O.routed_outputs(self.u, self.experts, self.idx[:, i - 1:i])[:, 0]
+            dt = time.perf_counter() - t0
+        elif i == K + 1:
+            kind, t0 = "shared", time.perf_counter()
+            self.ys = O.shared_expert(self.u, S)
+            self.g = O.shared_gate(self.u, S)
+            dt = time.perf_counter() - t0
+        else:
+            kind, t0 = "tail", time.perf_counter()
+            self.x = self.x + O.combine(self.w, self.y, self.g, self.ys)
+            self.pred = O.prerouter_predict(self.u, self.idx, P, cfg.E, K)[0]
+            dt = time.perf_counter() - t0
+        self.i += 1
+        if self.i == K + 3:
+            self.i, self.layer = 0, self.layer + 1
+            if self.layer == cfg.layers:
+                self.finished.append(self.x)
+                self.token, self.layer = self.token + 1, 0
+                self._new_token()
+        return kind, dt
+
+
+def oracle_token_seconds(items, cfg) -> float:
+    """Oracle seconds per token from timed items: per-kind means times the items of a token.
+
+    With every kind sampled a token costs ``layers * (t_route + K t_expert +
+    t_shared + t_tail)``; otherwise the plain item rate is scaled by the
+    ``layers * (K + 3)`` items of a token.
+    """
+    per_layer = {"route": 1, "expert": cfg.K, "shared": 1, "tail": 1}
+    by = {k: [t for kind, t in items if kind == k] for k in per_layer}
+    if all(by.values()):
+        return cfg.layers * sum(n * statistics.fmean(by[k]) for k, n in per_layer.items())
+    return sum(t for _, t in items) * cfg.layers * (cfg.K + 3) / len(items)
+
+
 def cpu_baseline(cfg, budget_s: float = 20.0):
-    """The float64 oracle on the host: tokens through the stack, layer by layer, bounded by a time budget."""
-    from oracle import moe_oracle as O
+    """The float64 oracle on the host: whole layers of one token until the time budget is spent."""
     cores = len(os.sched_getaffinity(0))
-    x = inputs.bf16_bits_to_f32(inputs.activations(cfg, step=0, T=1)).astype(np.float64)
-    t_oracle, layers_done = 0.0, 0
-    for l in range(cfg.layers):
-        L = inputs.layer(cfg, l)  # input generation: not timed
-        t0 = time.perf_counter()
-        u = O.layer_input(x, EPS)
-        r = O.layer_forward(u, L, cfg.K)
-        x = x + r["out"]
-        t_oracle += time.perf_counter() - t0
-        layers_done += 1
-        del L
-        if t_oracle > budget_s:
-            break
-    per_token = t_oracle * cfg.layers / layers_done
-    return {"value": 1.0 / per_token, "unit": "tok/s", "cores": cores, "kind": "oracle",
-            "sample": f"1 token through {layers_done} of {cfg.layers} layers of the 35B-shaped stack "
-                      f"(float64 numpy, BLAS threads = {cores}), scaled to {cfg.layers} layers"}
+    ref = OracleTokenPass(cfg)
+    items = []
+    while sum(t for _, t in items) < budget_s or ref.i != 0:
+        items.append(ref.step())
+    layers = len(items) // (cfg.K + 3)
+    return {"value": 1.0 / oracle_token_seconds(items, cfg), "unit": "tok/s", "cores": cores, "kind": "oracle",
+            "sample": f"{layers} layer passes of batch-1 tokens through the 35B-shaped stack (float64 numpy, "
+                      f"BLAS threads = {cores}), seconds per token = {cfg.layers} x one layer's items"}
+
+
+def decode_config(cfg, world: int) -> dict:
+    return {"workload": "35B-shaped MoE stack decode, batch 1 (40 layers, 256 experts, top-4, H 2048, "
+                        "I 512, shared expert I 512 + LoRA r16, Prerouter P 256)",
+            "tokens_per_step": cfg.T, "layers": cfg.layers, "parallelism": f"replicas x{world}"}
 
 
 def run_reference(args, rank, world):
+    """The oracle timed on the host cores (rank 0 only): each step is one oracle work item."""
     if rank != 0:
         return
     cfg = CONFIGS[CFG_ID]
-    vals = []
+    ref = OracleTokenPass(cfg)
     for _ in range(args.warmup):
-        pass  # the oracle has no warm state; warm-up steps are not repeated
-    for _ in range(args.steps):
-        vals.append(cpu_baseline(cfg, budget_s=max(5.0, 150.0 / max(args.steps, 1))))
-    v = statistics.median(x["value"] for x in vals)
-    cb = dict(vals[0])
-    cb["value"] = v
+        ref.step()
+    items = [ref.step() for _ in range(args.steps)]
+    v = 1.0 / oracle_token_seconds(items, cfg)
+    cores = len(os.sched_getaffinity(0))
+    sample = (f"{args.steps} oracle work items (route / one routed expert / shared expert / combine + Prerouter; "
+              f"{cfg.K + 3} per layer, {cfg.layers} layers per token) of batch-1 tokens, after {args.warmup} "
+              f"warm-up items; float64 numpy, BLAS threads = {cores}")
+    config = decode_config(cfg, world)
+    config["step"] = "one oracle work item of a token's pass (a bounded sample of the decode step)"
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tok/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / v, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "35B-shaped MoE stack decode, batch 1 (40 layers, 256 experts, top-4, H 2048)",
-                   "tokens_per_step": 1, "layers": cfg.layers},
-        "cpu_baseline": cb,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * sum(t for _, t in items) / len(items),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config,
+        "cpu_baseline": {"value": v, "unit": "tok/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": v, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 
@@ -485,9 +567,7 @@ def main():
         "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "35B-shaped MoE stack decode, batch 1 (40 layers, 256 experts, top-4, H 2048, "
-                               "I 512, shared expert I 512 + LoRA r16, Prerouter P 256)",
-                   "tokens_per_step": T, "layers": cfg.layers, "parallelism": f"replicas x{world}",
+        "config": {**decode_config(cfg, world),
                    "l2": "inputs larger than L2: 433 MB of weights read per step, a distinct token per step",
                    "path": "moe_stack_decode, " + ("one cooperative launch per token" if single
                                                      else "per-layer launches")},

@@ -41,3 +41,52 @@ def test_prefill_expert_flops_per_layer():
     routed = T * K * (2 * (2 * I) * H + 2 * H * I)
     shared = T * (2 * (2 * I) * H + 2 * H * I)
     assert bench.expert_flops(CONFIGS[3], T) == routed + shared == 104_689_827_840
+
+
+def _small_decode_cfg():
+    import dataclasses
+
+    return dataclasses.replace(CONFIGS[0], T=1, layers=3, lora_routed_down=True)
+
+
+def test_oracle_work_items_reproduce_the_oracle_stack_pass():
+    """The reference arm's item-by-item pass is the oracle's own stack pass, bit for bit."""
+    import numpy as np
+
+    from gen import inputs
+    from oracle import moe_oracle as O
+
+    cfg = _small_decode_cfg()
+    ref = bench.OracleTokenPass(cfg)
+    kinds = [ref.step()[0] for _ in range(2 * cfg.layers * (cfg.K + 3))]
+    assert kinds[:cfg.K + 3] == ["route"] + ["expert"] * cfg.K + ["shared", "tail"]
+    assert len(ref.finished) == 2 and ref.token == 2 and ref.layer == 0 and ref.i == 0
+    layers = [inputs.layer(cfg, l) for l in range(cfg.layers)]
+    for tok in range(2):
+        x0 = inputs.bf16_bits_to_f32(inputs.activations(cfg, step=tok, T=1)).astype(np.float64)
+        want = O.stack_forward(x0, layers, cfg.K, eps=bench.EPS)["x"]
+        assert np.array_equal(ref.finished[tok], want)
+
+
+def test_oracle_token_seconds_weights_each_kind_by_its_count():
+    cfg = _small_decode_cfg()  # K = 2: a layer is route + 2 experts + shared + tail
+    items = [("route", 1.0), ("expert", 2.0), ("expert", 4.0), ("shared", 3.0), ("tail", 0.5), ("route", 3.0)]
+    assert bench.oracle_token_seconds(items, cfg) == cfg.layers * (2.0 + 2 * 3.0 + 3.0 + 0.5)
+    part = [("route", 1.0), ("expert", 3.0)]  # not every kind sampled: plain item rate
+    assert bench.oracle_token_seconds(part, cfg) == 4.0 * cfg.layers * (cfg.K + 3) / 2
+
+
+def test_reference_arm_prints_one_line_in_the_native_arms_terms(capsys):
+    import json
+
+    class Args:
+        steps, warmup = 8, 1
+
+    bench.run_reference(Args, 0, 1)
+    line = json.loads(capsys.readouterr().out.strip())
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["unit"] == "tok/s"
+    assert line["steps"] == 8 and line["higher_is_better"] is True and line["value"] > 0
+    assert line["e2e"] == {"value": line["value"], "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    native = bench.decode_config(CONFIGS[bench.CFG_ID], 1)
+    assert {k: line["config"][k] for k in native} == native
