@@ -418,17 +418,38 @@ def oracle_token_seconds(items, cfg) -> float:
     return sum(t for _, t in items) * cfg.layers * (cfg.K + 3) / len(items)
 
 
-def cpu_baseline(cfg, budget_s: float = 20.0):
-    """The float64 oracle on the host: whole layers of one token until the time budget is spent."""
-    cores = len(os.sched_getaffinity(0))
+def blas_threads() -> int:
+    """Threads of the host BLAS pool the oracle's matmuls run on (the largest pool if several)."""
+    from threadpoolctl import threadpool_info
+    return max((p["num_threads"] for p in threadpool_info() if p.get("user_api") == "blas"), default=1)
+
+
+def _oracle_layers(cfg, budget_s: float):
     ref = OracleTokenPass(cfg)
     items = []
-    while sum(t for _, t in items) < budget_s or ref.i != 0:
+    while not items or ref.i != 0 or sum(t for _, t in items) < budget_s:
         items.append(ref.step())
-    layers = len(items) // (cfg.K + 3)
-    return {"value": 1.0 / oracle_token_seconds(items, cfg), "unit": "tok/s", "cores": cores, "kind": "oracle",
-            "sample": f"{layers} layer passes of batch-1 tokens through the 35B-shaped stack (float64 numpy, "
-                      f"BLAS threads = {cores}), seconds per token = {cfg.layers} x one layer's items"}
+    return items
+
+
+def cpu_baseline(cfg, budget_s: float = 20.0, one_thread_budget_s: float = 10.0):
+    """The float64 oracle on the host: whole layers of batch-1 tokens until each time budget is spent.
+
+    The headline figure uses every BLAS thread of the process; a second sample
+    with the BLAS pool limited to one thread is reported beside it.
+    """
+    from threadpoolctl import threadpool_limits
+    cores = blas_threads()
+    items = _oracle_layers(cfg, budget_s)
+    out = {"value": 1.0 / oracle_token_seconds(items, cfg), "unit": "tok/s", "cores": cores, "kind": "oracle",
+           "sample": f"{len(items) // (cfg.K + 3)} layer passes of batch-1 tokens through the 35B-shaped stack "
+                     f"(float64 numpy, BLAS threads = {cores}), seconds per token = {cfg.layers} x one layer's items"}
+    if one_thread_budget_s > 0:
+        with threadpool_limits(limits=1, user_api="blas"):
+            one = _oracle_layers(cfg, one_thread_budget_s)
+        out["one_thread"] = {"value": 1.0 / oracle_token_seconds(one, cfg), "unit": "tok/s", "cores": 1,
+                             "sample": f"{len(one) // (cfg.K + 3)} layer passes, BLAS threads = 1"}
+    return out
 
 
 def decode_config(cfg, world: int) -> dict:
@@ -447,7 +468,7 @@ def run_reference(args, rank, world):
         ref.step()
     items = [ref.step() for _ in range(args.steps)]
     v = 1.0 / oracle_token_seconds(items, cfg)
-    cores = len(os.sched_getaffinity(0))
+    cores = blas_threads()
     sample = (f"{args.steps} oracle work items (route / one routed expert / shared expert / combine + Prerouter; "
               f"{cfg.K + 3} per layer, {cfg.layers} layers per token) of batch-1 tokens, after {args.warmup} "
               f"warm-up items; float64 numpy, BLAS threads = {cores}")

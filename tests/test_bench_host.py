@@ -90,3 +90,12 @@ def test_reference_arm_prints_one_line_in_the_native_arms_terms(capsys):
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     native = bench.decode_config(CONFIGS[bench.CFG_ID], 1)
     assert {k: line["config"][k] for k in native} == native
+
+
+def test_cpu_baseline_runs_whole_layers():
+    cb = bench.cpu_baseline(CONFIGS[bench.CFG_ID], budget_s=0.0, one_thread_budget_s=1e-9)  # one layer each
+    assert cb["kind"] == "oracle" and cb["unit"] == "tok/s" and cb["value"] > 0 and cb["cores"] >= 1
+    assert cb["sample"].startswith("1 layer passes")
+    assert cb["one_thread"]["cores"] == 1 and cb["one_thread"]["value"] > 0
+    assert cb["one_thread"]["sample"].startswith("1 layer passes")
+    assert bench.blas_threads() == cb["cores"]  # the limit is lifted again afterwards
