@@ -41,7 +41,8 @@
  *     is one contiguous span (one bulk copy / one coalesced warp read).
  * Supported shapes: H a power of two in [256, 4096], I a power of two in
  *   [128, 2048], I_s == I, 1 <= K <= 8, K <= E <= 256, LoRA rank r <= 32,
- *   Prerouter E % 8 == 0 and P % 8 == 0.
+ *   Prerouter E % 8 == 0 and P % 8 == 0, 0 <= T <= MOE_MAX_TOKENS tokens per
+ *   call.
  */
 #ifndef MOE_H
 #define MOE_H
@@ -52,6 +53,11 @@
 #ifdef __cplusplus
 extern "C" {
 #endif
+
+/* Most tokens one call takes: the GEMV kernels walk tokens in passes of 8,
+ * one grid row per pass, and a grid has at most 65,535 rows.  A larger T
+ * returns MOE_ERR_UNSUPPORTED (workspace queries return 0). */
+#define MOE_MAX_TOKENS 524280
 
 typedef enum {
   MOE_OK = 0,

@@ -37,6 +37,51 @@ def _p(t) -> int | None:
     return None if t is None else t.data_ptr()
 
 
+# Tensors that hold bf16 values may be typed bf16 or carry the bits as a 16-bit integer.
+BF16_BITS = tuple(d for d in (torch.bfloat16, torch.int16, getattr(torch, "uint16", None)) if d is not None)
+F32, I32, I64 = (torch.float32,), (torch.int32,), (torch.int64,)
+
+
+def _arg(fn: str, name: str, t, dtypes, numel: int = 0, optional: bool = False) -> int | None:
+    """Address of a tensor argument after checking it can be handed to the library.
+
+    The library reads and writes device memory through the raw address, so a
+    host tensor, a strided view, a wrong element type or a buffer smaller than
+    the call touches is refused here, before any launch.
+    """
+    if t is None:
+        if optional:
+            return None
+        raise ValueError(f"{fn}: {name} is required")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{fn}: {name} must be a torch.Tensor, got {type(t).__name__}")
+    if t.device.type != "cuda":
+        raise ValueError(f"{fn}: {name} must be a CUDA tensor, got one on {t.device}")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise ValueError(f"{fn}: {name} has dtype {t.dtype}, expected {' or '.join(str(d) for d in dtypes)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{fn}: {name} must be contiguous")
+    if t.numel() < numel:
+        raise ValueError(f"{fn}: {name} holds {t.numel()} elements, the call needs {numel}")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{fn}: {name} is on {t.device}, the current device is cuda:{torch.cuda.current_device()}")
+    return t.data_ptr()
+
+
+def _rows(fn: str, name: str, t, width: int, dtypes) -> int:
+    """Row count of a 2-D ``[T, width]`` tensor argument (checked like :func:`_arg`)."""
+    if not isinstance(t, torch.Tensor) or t.dim() != 2 or t.shape[1] != width:
+        shape = tuple(t.shape) if isinstance(t, torch.Tensor) else type(t).__name__
+        raise ValueError(f"{fn}: {name} must be [T, {width}], got {shape}")
+    _arg(fn, name, t, dtypes)
+    return t.shape[0]
+
+
+def _ws(fn: str, t) -> tuple[int, int]:
+    """Address and byte size of a workspace tensor (its size is checked by the library)."""
+    return _arg(fn, "workspace", t, None), t.numel() * t.element_size()
+
+
 def _check(fn: str, code: int):
     if code != _lib.MOE_OK:
         raise MoEError(fn, code)
@@ -55,28 +100,41 @@ def moe_expert_block_bytes(H: int, I: int) -> int:
 
 
 def moe_rmsnorm_bf16(x: torch.Tensor, eps: float, u: torch.Tensor, stream=None):
+    fn = "moe_rmsnorm_bf16"
+    if not isinstance(x, torch.Tensor) or x.dim() != 2:
+        raise ValueError(f"{fn}: x must be [T, H]")
     T, H = x.shape
-    _check("moe_rmsnorm_bf16", lib().moe_rmsnorm_bf16(_p(x), T, H, eps, _p(u), _stream(stream)))
+    px, pu = _arg(fn, "x", x, F32), _arg(fn, "u", u, BF16_BITS, T * H)
+    _check(fn, lib().moe_rmsnorm_bf16(px, T, H, eps, pu, _stream(stream)))
 
 
 def moe_route_topk(layer: DeviceLayer, u: torch.Tensor, K: int, logits: torch.Tensor, idx: torch.Tensor,
                    w: torch.Tensor, stream=None):
-    T = u.shape[0]
-    _check("moe_route_topk", lib().moe_route_topk(ctypes.byref(layer.struct), _p(u), T, K, _p(logits), _p(idx),
-                                                  _p(w), _stream(stream)))
+    fn, L = "moe_route_topk", layer.struct
+    T = _rows(fn, "u", u, L.H, BF16_BITS)
+    args = (_arg(fn, "logits", logits, F32, T * L.E), _arg(fn, "idx", idx, I32, T * K), _arg(fn, "w", w, F32, T * K))
+    _check(fn, lib().moe_route_topk(ctypes.byref(L), _p(u), T, K, *args, _stream(stream)))
 
 
 def moe_workspace_size(layer: DeviceLayer, T: int, K: int) -> int:
     return lib().moe_workspace_size(ctypes.byref(layer.struct), T, K)
 
 
+def _expert_args(fn: str, layer: DeviceLayer, u, K: int, idx, w, out, out_mode: int, perm_out):
+    L = layer.struct
+    T = _rows(fn, "u", u, L.H, BF16_BITS)
+    out_types = BF16_BITS if out_mode == OUT_BF16 else F32
+    return T, (_arg(fn, "idx", idx, I32, T * K), _arg(fn, "w", w, F32, T * K), _arg(fn, "out", out, out_types, T * L.H),
+               out_mode, _arg(fn, "perm_out", perm_out, I32, T * K, optional=True))
+
+
 def moe_expert_forward(layer: DeviceLayer, u: torch.Tensor, K: int, idx: torch.Tensor, w: torch.Tensor,
                        out: torch.Tensor, out_mode: int, workspace: torch.Tensor, perm_out: torch.Tensor | None = None,
                        stream=None):
-    T = u.shape[0]
-    _check("moe_expert_forward", lib().moe_expert_forward(
-        ctypes.byref(layer.struct), _p(u), T, K, _p(idx), _p(w), _p(out), out_mode, _p(perm_out), _p(workspace),
-        workspace.numel() * workspace.element_size(), _stream(stream)))
+    fn = "moe_expert_forward"
+    T, args = _expert_args(fn, layer, u, K, idx, w, out, out_mode, perm_out)
+    _check(fn, lib().moe_expert_forward(ctypes.byref(layer.struct), _p(u), T, K, *args, *_ws(fn, workspace),
+                                        _stream(stream)))
 
 
 def moe_noalloc_scratch_bytes() -> int:
@@ -91,9 +149,9 @@ def moe_expert_forward_noalloc(layer: DeviceLayer, u: torch.Tensor, K: int, idx:
     calls that overlap on the GPU race; the first call on a device should come
     before any stream capture on it.
     """
-    T = u.shape[0]
-    _check("moe_expert_forward_noalloc", lib().moe_expert_forward_noalloc(
-        ctypes.byref(layer.struct), _p(u), T, K, _p(idx), _p(w), _p(out), out_mode, _p(perm_out), _stream(stream)))
+    fn = "moe_expert_forward_noalloc"
+    T, args = _expert_args(fn, layer, u, K, idx, w, out, out_mode, perm_out)
+    _check(fn, lib().moe_expert_forward_noalloc(ctypes.byref(layer.struct), _p(u), T, K, *args, _stream(stream)))
 
 
 def prerouter_workspace_size(head: DeviceHead, T: int) -> int:
@@ -102,16 +160,24 @@ def prerouter_workspace_size(head: DeviceHead, T: int) -> int:
 
 def prerouter_predict(head: DeviceHead, u: torch.Tensor, sel: torch.Tensor, K_next: int, pred: torch.Tensor,
                       scores: torch.Tensor, workspace: torch.Tensor, stream=None):
+    fn, P = "prerouter_predict", head.struct
+    if not isinstance(sel, torch.Tensor) or sel.dim() != 2:
+        raise ValueError(f"{fn}: sel must be [T, K]")
     T, K = sel.shape
-    _check("prerouter_predict", lib().prerouter_predict(
-        ctypes.byref(head.struct), _p(u), _p(sel), T, K, K_next, _p(pred), _p(scores), _p(workspace),
-        workspace.numel() * workspace.element_size(), _stream(stream)))
+    if _rows(fn, "u", u, P.H, BF16_BITS) != T:
+        raise ValueError(f"{fn}: u has {u.shape[0]} rows, sel has {T}")
+    args = (_arg(fn, "sel", sel, I32), K_next, _arg(fn, "pred", pred, I32, T * K_next),
+            _arg(fn, "scores", scores, F32, T * P.E_next))
+    _check(fn, lib().prerouter_predict(ctypes.byref(P), _p(u), args[0], T, K, *args[1:], *_ws(fn, workspace),
+                                       _stream(stream)))
 
 
 class StackStructs:
     """Contiguous host arrays of ``moe_layer`` / ``moe_prerouter`` structs for the stack entry points."""
 
     def __init__(self, layers, heads=None):
+        # The structs hold raw device addresses: keep the tensors behind them alive as long as this object.
+        self._owners = (layers, heads)
         if isinstance(layers, DeviceStack):
             self.n, self.layers, self.heads = layers.n, layers.layer_array, layers.head_array
             return
@@ -132,8 +198,15 @@ PATH_AUTO, PATH_LAYERS, PATH_SINGLE = 0, 1, 2
 
 def stack_opts(timeout_ns: int = 0, path: int = PATH_AUTO, drop_layer: int = -1, drop_cta: int = -1,
                trace: torch.Tensor | None = None):
-    """moe_stack_opts; drop_layer/drop_cta (>= 0) arm the timeout-path test hook; trace: int64 device tensor."""
-    return _lib.moe_stack_opts(timeout_ns, path, drop_layer + 1 if drop_layer >= 0 else 0, drop_cta, _p(trace))
+    """moe_stack_opts; drop_layer/drop_cta (>= 0) arm the timeout-path test hook.
+
+    ``trace``: int64 device tensor of ``n_layers * moe_stack_grid() * 16`` stamps
+    (checked against the stack when the options are used).
+    """
+    o = _lib.moe_stack_opts(timeout_ns, path, drop_layer + 1 if drop_layer >= 0 else 0, drop_cta,
+                            _arg("stack_opts", "trace", trace, I64, optional=True))
+    o.trace_tensor = trace  # keeps the buffer alive and lets moe_stack_decode check its size
+    return o
 
 
 def moe_stack_grid() -> int:
@@ -143,12 +216,22 @@ def moe_stack_grid() -> int:
 def moe_stack_decode(stack: StackStructs, x: torch.Tensor, K: int, K_next: int, eps: float, workspace: torch.Tensor,
                      x_trace=None, u_trace=None, idx_all=None, true_idx_all=None, pred_all=None,
                      use_predicted_routing=False, err_word=None, opts=None, stream=None):
-    T = x.shape[0]
-    _check("moe_stack_decode", lib().moe_stack_decode(
-        stack.layers, stack.heads_ptr(), stack.n, T, K, K_next, eps, _p(x), _p(x_trace), _p(u_trace), _p(idx_all),
-        _p(true_idx_all), _p(pred_all), int(bool(use_predicted_routing)), _p(err_word),
-        None if opts is None else ctypes.byref(opts), _p(workspace), workspace.numel() * workspace.element_size(),
-        _stream(stream)))
+    fn, n, H = "moe_stack_decode", stack.n, stack.layers[0].H
+    T = _rows(fn, "x", x, H, F32)
+    ptrs = (_arg(fn, "x_trace", x_trace, F32, n * T * H, optional=True),
+            _arg(fn, "u_trace", u_trace, BF16_BITS, n * T * H, optional=True),
+            _arg(fn, "idx_all", idx_all, I32, n * T * K, optional=True),
+            _arg(fn, "true_idx_all", true_idx_all, I32, n * T * K, optional=True),
+            _arg(fn, "pred_all", pred_all, I32, n * T * K_next, optional=True))
+    err = _arg(fn, "err_word", err_word, I32, 1, optional=True)
+    trace = getattr(opts, "trace_tensor", None) if opts is not None else None
+    if trace is not None:
+        _arg(fn, "opts.trace", trace, I64, n * moe_stack_grid() * 16)
+    elif opts is not None and opts.trace:
+        raise ValueError(f"{fn}: opts.trace was set without a tensor; build the options with stack_opts()")
+    _check(fn, lib().moe_stack_decode(
+        stack.layers, stack.heads_ptr(), n, T, K, K_next, eps, _p(x), *ptrs, int(bool(use_predicted_routing)), err,
+        None if opts is None else ctypes.byref(opts), *_ws(fn, workspace), _stream(stream)))
 
 
 def workspace(nbytes: int, device="cuda") -> torch.Tensor:

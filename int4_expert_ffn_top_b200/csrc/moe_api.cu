@@ -34,7 +34,7 @@ bool qrows_ok(const moe_qrows& m, int out_dim, int in_dim, int bits) {
 
 moe_status check_layer(const moe_layer* L, int T, int K) {
   if (!L) return MOE_ERR_INVALID_ARG;
-  if (T < 0 || K < 1 || K > 8) return MOE_ERR_UNSUPPORTED;
+  if (T < 0 || T > MOE_MAX_TOKENS || K < 1 || K > 8) return MOE_ERR_UNSUPPORTED;
   if (!h_ok(L->H) || !i_ok(L->I) || L->I_s != L->I) return MOE_ERR_UNSUPPORTED;
   if (L->E < K || L->E > 256 || L->r < 0 || L->r > 32) return MOE_ERR_UNSUPPORTED;
   if (!qrows_ok(L->router, L->E, L->H, 8)) return MOE_ERR_INVALID_ARG;
@@ -465,7 +465,7 @@ static size_t ws_bytes_for(const moe_layer* L, int T, int K) {
 }
 
 size_t moe_workspace_size(const moe_layer* L, int32_t T, int32_t K) {
-  if (!L || T < 0 || K < 1) return 0;
+  if (!L || T < 0 || T > MOE_MAX_TOKENS || K < 1) return 0;
   return ws_bytes_for(L, T, K);
 }
 
@@ -505,7 +505,7 @@ moe_status moe_expert_forward(const moe_layer* L, const uint16_t* u, int32_t T, 
 }
 
 size_t prerouter_workspace_size(const moe_prerouter* head, int32_t T) {
-  if (!head || T < 0) return 0;
+  if (!head || T < 0 || T > MOE_MAX_TOKENS) return 0;
   return prerouter_ws(head, T);
 }
 
@@ -513,7 +513,7 @@ moe_status prerouter_predict(const moe_prerouter* head, const uint16_t* u, const
                              int32_t K_next, int32_t* pred, float* scores, void* workspace, size_t ws_bytes,
                              void* stream) {
   if (!head) return MOE_ERR_INVALID_ARG;
-  if (T < 0 || K < 1 || K > 8 || K_next < 1 || K_next > 8) return MOE_ERR_UNSUPPORTED;
+  if (T < 0 || T > MOE_MAX_TOKENS || K < 1 || K > 8 || K_next < 1 || K_next > 8) return MOE_ERR_UNSUPPORTED;
   if (!h_ok(head->H) || head->E < K || head->E > 256 || head->E % 8 || head->E_next < K_next ||
       head->E_next > 256 || head->P < 8 || head->P % 8)
     return MOE_ERR_UNSUPPORTED;
@@ -766,7 +766,7 @@ int32_t moe_stack_grid(void) {
 
 size_t moe_stack_workspace_size(const moe_layer* layers, const moe_prerouter* heads, int32_t n_layers, int32_t T,
                                 int32_t K, int32_t K_next) {
-  if (!layers || n_layers < 1 || T < 0 || K < 1) return 0;
+  if (!layers || n_layers < 1 || T < 0 || T > MOE_MAX_TOKENS || K < 1) return 0;
   return carve_stack(nullptr, &layers[0], heads, T, K, K_next, ll_bound(&layers[0], heads, K, n_layers)).bytes;
 }
 

@@ -90,6 +90,28 @@ def test_host_side_rejections(lib):
                                 None, 0, None) == _lib.MOE_ERR_INVALID_ARG
 
 
+def test_token_limit_is_rejected_on_the_host(lib):
+    import re as _re
+
+    from int4_expert_ffn_top_b200 import _lib
+    hdr = open(os.path.join(ROOT, "include", "moe.h")).read()
+    assert int(_re.search(r"#define MOE_MAX_TOKENS (\d+)", hdr).group(1)) == _lib.MOE_MAX_TOKENS == 65535 * 8
+    L = _lib.moe_layer()
+    L.H, L.E, L.I, L.I_s, L.r = 2048, 256, 512, 512, 16
+    big = _lib.MOE_MAX_TOKENS + 1
+    assert lib.moe_route_topk(ctypes.byref(L), None, big, 4, None, None, None, None) == _lib.MOE_ERR_UNSUPPORTED
+    assert lib.moe_expert_forward(ctypes.byref(L), None, big, 4, None, None, None, 0, None, None, 0,
+                                  None) == _lib.MOE_ERR_UNSUPPORTED
+    assert lib.moe_workspace_size(ctypes.byref(L), big, 4) == 0
+    assert lib.moe_workspace_size(ctypes.byref(L), _lib.MOE_MAX_TOKENS, 4) > 0
+    P = _lib.moe_prerouter()
+    P.H, P.E, P.P, P.E_next = 2048, 256, 256, 256
+    assert lib.prerouter_predict(ctypes.byref(P), None, None, big, 4, 4, None, None, None, 0,
+                                 None) == _lib.MOE_ERR_UNSUPPORTED
+    assert lib.prerouter_workspace_size(ctypes.byref(P), big) == 0
+    assert lib.moe_stack_workspace_size(ctypes.byref(L), None, 1, big, 4, 4) == 0
+
+
 def test_workspace_sizes_grow_with_tokens(lib):
     from int4_expert_ffn_top_b200 import _lib
     L = _lib.moe_layer()
