@@ -152,7 +152,8 @@ moe_status moe_route_topk(const moe_layer* L, const uint16_t* u, int32_t T, int3
  *   for expert e = idx[t][k]; shared expert likewise with its LoRA deltas;
  *   g_t = sigmoid(shared_gate . u_t);
  *   out_t = sum_{k=0}^{K-1} w[t][k] y_{t,k} + g_t y_shared,t   (k order fixed)
- * u [T][H] bf16; idx [T][K] int32 in [0,E); w [T][K] fp32.
+ * u [T][H] bf16; idx [T][K] int32 in [0,E) (a value outside is clamped to
+ *   0 or E-1, so no read leaves the pool); w [T][K] fp32.
  * out_mode 0: out [T][H] fp32 = result;  1: out [T][H] bf16 = result;
  *          2: out [T][H] fp32 += result (residual stream).
  * perm_out: if not NULL, receives the expert-sorted slot order [T*K] int32
@@ -177,7 +178,9 @@ size_t moe_workspace_size(const moe_layer* L, int32_t T, int32_t K);
 
 /*
  * Prerouter prediction (see moe_prerouter).  u [T][H] bf16; sel [T][K] int32
- * = experts executed at this layer; pred [T][K_next] int32 (same ordering and
+ * = experts executed at this layer, distinct within a row (each entry adds its
+ * W1 column once, so distinct entries give the multi-hot product; a value
+ * outside [0,E) is clamped to 0 or E-1); pred [T][K_next] int32 (same ordering and
  * tie rule as moe_route_topk); scores [T][E_next] fp32 (required output, the
  * p vector); workspace >= prerouter_workspace_size(head, T) bytes.
  */
