@@ -264,6 +264,17 @@ def launches_per_step(cfg, single: bool, predicted=False) -> int:
     return cfg.layers * per_layer + (cfg.layers - 1 if predicted else 0)
 
 
+def smi_gpu_id(local: int) -> str:
+    """nvidia-smi ``--id`` of this process's CUDA device ``local``.
+
+    CUDA_VISIBLE_DEVICES renumbers devices for CUDA but not for nvidia-smi, so
+    its ``local``-th entry (an index or a GPU UUID) names the GPU; without it
+    the CUDA index is the nvidia-smi index.
+    """
+    vis = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    return vis[local] if local < len(vis) else str(local)
+
+
 class Clocks:
     """nvidia-smi samples (SM clock, throttle reasons), started before the warm-up so that
     its start-up does not fall in the timed region; samples are kept by their own timestamp."""
@@ -273,7 +284,7 @@ class Clocks:
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+        self.gpu = smi_gpu_id(gpu_index)
         self.proc = None
         self.lines = []
         self.window = None

@@ -99,3 +99,13 @@ def test_cpu_baseline_runs_whole_layers():
     assert cb["one_thread"]["cores"] == 1 and cb["one_thread"]["value"] > 0
     assert cb["one_thread"]["sample"].startswith("1 layer passes")
     assert bench.blas_threads() == cb["cores"]  # the limit is lifted again afterwards
+
+
+def test_clock_sampler_names_the_visible_gpu(monkeypatch):
+    monkeypatch.delenv("CUDA_VISIBLE_DEVICES", raising=False)
+    assert bench.smi_gpu_id(3) == "3"
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "4,6")
+    assert bench.smi_gpu_id(0) == "4" and bench.smi_gpu_id(1) == "6"
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "GPU-0a1b, GPU-2c3d")
+    assert bench.smi_gpu_id(1) == "GPU-2c3d"
+    assert bench.Clocks(0).gpu == "GPU-0a1b"
