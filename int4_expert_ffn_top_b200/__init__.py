@@ -182,6 +182,10 @@ class StackStructs:
             self.n, self.layers, self.heads = layers.n, layers.layer_array, layers.head_array
             return
         self.n = len(layers)
+        if self.n == 0:
+            raise ValueError("StackStructs: a stack needs at least one layer")
+        if heads is not None and len(heads) != self.n:
+            raise ValueError(f"StackStructs: {len(heads)} Prerouter heads for {self.n} layers")
         self.layers = (_lib.moe_layer * self.n)(*[l.struct for l in layers])
         self.heads = None if heads is None else (_lib.moe_prerouter * self.n)(*[h.struct for h in heads])
 

@@ -175,3 +175,12 @@ def test_stack_structs_keep_the_device_tensors_alive():
     del layer
     assert ref() is not None and st.n == 1
     assert isinstance(st.layers, ctypes.Array)
+
+
+def test_stack_structs_refuse_an_empty_stack_or_mismatched_heads():
+    with pytest.raises(ValueError, match="at least one layer"):
+        M.StackStructs([])
+    with pytest.raises(ValueError, match="heads"):
+        M.StackStructs([FakeLayer(), FakeLayer()], [FakeHead()])
+    st = M.StackStructs([FakeLayer()], [FakeHead()])
+    assert st.heads_ptr() is not None
