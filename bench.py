@@ -154,7 +154,12 @@ def prefill_leg(dev, M, passes: int = 5):
                            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                                         "frac": achieved / peak, "peak_kind": peak_kind,
                                         "scope": "every kernel of one layer's moe_expert_forward (the two grouped "
-                                                 "GEMMs dominate), timed alone"}},
+                                                 "GEMMs dominate), timed alone",
+                                        "traffic": None,
+                                        "traffic_note": "DRAM bytes were captured for the gate/up grouped GEMM at "
+                                                        "512 tokens only (profiles/grouped_gemm_35b_prefill_512tok_"
+                                                        "full.md); its weight bytes do not grow with tokens, so no "
+                                                        "full-size figure is scaled from it"}},
     }
 
 
