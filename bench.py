@@ -269,6 +269,38 @@ def launches_per_step(cfg, single: bool, predicted=False) -> int:
     return cfg.layers * per_layer + (cfg.layers - 1 if predicted else 0)
 
 
+def headline_line(cfg, world: int, steps: int, warmup: int, ms: float, value: float, e2e_value: float,
+                  single: bool, clocks: dict) -> dict:
+    """The JSON line of the decode headline from the measured numbers.
+
+    ``ms`` is the max-over-ranks device time of the ``steps`` timed steps and
+    ``value`` the whole-job rate from it; the roofline numerator is the
+    algorithmic bytes of one step (one stack launch on the single-launch path)
+    over the mean step time.
+    """
+    T = cfg.T
+    peak, peak_kind = peaks()
+    bytes_step = token_layer_bytes(cfg) * cfg.layers * T
+    achieved = bytes_step / (ms / steps / 1000.0) / 1e9
+    return {
+        "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": steps,
+        "warmup": warmup, "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {**decode_config(cfg, world),
+                   "l2": "inputs larger than L2: 433 MB of weights read per step, a distinct token per step",
+                   "path": "moe_stack_decode, " + ("one cooperative launch per token" if single
+                                                     else "per-layer launches")},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": measured_traffic(cfg.layers) if single else None, "peak_kind": peak_kind,
+                     "scope": "stack kernel (the whole step)" if single else "whole step (all launches)",
+                     "algorithmic_bytes_per_step": bytes_step},
+        "e2e": {"value": e2e_value, "unit": "tok/s", "h2d_bytes_per_step": T * cfg.H * 4,
+                "d2h_bytes_per_step": T * cfg.H * 4},
+        "gpu_launches": launches_per_step(cfg, single) * steps,
+        "clocks": clocks,
+    }
+
+
 def smi_gpu_id(local: int) -> str:
     """nvidia-smi ``--id`` of this process's CUDA device ``local``.
 
@@ -597,26 +629,7 @@ def main():
     ms_e2e = max_over_ranks(ms_e2e, dist, dev)
     e2e_value = whole_job_rate(T * e2e_steps, world, ms_e2e)
 
-    peak, peak_kind = peaks()
-    bytes_step = token_layer_bytes(cfg) * cfg.layers * T
-    achieved = bytes_step / (ms / args.steps / 1000.0) / 1e9
-    out = {
-        "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {**decode_config(cfg, world),
-                   "l2": "inputs larger than L2: 433 MB of weights read per step, a distinct token per step",
-                   "path": "moe_stack_decode, " + ("one cooperative launch per token" if single
-                                                     else "per-layer launches")},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": measured_traffic(cfg.layers) if single else None, "peak_kind": peak_kind,
-                     "scope": "stack kernel (the whole step)" if single else "whole step (all launches)",
-                     "algorithmic_bytes_per_step": bytes_step},
-        "e2e": {"value": e2e_value, "unit": "tok/s", "h2d_bytes_per_step": T * cfg.H * 4,
-                "d2h_bytes_per_step": T * cfg.H * 4},
-        "gpu_launches": launches_per_step(cfg, single) * args.steps,
-        "clocks": clk.summary(),
-    }
+    out = headline_line(cfg, world, args.steps, args.warmup, ms, value, e2e_value, single, clk.summary())
     if not args.no_prefill:
         del stack, st, ws, xpool
         torch.cuda.empty_cache()

@@ -1,9 +1,12 @@
-"""The benchmark's roofline numerators, recomputed term by term from the storage formats."""
+"""Host-side parts of bench.py: roofline numerators from the storage formats, the oracle reference arm, the
+JSON line."""
 import os
 import sys
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
+
+import pytest  # noqa: E402
 
 import bench  # noqa: E402
 from gen import CONFIGS  # noqa: E402
@@ -109,3 +112,26 @@ def test_clock_sampler_names_the_visible_gpu(monkeypatch):
     monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "GPU-0a1b, GPU-2c3d")
     assert bench.smi_gpu_id(1) == "GPU-2c3d"
     assert bench.Clocks(0).gpu == "GPU-0a1b"
+
+
+def test_headline_line_carries_every_contract_key():
+    cfg = CONFIGS[bench.CFG_ID]
+    steps, ms, world = 2000, 1900.0, 2
+    value = bench.whole_job_rate(cfg.T * steps, world, ms)
+    clocks = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    line = bench.headline_line(cfg, world, steps, 20, ms, value, 900.0, True, clocks)
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+        assert key in line, key
+    assert line["value"] == pytest.approx(2 * steps / 1.9) and line["ms_per_step"] == pytest.approx(0.95)
+    assert line["n_gpus"] == 2 and line["scaling"] == "weak" and line["config"]["parallelism"] == "replicas x2"
+    assert line["config"]["workload"] and line["clocks"] is clocks
+    r = line["roofline"]
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["algorithmic_bytes_per_step"] == 433_402_880
+    assert r["achieved"] == pytest.approx(433_402_880 / 0.95e-3 / 1e9)
+    assert r["frac"] == pytest.approx(r["achieved"] / r["peak"])
+    assert line["e2e"] == {"value": 900.0, "unit": "tok/s", "h2d_bytes_per_step": 2048 * 4,
+                           "d2h_bytes_per_step": 2048 * 4}
+    assert line["gpu_launches"] == steps  # one cooperative launch per token
+    per_layer = bench.headline_line(cfg, 1, steps, 20, ms, value, 900.0, False, clocks)
+    assert per_layer["gpu_launches"] == steps * cfg.layers * 10 and per_layer["roofline"]["traffic"] is None
