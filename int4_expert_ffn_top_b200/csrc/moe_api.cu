@@ -41,6 +41,43 @@ moe_status check_layer(const moe_layer* L, int T, int K) {
   return MOE_OK;
 }
 
+size_t block_bytes(int H, int I) {
+  return static_cast<size_t>(2 * I) * qrow_bytes(H, 4) + static_cast<size_t>(H) * qrow_bytes(I, 4);
+}
+
+// Weight pointers moe_expert_forward reads besides the router (after check_layer).
+moe_status check_expert_weights(const moe_layer* L) {
+  if (!L->pool || !aligned(L->pool, 256) || L->expert_stride < static_cast<int64_t>(block_bytes(L->H, L->I)) ||
+      L->expert_stride % 256)
+    return MOE_ERR_INVALID_ARG;
+  if (!qrows_ok(L->shared_gate, 1, L->H, 8) || !L->shared_block || !aligned(L->shared_block, 16))
+    return MOE_ERR_INVALID_ARG;
+  if (L->r > 0) {
+    for (int p = 0; p < 3; ++p)
+      if ((L->sh_lora_A[p] != nullptr) != (L->sh_lora_B[p] != nullptr)) return MOE_ERR_INVALID_ARG;
+    if ((L->ex_lora_A != nullptr) != (L->ex_lora_B != nullptr)) return MOE_ERR_INVALID_ARG;
+    const void* lp[8] = {L->sh_lora_A[0], L->sh_lora_A[1], L->sh_lora_A[2], L->ex_lora_A,
+                         L->sh_lora_B[0], L->sh_lora_B[1], L->sh_lora_B[2], L->ex_lora_B};
+    for (const void* p : lp)
+      if (p && !aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+  }
+  return MOE_OK;
+}
+
+// Shapes a Prerouter head supports for (K, K_next).
+moe_status check_head_shape(const moe_prerouter* P, int K, int K_next) {
+  if (K < 1 || K > 8 || K_next < 1 || K_next > 8) return MOE_ERR_UNSUPPORTED;
+  if (!h_ok(P->H) || P->E < K || P->E > 256 || P->E % 8 || P->E_next < K_next || P->E_next > 256 || P->P < 8 ||
+      P->P % 8)
+    return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status check_head_weights(const moe_prerouter* P) {
+  if (!P->W1 || !P->b1 || !P->W2 || !P->b2 || !aligned(P->W1, 16) || !aligned(P->W2, 16)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
 // Workspace carve-up of moe_expert_forward.
 struct Ws {
   void* base;
@@ -427,7 +464,7 @@ size_t moe_qrow_bytes(int32_t in_dim, int32_t bits) {
 
 size_t moe_expert_block_bytes(int32_t H, int32_t I) {
   if (H <= 0 || I <= 0 || H % 64 || I % 64) return 0;
-  return static_cast<size_t>(2 * I) * qrow_bytes(H, 4) + static_cast<size_t>(H) * qrow_bytes(I, 4);
+  return block_bytes(H, I);
 }
 
 moe_status moe_rmsnorm_bf16(const float* x, int32_t T, int32_t H, float eps, uint16_t* u, void* stream) {
@@ -476,20 +513,9 @@ moe_status moe_expert_forward(const moe_layer* L, const uint16_t* u, int32_t T, 
   if (s != MOE_OK) return s;
   if (out_mode < 0 || out_mode > 2) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
-  if (!u || !idx || !w || !out || !L->pool || !aligned(u, 16) || !aligned(L->pool, 256) ||
-      L->expert_stride < static_cast<int64_t>(moe_expert_block_bytes(L->H, L->I)) || L->expert_stride % 256)
-    return MOE_ERR_INVALID_ARG;
-  if (!qrows_ok(L->shared_gate, 1, L->H, 8) || !L->shared_block || !aligned(L->shared_block, 16))
-    return MOE_ERR_INVALID_ARG;
-  if (L->r > 0) {
-    for (int p = 0; p < 3; ++p)
-      if ((L->sh_lora_A[p] != nullptr) != (L->sh_lora_B[p] != nullptr)) return MOE_ERR_INVALID_ARG;
-    if ((L->ex_lora_A != nullptr) != (L->ex_lora_B != nullptr)) return MOE_ERR_INVALID_ARG;
-    const void* lp[8] = {L->sh_lora_A[0], L->sh_lora_A[1], L->sh_lora_A[2], L->ex_lora_A,
-                         L->sh_lora_B[0], L->sh_lora_B[1], L->sh_lora_B[2], L->ex_lora_B};
-    for (const void* p : lp)
-      if (p && !aligned(p, 16)) return MOE_ERR_INVALID_ARG;
-  }
+  if (!u || !idx || !w || !out || !aligned(u, 16)) return MOE_ERR_INVALID_ARG;
+  s = check_expert_weights(L);
+  if (s != MOE_OK) return s;
   if (!workspace || !aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < ws_bytes_for(L, T, K)) return MOE_ERR_WORKSPACE;
   const Ws ws = carve(workspace, T, K, L->E, L->I, L->r);
@@ -513,14 +539,13 @@ moe_status prerouter_predict(const moe_prerouter* head, const uint16_t* u, const
                              int32_t K_next, int32_t* pred, float* scores, void* workspace, size_t ws_bytes,
                              void* stream) {
   if (!head) return MOE_ERR_INVALID_ARG;
-  if (T < 0 || T > MOE_MAX_TOKENS || K < 1 || K > 8 || K_next < 1 || K_next > 8) return MOE_ERR_UNSUPPORTED;
-  if (!h_ok(head->H) || head->E < K || head->E > 256 || head->E % 8 || head->E_next < K_next ||
-      head->E_next > 256 || head->P < 8 || head->P % 8)
-    return MOE_ERR_UNSUPPORTED;
+  if (T < 0 || T > MOE_MAX_TOKENS) return MOE_ERR_UNSUPPORTED;
+  moe_status s = check_head_shape(head, K, K_next);
+  if (s != MOE_OK) return s;
   if (T == 0) return MOE_OK;
-  if (!u || !sel || !pred || !scores || !head->W1 || !head->b1 || !head->W2 || !head->b2 || !aligned(u, 16) ||
-      !aligned(head->W1, 16) || !aligned(head->W2, 16))
-    return MOE_ERR_INVALID_ARG;
+  if (!u || !sel || !pred || !scores || !aligned(u, 16)) return MOE_ERR_INVALID_ARG;
+  s = check_head_weights(head);
+  if (s != MOE_OK) return s;
   if (!workspace || !aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < prerouter_ws(head, T)) return MOE_ERR_WORKSPACE;
   float* z = static_cast<float*>(workspace);
@@ -787,8 +812,18 @@ moe_status moe_stack_decode(const moe_layer* layers, const moe_prerouter* heads,
     if (heads && (heads[l].H != layers[0].H || heads[l].E != layers[0].E || heads[l].E_next != heads[0].E_next ||
                   heads[l].P != heads[0].P))
       return MOE_ERR_UNSUPPORTED;
+    if (heads) {
+      const moe_status hs = check_head_shape(&heads[l], K, K_next);
+      if (hs != MOE_OK) return hs;
+    }
   }
   if (T == 0) return MOE_OK;
+  // Every layer's weights are checked here, so that no launch happens for a stack that would fail part-way.
+  for (int l = 0; l < n_layers; ++l) {
+    moe_status s = check_expert_weights(&layers[l]);
+    if (s == MOE_OK && heads) s = check_head_weights(&heads[l]);
+    if (s != MOE_OK) return s;
+  }
   const size_t llb = ll_bound(&layers[0], heads, K, n_layers);
   const StackWs need = carve_stack(nullptr, &layers[0], heads, T, K, K_next, llb);
   if (!workspace || !aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;

@@ -165,3 +165,87 @@ def test_expert_block_layout_decodes_back_to_the_expert():
     off = 2 * I * rgu
     for o in (0, 7, H - 1):
         assert np.array_equal(decode(blk[off + o * rdn:off + (o + 1) * rdn], I), dn[o])
+
+
+# Well-formed structs whose pointers are aligned stand-in addresses.  The calls
+# below end at a host-side check (a zero-byte workspace at the latest), so no
+# address is ever used on a device.
+def _fake_layer(base: int):
+    from int4_expert_ffn_top_b200 import _lib
+    from int4_expert_ffn_top_b200.weights import block_stride
+    L = _lib.moe_layer()
+    L.H, L.E, L.I, L.I_s, L.r = 2048, 256, 512, 512, 16
+    L.router = _lib.moe_qrows(base + 0x1000, 256, 2048, 8)
+    L.shared_gate = _lib.moe_qrows(base + 0x2000, 1, 2048, 8)
+    L.shared_block = base + 0x3000
+    for i in range(3):
+        L.sh_lora_A[i], L.sh_lora_B[i] = base + 0x4000 + 0x100 * i, base + 0x5000 + 0x100 * i
+    L.lora_scale = 1.0
+    L.pool = base + 0x100000
+    L.expert_stride = block_stride(2048, 512)
+    return L
+
+
+def _fake_head(base: int):
+    from int4_expert_ffn_top_b200 import _lib
+    P = _lib.moe_prerouter()
+    P.W1, P.b1, P.W2, P.b2 = base + 0x6000, base + 0x7000, base + 0x8000, base + 0x9000
+    P.H, P.E, P.P, P.E_next = 2048, 256, 256, 256
+    return P
+
+
+FAKE_WS = 0x7f0000000000  # 256-byte aligned, never dereferenced: every call is refused before it
+
+
+def test_well_formed_calls_pass_every_host_check(lib):
+    from int4_expert_ffn_top_b200 import _lib
+    L, P = _fake_layer(0x10000000), _fake_head(0x20000000)
+    dev = 0x30000000
+    assert lib.moe_expert_forward(ctypes.byref(L), dev, 1, 4, dev, dev, dev, 0, None, FAKE_WS, 0,
+                                  None) == _lib.MOE_ERR_WORKSPACE
+    assert lib.prerouter_predict(ctypes.byref(P), dev, dev, 1, 4, 4, dev, dev, FAKE_WS, 0,
+                                 None) == _lib.MOE_ERR_WORKSPACE
+    layers = (_lib.moe_layer * 3)(*[_fake_layer(0x10000000 * (l + 1)) for l in range(3)])
+    heads = (_lib.moe_prerouter * 3)(*[_fake_head(0x40000000 * (l + 1)) for l in range(3)])
+    assert lib.moe_stack_decode(layers, heads, 3, 1, 4, 4, 1e-6, dev, None, None, None, None, None, 0, None, None,
+                                FAKE_WS, 0, None) == _lib.MOE_ERR_WORKSPACE
+
+
+def test_stack_weights_of_every_layer_are_checked_before_any_launch(lib):
+    from int4_expert_ffn_top_b200 import _lib
+
+    def stack_status(edit_layer=None, edit_head=None, K_next=4):
+        layers = (_lib.moe_layer * 3)(*[_fake_layer(0x10000000 * (l + 1)) for l in range(3)])
+        heads = (_lib.moe_prerouter * 3)(*[_fake_head(0x40000000 * (l + 1)) for l in range(3)])
+        if edit_layer:
+            edit_layer(layers[2])
+        if edit_head:
+            edit_head(heads[2])
+        return lib.moe_stack_decode(layers, heads, 3, 1, 4, K_next, 1e-6, 0x30000000, None, None, None, None, None,
+                                    0, None, None, FAKE_WS, 0, None)
+
+    def no_pool(L):
+        L.pool = None
+
+    def short_stride(L):
+        L.expert_stride = 256
+
+    def half_lora(L):
+        L.sh_lora_B[1] = None
+
+    def no_w1(P):
+        P.W1 = None
+
+    def odd_w2(P):
+        P.W2 = P.W2 + 8
+
+    def small_e_next(P):
+        P.E_next = 2
+
+    for edit in (no_pool, short_stride, half_lora):
+        assert stack_status(edit_layer=edit) == _lib.MOE_ERR_INVALID_ARG, edit.__name__
+    for edit in (no_w1, odd_w2):
+        assert stack_status(edit_head=edit) == _lib.MOE_ERR_INVALID_ARG, edit.__name__
+    assert stack_status(edit_head=small_e_next) == _lib.MOE_ERR_UNSUPPORTED
+    assert stack_status(K_next=9) == _lib.MOE_ERR_UNSUPPORTED
+    assert stack_status() == _lib.MOE_ERR_WORKSPACE
