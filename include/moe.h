@@ -17,7 +17,10 @@
  * --------------------------------
  * Ownership:  the caller allocates every device buffer (weights, activations,
  *             outputs, workspace).  The library allocates nothing and keeps no
- *             state between calls.  All pointers are device pointers unless a
+ *             state between calls, apart from the allocation-free variant's
+ *             fixed scratch array (moe_expert_forward_noalloc) and the looked-up
+ *             address of the driver's tensor-map encoder.  All pointers are
+ *             device pointers unless a
  *             comment says "host".  Structs are read on the host during the call
  *             and may be freed when it returns.
  * Asynchrony: work is enqueued on `stream` (a cudaStream_t passed as void*;
@@ -173,7 +176,8 @@ moe_status moe_expert_forward(const moe_layer* L, const uint16_t* u, int32_t T, 
                               const int32_t* idx, const float* w, void* out, int32_t out_mode,
                               int32_t* perm_out, void* workspace, size_t ws_bytes, void* stream);
 
-/* Scratch bytes moe_expert_forward needs for (L, T, K) (host). */
+/* Scratch bytes moe_expert_forward needs for (L, T, K) (host); 0 for a NULL
+ * layer, T < 0, T > MOE_MAX_TOKENS or K < 1. */
 size_t moe_workspace_size(const moe_layer* L, int32_t T, int32_t K);
 
 /*
@@ -188,6 +192,8 @@ moe_status prerouter_predict(const moe_prerouter* head, const uint16_t* u, const
                              int32_t T, int32_t K, int32_t K_next, int32_t* pred, float* scores,
                              void* workspace, size_t ws_bytes, void* stream);
 
+/* Scratch bytes prerouter_predict needs for T tokens (host); 0 for a NULL head,
+ * T < 0 or T > MOE_MAX_TOKENS. */
 size_t prerouter_workspace_size(const moe_prerouter* head, int32_t T);
 
 /* Options of moe_stack_decode (NULL = all defaults). */
@@ -244,6 +250,8 @@ moe_status moe_stack_decode(const moe_layer* layers, const moe_prerouter* heads,
                             int32_t use_predicted_routing, int32_t* err_word, const moe_stack_opts* opts,
                             void* workspace, size_t ws_bytes, void* stream);
 
+/* Scratch bytes moe_stack_decode needs (host); 0 for NULL layers,
+ * n_layers < 1, T < 0, T > MOE_MAX_TOKENS or K < 1. */
 size_t moe_stack_workspace_size(const moe_layer* layers, const moe_prerouter* heads, int32_t n_layers, int32_t T,
                                 int32_t K, int32_t K_next);
 
