@@ -249,3 +249,38 @@ def test_stack_weights_of_every_layer_are_checked_before_any_launch(lib):
     assert stack_status(edit_head=small_e_next) == _lib.MOE_ERR_UNSUPPORTED
     assert stack_status(K_next=9) == _lib.MOE_ERR_UNSUPPORTED
     assert stack_status() == _lib.MOE_ERR_WORKSPACE
+
+
+def test_header_is_plain_c99_and_the_library_links_from_c(lib):
+    """A C program (no C++, no torch) compiles against include/moe.h with -pedantic -Werror, links libmoe.so and
+    calls the host-only entry points; the one compute entry point it calls is refused before any launch."""
+    import shutil
+    import subprocess
+
+    from int4_expert_ffn_top_b200 import build as B
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    out_dir = os.path.join(ROOT, "_build", "c_abi_check")
+    os.makedirs(out_dir, exist_ok=True)
+    src, exe = os.path.join(out_dir, "main.c"), os.path.join(out_dir, "main")
+    with open(src, "w") as f:
+        f.write(r'''
+#include <stdio.h>
+#include <string.h>
+#include "moe.h"
+int main(void) {
+  moe_layer L;
+  memset(&L, 0, sizeof L);
+  L.H = 2048; L.E = 256; L.I = 512; L.I_s = 512; L.r = 16;
+  printf("%s|%zu|%zu|%d|%zu\n", moe_status_string(MOE_ERR_WORKSPACE), moe_expert_block_bytes(2048, 512),
+         moe_qrow_bytes(2048, 8), (int)moe_route_topk(&L, NULL, 1, 4, NULL, NULL, NULL, NULL),
+         moe_workspace_size(&L, MOE_MAX_TOKENS + 1, 4));
+  return 0;
+}
+''')
+    lib_dir = os.path.dirname(B.LIB)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    src, "-o", exe, "-L", lib_dir, "-lmoe", f"-Wl,-rpath,{lib_dir}"], check=True, timeout=120)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60, check=True)
+    assert r.stdout.strip() == "workspace too small|1769472|2176|1|0"  # router rows missing -> invalid argument
