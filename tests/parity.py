@@ -37,10 +37,30 @@ def qmat_abs_terms(m: dict) -> np.ndarray:
     return np.abs(q - mid) * s + np.abs(b + mid * s)
 
 
+def fp16_input_error(u: np.ndarray) -> np.ndarray:
+    """|u - fp16(u)|: the GEMV kernels multiply weights by the activations rounded to fp16.
+
+    bf16 values convert to fp16 exactly down to 2^-17 in magnitude; below that
+    (fp16 subnormals) the conversion rounds, which this term accounts for.
+    """
+    u = np.asarray(u, np.float64)
+    return np.abs(u - u.astype(np.float16).astype(np.float64))
+
+
 def router_tau(u: np.ndarray, router: dict, n_round: int = 64) -> np.ndarray:
-    """Bound [T, E] on |fp32 GPU logit - exact logit| for inputs u (bf16 values)."""
+    """Bound [T, E] on |fp32 GPU logit - exact logit| for inputs u (bf16 values).
+
+    ``n_round`` fp32 roundings on the path of any product term (the router
+    kernel takes at most 38 at H = 4096: 16 within a 16-element chunk, 2 per
+    chunk of a lane, a 5-level lane reduction, the bias add), plus the exact
+    effect of rounding u to fp16 in the ``s (q - mid)`` part of the split dot.
+    """
     beta = np.abs(np.asarray(router["beta"], np.float64))
-    return n_round * EPS32 * (np.abs(u) @ qmat_abs_terms(router).T) + 4 * EPS32 * beta
+    mid = 8 if router["bits"] == 4 else 128
+    q = O.unpack_codes(router["q"], router["bits"]).astype(np.float64)
+    s = np.repeat(router["s"].astype(np.float64), 64, 1)
+    return (n_round * EPS32 * (np.abs(u) @ qmat_abs_terms(router).T) + 4 * EPS32 * beta
+            + fp16_input_error(u) @ (np.abs(q - mid) * s).T)
 
 
 def check_topk(gpu_idx, ref, tau_row, K: int, exact_order: bool = True) -> int:

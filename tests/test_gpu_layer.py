@@ -12,7 +12,7 @@ import torch
 
 from gen import CONFIGS, inputs
 from oracle import moe_oracle as O
-from parity import EPS32, assert_close_inf, check_bf16_rounding, check_topk, router_tau
+from parity import EPS32, assert_close_inf, check_bf16_rounding, check_topk, fp16_input_error, router_tau
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -94,6 +94,7 @@ def prerouter_tau(u, sel, head, E, n_round=128):
     W2 = np.abs(head["W2"].astype(np.float64))
     xin = np.concatenate([np.abs(u), O.multi_hot(sel, E)], axis=1)
     a_err = n_round * EPS32 * (xin @ W1.T + np.abs(head["b1"].astype(np.float64)))
+    a_err = a_err + fp16_input_error(u) @ W1[:, :u.shape[1]].T  # u enters W1 rounded to fp16
     z = np.abs(O.silu(np.concatenate([u, O.multi_hot(sel, E)], 1) @ head["W1"].astype(np.float64).T
                       + head["b1"].astype(np.float64)))
     return (1.1 * a_err + 8 * EPS32 * z) @ W2.T + n_round * EPS32 * (z @ W2.T + np.abs(head["b2"].astype(np.float64)))
