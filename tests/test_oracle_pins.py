@@ -363,6 +363,28 @@ def test_prerouter_closed_forms():
     assert np.all(O.multi_hot(sel, E).sum(1) == 2)
 
 
+def test_prerouter_reads_the_executed_experts_under_predicted_routing():
+    """The head's multi-hot input is the set the layer executed, not the router's own top-K: with a head
+    that maps the multi-hot through a permutation, the prediction is the permuted executed set."""
+    cfg = CONFIGS[0]
+    L = _tiny_layer(cfg)
+    E, H, P = cfg.E, cfg.H, cfg.P
+    rng = np.random.default_rng(12)
+    pi = rng.permutation(E)
+    W1 = np.zeros((P, H + E), np.float16)
+    W1[np.arange(E), H + np.arange(E)] = 2.0  # z_e = silu(2 * multi_hot_e); the u columns are zero
+    W2 = np.zeros((E, P), np.float16)
+    W2[pi, np.arange(E)] = 1.0                 # p[pi[e]] = z_e
+    L["prerouter"] = dict(W1=W1, b1=np.zeros(P, np.float16), W2=W2, b2=np.zeros(E, np.float16))
+    u = inputs.bf16_bits_to_f32(inputs.activations(cfg)).astype(np.float64)
+    true_idx = O.layer_forward(u, L, cfg.K)["true_idx"]
+    forced = (true_idx + 5) % E  # never the router's own choice
+    r = O.layer_forward(u, L, cfg.K, routing=forced)
+    for t in range(cfg.T):
+        assert sorted(r["pred"][t]) == sorted(pi[forced[t]])
+        assert not set(r["pred"][t]) & set(pi[true_idx[t]])
+
+
 # ----------------------------------------------------------------------------- buckets
 def test_buckets_brute_force_and_invariants():
     rng = np.random.default_rng(10)
@@ -381,6 +403,40 @@ def test_buckets_brute_force_and_invariants():
 
 
 # ----------------------------------------------------------------------------- pin sensitivity
+def _ffn_lora_after_silu(u, ex, lora_gate=None, lora_up=None, lora_down=None):
+    """Planted mistake: the gate projection's LoRA delta added after SiLU instead of before."""
+    Wgu = O.dequant(ex["gate_up"])
+    I = Wgu.shape[0] // 2
+    a = np.asarray(u, np.float64) @ Wgu[:I].T
+    b = np.asarray(u, np.float64) @ Wgu[I:].T + O.lora_delta(u, lora_up)
+    h = (O.silu(a) + O.lora_delta(u, lora_gate)) * b
+    return h @ O.dequant(ex["down"]).T + O.lora_delta(h, lora_down)
+
+
+def _prerouter_on_true_topk(monkeypatch):
+    """Planted mistake: the head's multi-hot built from the router's own top-K instead of the executed set."""
+    layer_forward = O.layer_forward
+
+    def lf(u, L, K, routing=None, K_next=None):
+        r = layer_forward(u, L, K, routing, K_next)
+        if "prerouter" in L:
+            r["pred"], r["p"] = O.prerouter_predict(u, r["true_idx"], L["prerouter"], r["logits"].shape[1],
+                                                    K_next or K)
+        return r
+
+    monkeypatch.setattr(O, "layer_forward", lf)
+    return O.prerouter_predict
+
+
+def _reverse_within_buckets(b):
+    perm = b["perm"].copy()
+    for e in range(len(b["count"])):
+        perm[b["offset"][e]:b["offset"][e + 1]] = perm[b["offset"][e]:b["offset"][e + 1]][::-1]
+    inv = np.empty_like(perm)
+    inv[perm] = np.arange(perm.size)
+    return dict(b, perm=perm, inv=inv)
+
+
 def test_planted_mistakes_are_caught(monkeypatch):
     """Plant plausible mistakes in the oracle (on the CPU) and check a pin fails for each."""
     planted = {
@@ -401,12 +457,34 @@ def test_planted_mistakes_are_caught(monkeypatch):
             O, "layer_forward", lambda u, L, K, routing=None, K_next=None, _f=O.layer_forward: _f(u, L, K, None, K_next)),
         "layer input not rounded to bf16": lambda: monkeypatch.setattr(
             O, "layer_input", lambda x, eps=1e-6: O.rmsnorm(x, eps)),
+        "gating softmax over all E, not the K": lambda: monkeypatch.setattr(
+            O, "gating", lambda l, idx: np.take_along_axis(
+                np.exp(l - l.max(1, keepdims=True)) / np.exp(l - l.max(1, keepdims=True)).sum(1, keepdims=True),
+                idx, axis=1)),
+        "LoRA delta dropped": lambda: monkeypatch.setattr(O, "lora_delta", lambda x, lo: 0.0),
+        "gate LoRA added after the activation": lambda: monkeypatch.setattr(O, "expert_ffn", _ffn_lora_after_silu),
+        "shared gate ignored": lambda: monkeypatch.setattr(
+            O, "shared_gate", lambda u, sh: np.ones(np.asarray(u).shape[0])),
+        "combine drops the shared expert": lambda: monkeypatch.setattr(
+            O, "combine", lambda w, y, g, ys: np.einsum("tk,tkh->th", w, y)),
+        "Prerouter fed the router's own top-K": lambda: monkeypatch.setattr(
+            O, "prerouter_predict", _prerouter_on_true_topk(monkeypatch)),
+        "bucket order descending within an expert": lambda: monkeypatch.setattr(
+            O, "buckets", lambda idx, E, _b=O.buckets: _reverse_within_buckets(_b(idx, E))),
+        "router offset beta ignored": lambda: monkeypatch.setattr(
+            O, "router_logits", lambda u, R, _r=O.router_logits: _r(u, dict(R, beta=np.zeros_like(R["beta"])))),
+        "RMSNorm without eps": lambda: monkeypatch.setattr(
+            O, "rmsnorm", lambda x, eps=1e-6, _n=O.rmsnorm: _n(x, 0.0)),
     }
     pins = [test_hand_built_words, lambda: test_dequant_exhaustive_codes_exact(4), test_dequant_group_boundaries,
             test_expert_ffn_closed_form_on_selection_weights, test_topk_brute_force_with_ties,
             test_topk_all_equal_gives_lowest_indices, test_activation_closed_forms,
             test_router_closed_form_on_one_hot_weights, test_stack_forward_with_zero_experts_keeps_the_residual,
-            test_stack_forward_predicted_routing_executes_the_previous_prediction]
+            test_stack_forward_predicted_routing_executes_the_previous_prediction, test_rmsnorm_closed_forms,
+            test_gating_closed_forms, test_lora_unmerged_equals_merged_and_one_hot, test_shared_gate_half_on_zero_weights,
+            test_layer_with_zero_routed_experts_is_half_shared, test_layer_sparse_equals_dense_masked_mixture,
+            test_prerouter_closed_forms, test_prerouter_reads_the_executed_experts_under_predicted_routing,
+            test_buckets_brute_force_and_invariants]
     for name, plant in planted.items():
         plant()
         failed = False
