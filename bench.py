@@ -8,7 +8,12 @@ an independent replica (batch-1 decode does not shard; weak scaling).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
-Prints one JSON line on rank 0.
+Prints one JSON line on rank 0.  Beside the headline it reports the 35B-shaped
+prefill (3,328 tokens), the 8B-shaped decode and a 64-token batched decode with
+predicted routing, and, at N = 1, the float64 oracle timed on the host cores.
+``--impl reference`` times only that oracle, on rank 0: each step is one of
+its work items for a batch-1 token (route, one routed expert, shared expert,
+combine + Prerouter), and seconds per token are taken from the per-kind means.
 """
 from __future__ import annotations
 
