@@ -283,6 +283,80 @@ def test_lora_unmerged_equals_merged_and_one_hot():
     assert np.array_equal(d[:, 41], x[:, 17]) and np.count_nonzero(d) == np.count_nonzero(x[:, 17])
 
 
+def _one_hot_lora(out_dim, in_dim, i, j, c, r=2):
+    """Rank-r adapter whose only nonzero path maps input ``i`` to output ``j`` with gain ``c`` (through rank 1)."""
+    A = np.zeros((r, in_dim), np.float16)
+    A[1, i] = 1
+    B = np.zeros((out_dim, r), np.float16)
+    B[j, 1] = c
+    return dict(A=A, B=B, scale=1.0)
+
+
+def test_lora_on_every_projection_closed_form():
+    """Selection-matrix expert with a one-hot adapter on each of gate, up and down (2kiu.com, "Recover-LoRA"
+    bullet: the adapter stays unmerged on the frozen base).  Each adapter adds ``c * input[i]`` to one output of
+    its own projection, before the activation, so the closed form says which projection carries which adapter;
+    the shared expert must wire ``lora_gate`` / ``lora_up`` / ``lora_down`` to the same projections."""
+    rng = np.random.default_rng(13)
+    H, I = 128, 64
+    ex, pg, pu, sig, s, sd = _perm_expert(H, I, rng)
+    u = O.round_bf16(rng.standard_normal((4, H)))
+    (ig, jg, cg), (iu, ju, cu), (ih, od, cd) = (5, 7, 0.5), (9, 11, -0.25), (13, 17, 0.75)
+    lg, lu, ld = _one_hot_lora(I, H, ig, jg, cg), _one_hot_lora(I, H, iu, ju, cu), _one_hot_lora(H, I, ih, od, cd)
+    g = s * u[:, pg]
+    g[:, jg] += cg * u[:, ig]
+    up = 2 * s * u[:, pu]
+    up[:, ju] += cu * u[:, iu]
+    h = g / (1 + np.exp(-g)) * up
+    want = -3 * sd * h[:, sig]
+    want[:, od] += cd * h[:, ih]
+    assert np.allclose(O.expert_hidden(u, ex, lg, lu), h, rtol=1e-13, atol=1e-15)
+    assert np.allclose(O.expert_ffn(u, ex, lg, lu, ld), want, rtol=1e-13, atol=1e-15)
+    sh = dict(ex, lora_gate=lg, lora_up=lu, lora_down=ld)
+    assert np.allclose(O.shared_expert(u, sh), want, rtol=1e-13, atol=1e-15)
+
+
+def test_lora_unmerged_equals_merged_on_up_and_down():
+    """``W + B A`` merged into the dequantised up and down matrices equals the unmerged deltas."""
+    rng = np.random.default_rng(14)
+    cfg = CONFIGS[0]
+    ex = inputs.expert(cfg, 0, 2)
+    H, I, r = cfg.H, cfg.I, 4
+    lo = lambda o, i: dict(A=(rng.standard_normal((r, i)) * 0.05).astype(np.float16),
+                           B=(rng.standard_normal((o, r)) * 0.05).astype(np.float16), scale=1.0)
+    lu, ld = lo(I, H), lo(H, I)
+    Wgu = O.dequant(ex["gate_up"])
+    Wu = Wgu[I:] + lu["B"].astype(np.float64) @ lu["A"].astype(np.float64)
+    Wd = O.dequant(ex["down"]) + ld["B"].astype(np.float64) @ ld["A"].astype(np.float64)
+    u = rng.standard_normal((3, H))
+    a = u @ Wgu[:I].T
+    want = (a / (1 + np.exp(-a)) * (u @ Wu.T)) @ Wd.T
+    assert np.allclose(O.expert_ffn(u, ex, lora_up=lu, lora_down=ld), want, rtol=1e-11, atol=1e-11)
+
+
+def test_routed_down_lora_reaches_the_layer_output():
+    """A one-hot down adapter on every routed expert (the batched-decode workload's LoRA) adds
+    ``c * h_e[i]`` to output ``o`` of every slot; through the combine the layer output moves by
+    ``sum_k w_k c h_{e_k}[i]`` at ``o`` and nowhere else."""
+    cfg = CONFIGS[0]
+    L = _tiny_layer(cfg)
+    u = O.round_bf16(inputs.bf16_bits_to_f32(inputs.activations(cfg)).astype(np.float64))
+    ih, od, cd = 3, 29, 0.625
+    base = O.layer_forward(u, L, cfg.K)
+    for e in L["experts"]:
+        L["experts"][e]["down_lora"] = _one_hot_lora(cfg.H, cfg.I, ih, od, cd)
+    r = O.layer_forward(u, L, cfg.K)
+    assert np.array_equal(r["idx"], base["idx"])
+    hk = np.stack([[O.expert_hidden(u[t:t + 1], L["experts"][int(e)])[0, ih] for e in base["idx"][t]]
+                   for t in range(cfg.T)])
+    dy = r["y"] - base["y"]
+    assert np.allclose(dy[:, :, od], cd * hk, rtol=1e-12, atol=1e-15)
+    assert np.count_nonzero(np.delete(dy, od, axis=2)) == 0
+    dout = r["out"] - base["out"]
+    assert np.allclose(dout[:, od], (base["w"] * cd * hk).sum(1), rtol=1e-11, atol=1e-15)
+    assert np.count_nonzero(np.delete(dout, od, axis=1)) == 0
+
+
 def test_shared_gate_half_on_zero_weights():
     H = 128
     sh = dict(gate=zero_qmat(1, H, s=0.01 / 16, bits=8))
@@ -475,6 +549,18 @@ def test_planted_mistakes_are_caught(monkeypatch):
             O, "router_logits", lambda u, R, _r=O.router_logits: _r(u, dict(R, beta=np.zeros_like(R["beta"])))),
         "RMSNorm without eps": lambda: monkeypatch.setattr(
             O, "rmsnorm", lambda x, eps=1e-6, _n=O.rmsnorm: _n(x, 0.0)),
+        "up LoRA dropped": lambda: monkeypatch.setattr(
+            O, "expert_ffn", lambda u, ex, lora_gate=None, lora_up=None, lora_down=None, _f=O.expert_ffn:
+            _f(u, ex, lora_gate, None, lora_down)),
+        "down LoRA dropped": lambda: monkeypatch.setattr(
+            O, "expert_ffn", lambda u, ex, lora_gate=None, lora_up=None, lora_down=None, _f=O.expert_ffn:
+            _f(u, ex, lora_gate, lora_up, None)),
+        "routed down LoRA dropped": lambda: monkeypatch.setattr(
+            O, "routed_outputs", lambda u, experts, idx, _r=O.routed_outputs: _r(
+                u, {e: {k: v for k, v in ex.items() if k != "down_lora"} for e, ex in experts.items()}, idx)),
+        "shared gate/up adapters swapped": lambda: monkeypatch.setattr(
+            O, "shared_expert", lambda u, sh, _f=O.expert_ffn: _f(u, sh, sh.get("lora_up"), sh.get("lora_gate"),
+                                                                  sh.get("lora_down"))),
     }
     pins = [test_hand_built_words, lambda: test_dequant_exhaustive_codes_exact(4), test_dequant_group_boundaries,
             test_expert_ffn_closed_form_on_selection_weights, test_topk_brute_force_with_ties,
@@ -484,7 +570,8 @@ def test_planted_mistakes_are_caught(monkeypatch):
             test_gating_closed_forms, test_lora_unmerged_equals_merged_and_one_hot, test_shared_gate_half_on_zero_weights,
             test_layer_with_zero_routed_experts_is_half_shared, test_layer_sparse_equals_dense_masked_mixture,
             test_prerouter_closed_forms, test_prerouter_reads_the_executed_experts_under_predicted_routing,
-            test_buckets_brute_force_and_invariants]
+            test_buckets_brute_force_and_invariants, test_lora_on_every_projection_closed_form,
+            test_lora_unmerged_equals_merged_on_up_and_down, test_routed_down_lora_reaches_the_layer_output]
     for name, plant in planted.items():
         plant()
         failed = False
