@@ -537,6 +537,98 @@ def run_reference(args, rank, world):
     }), flush=True)
 
 
+# Stamp slots of moe_stack_opts.trace written by the single-launch kernel (see include/moe.h), and the
+# spans between them that --diag-stack --trace reports.
+TRACE_SPANS = [(0, 1, "A: x received -> RMSNorm done, layer weights landed"),
+               (1, 2, "A: router / shared-gate / LoRA-A rows published"),
+               (2, 3, "A: shared (gate, up) dots + Prerouter u part (during the logits hop)"),
+               (3, 4, "A->B: rest of the logits hop"),
+               (4, 5, "B: top-K (every warp)"),
+               (5, 6, "B: routed copies issued"),
+               (6, 15, "B: copies issued -> first routed rows landed"),
+               (6, 7, "B: (gate, up) pairs done"),
+               (7, 8, "B: hidden published + previous head's output rows (during the hidden hop)"),
+               (8, 9, "B->C: rest of the hidden-vector hop"),
+               (9, 10, "C: hidden vector to pair order, sums, LoRA A, down rows landed"),
+               (10, 11, "C: down sub-rows"),
+               (11, 12, "C: combine, x rows published")]
+
+
+def _span_stats(v) -> str:
+    return (f"mean {v.mean():8.2f}  p90 {np.percentile(v, 90):8.2f}  max {v.max():8.2f}" if v.size
+            else "(not recorded)")
+
+
+def diag_stack(args):
+    """Diagnostic run of the batch-1 stack (no JSON line): the first --layers layers of the 35B shape (or
+    --cfg), --runs tokens on --path; with --trace, per-phase times from the kernel's %globaltimer stamps."""
+    import torch
+    import int4_expert_ffn_top_b200 as M
+    cfg = CONFIGS[args.cfg]
+    stack = M.DeviceStack(cfg, lambda l: inputs.layer(cfg, l), n_layers=args.layers)
+    st = M.StackStructs(stack)
+    ws = M.workspace(M.moe_stack_workspace_size(st, 1, cfg.K, cfg.K))
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    toks = [torch.from_numpy(inputs.bf16_bits_to_f32(inputs.activations(cfg, step=1 + i, T=1))).cuda() for i in range(8)]
+    x = torch.empty_like(toks[0])
+    trace = torch.zeros((stack.n, M.moe_stack_grid(), 16), dtype=torch.int64, device="cuda") if args.trace else None
+    opts = M.stack_opts(path=args.path, trace=trace)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.runs):
+        x.copy_(toks[i % len(toks)])
+        M.moe_stack_decode(st, x, cfg.K, cfg.K, EPS, ws, err_word=err, opts=opts)
+    e1.record()
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise SystemExit(f"moe_stack_decode reported status {int(err.item())}")
+    print(f"{cfg.name}, {stack.n} layers, path {args.path}: {args.runs} tokens, "
+          f"{e0.elapsed_time(e1) / args.runs:.3f} ms per token" + (" (with tracing)" if args.trace else ""))
+    if not args.trace:
+        return
+    raw = trace.cpu().numpy()
+    ok = raw != 0
+    tr = (raw.astype(np.float64) - raw[ok].min()) / 1000.0  # us
+    print("per span, us (mean / p90 / max over CTAs, layers 1..n-1):")
+    for i, j, name in TRACE_SPANS:
+        m = ok[1:, :, i] & ok[1:, :, j]
+        print(f"  {name:78s} {_span_stats((tr[1:, :, j] - tr[1:, :, i])[m])}")
+    m = ok[1:, :, 0] & ok[:-1, :, 12]
+    print(f"  {'C->A: residual hop (own x rows published -> next layer x received)':78s} "
+          f"{_span_stats((tr[1:, :, 0] - tr[:-1, :, 12])[m])}")
+    period = np.diff(tr[:, :, 12].max(axis=1))
+    print(f"layer period (latest CTA's x rows published), us: mean {period.mean():.2f}")
+
+
+def diag_expert(args):
+    """Diagnostic run of one layer's moe_expert_forward (no JSON line): layer 1 of --cfg (default: the 35B-shaped
+    prefill, Zipf-offset router) on --tokens tokens, routed on the GPU, --runs calls; for profilers."""
+    import torch
+    import int4_expert_ffn_top_b200 as M
+    cfg = CONFIGS[args.cfg if args.cfg != CFG_ID else PREFILL_CFG_ID]
+    T, K = args.tokens, cfg.K
+    lay = M.DeviceLayer(cfg, inputs.layer(cfg, 1))
+    u = torch.from_numpy(inputs.activations(cfg, step=9, T=T).view(np.int16)).cuda()
+    logits = torch.empty((T, cfg.E), device="cuda")
+    idx = torch.empty((T, K), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, K), device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    M.moe_route_topk(lay, u, K, logits, idx, w, err_word=err)
+    out = torch.empty((T, cfg.H), device="cuda")
+    ws = M.workspace(M.moe_workspace_size(lay, T, K))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.runs):
+        M.moe_expert_forward(lay, u, K, idx, w, out, 0, ws, err_word=err)
+    e1.record()
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise SystemExit(f"moe_expert_forward reported status {int(err.item())}")
+    ms = e0.elapsed_time(e1) / args.runs
+    print(f"{cfg.name}, one layer's expert forward at {T} tokens: {ms:.3f} ms per call "
+          f"({expert_flops(cfg, T) / (ms / 1000.0) / 1e12:.1f} TFLOP/s)")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -547,8 +639,21 @@ def main():
     ap.add_argument("--no-prefill", action="store_true", help="skip the 3,328-token prefill leg")
     ap.add_argument("--no-extra", action="store_true", help="skip the 8B-shaped and batched decode legs")
     ap.add_argument("--path", type=int, default=0, help="0 auto, 1 per-layer launches, 2 single launch")
+    ap.add_argument("--diag-stack", action="store_true",
+                    help="diagnostic batch-1 stack run (for profilers and the phase trace); prints no JSON line")
+    ap.add_argument("--cfg", type=int, default=CFG_ID, help="--diag-stack: workload shape (gen.configs index)")
+    ap.add_argument("--layers", type=int, default=None, help="--diag-stack: first N layers (default: all)")
+    ap.add_argument("--runs", type=int, default=4, help="--diag-stack: tokens run through the stack")
+    ap.add_argument("--trace", action="store_true", help="--diag-stack: print per-phase times")
+    ap.add_argument("--diag-expert", action="store_true",
+                    help="diagnostic run of one layer's expert forward (for profilers); prints no JSON line")
+    ap.add_argument("--tokens", type=int, default=3328, help="--diag-expert: tokens per call")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.diag_stack:
+        return diag_stack(args)
+    if args.diag_expert:
+        return diag_expert(args)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -27,8 +27,18 @@
  *             NULL = legacy default stream).  A call returns after enqueueing.
  * Errors:     argument/shape checks run on the host before any launch and return
  *             MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED / MOE_ERR_WORKSPACE with
- *             nothing enqueued.  A failed launch returns MOE_ERR_CUDA.  Calls
- *             with device-side bounded waits also report through an error word.
+ *             nothing enqueued.  A failed launch returns MOE_ERR_CUDA.  What the
+ *             device finds while the work runs is reported through an optional
+ *             error word (err_word: one device int32, or NULL to ignore): a call
+ *             stores a nonzero moe_status there if the slot still holds 0 (the
+ *             first error wins) and never clears it, so one word can collect the
+ *             status of many calls; read it after synchronising the stream.
+ *             MOE_ERR_TIMEOUT: a device-side bounded wait gave up (the call's
+ *             outputs are then undefined).  MOE_ERR_RANGE: an activation u is
+ *             outside fp16's range (|u| > 65504); the kernels multiply bf16
+ *             activations as fp16, which holds every bf16 value up to 65504
+ *             exactly down to 2^-14 and rounds smaller ones (gradual underflow),
+ *             so that row's outputs are undefined.
  * Determinism: results are bitwise reproducible for fixed inputs and launch
  *             shapes; no atomics accumulate into outputs.
  * Formats:    bf16/fp16 values are passed as their 16-bit patterns.
@@ -68,7 +78,8 @@ typedef enum {
   MOE_ERR_UNSUPPORTED = 2,  /* shape outside the supported set above */
   MOE_ERR_WORKSPACE = 3,    /* workspace smaller than moe_workspace_size() */
   MOE_ERR_CUDA = 4,         /* a kernel launch failed (cudaGetLastError) */
-  MOE_ERR_TIMEOUT = 5       /* a device-side bounded wait gave up */
+  MOE_ERR_TIMEOUT = 5,      /* a device-side bounded wait gave up */
+  MOE_ERR_RANGE = 6         /* an activation outside the fp16 range the kernels compute in (|u| > 65504) */
 } moe_status;
 
 /* A quantised matrix stored as out_dim row records (see Formats), 16-byte aligned. */
@@ -145,7 +156,7 @@ moe_status moe_rmsnorm_bf16(const float* x, int32_t T, int32_t H, float eps, uin
  * w [T][K] fp32.  Two launches.
  */
 moe_status moe_route_topk(const moe_layer* L, const uint16_t* u, int32_t T, int32_t K,
-                          float* logits, int32_t* idx, float* w, void* stream);
+                          float* logits, int32_t* idx, float* w, int32_t* err_word, void* stream);
 
 /*
  * Routed experts + shared expert + combine for T tokens with K experts each
@@ -169,12 +180,13 @@ moe_status moe_route_topk(const moe_layer* L, const uint16_t* u, int32_t T, int3
  *   tensor cores over per-expert token buckets, where the dequantised weights
  *   and the SwiGLU output are rounded to fp16 and products accumulate in fp32.
  * Bounded waits: every device-side wait of the tensor-core path gives up after
- *   2 s, so a call always completes; a wait that ran out leaves the output
- *   incomplete and is not reflected in the (asynchronous) return status.
+ *   2 s, so a call always completes; a wait that ran out stores MOE_ERR_TIMEOUT
+ *   in err_word (see Errors) and leaves the output undefined.
  */
 moe_status moe_expert_forward(const moe_layer* L, const uint16_t* u, int32_t T, int32_t K,
                               const int32_t* idx, const float* w, void* out, int32_t out_mode,
-                              int32_t* perm_out, void* workspace, size_t ws_bytes, void* stream);
+                              int32_t* perm_out, void* workspace, size_t ws_bytes, int32_t* err_word,
+                              void* stream);
 
 /* Scratch bytes moe_expert_forward needs for (L, T, K) (host); 0 for a NULL
  * layer, T < 0, T > MOE_MAX_TOKENS or K < 1. */
@@ -190,7 +202,7 @@ size_t moe_workspace_size(const moe_layer* L, int32_t T, int32_t K);
  */
 moe_status prerouter_predict(const moe_prerouter* head, const uint16_t* u, const int32_t* sel,
                              int32_t T, int32_t K, int32_t K_next, int32_t* pred, float* scores,
-                             void* workspace, size_t ws_bytes, void* stream);
+                             void* workspace, size_t ws_bytes, int32_t* err_word, void* stream);
 
 /* Scratch bytes prerouter_predict needs for T tokens (host); 0 for a NULL head,
  * T < 0 or T > MOE_MAX_TOKENS. */
@@ -198,20 +210,25 @@ size_t prerouter_workspace_size(const moe_prerouter* head, int32_t T);
 
 /* Options of moe_stack_decode (NULL = all defaults). */
 typedef struct {
-  int64_t timeout_ns;  /* bound on every device-side wait of the single-launch path; <= 0: 1 s */
+  int64_t timeout_ns;  /* bound on every device-side wait (single-launch kernel; per-layer grouped GEMMs);
+                          <= 0: 1 s for the single launch, 2 s for the GEMMs */
   int32_t path;        /* 0: automatic; 1: per-layer launches; 2: single-launch kernel (MOE_ERR_UNSUPPORTED if
-                          the shapes are not eligible) */
-  int32_t test_drop_layer;  /* test hook for the timeout path, 0 = off; L > 0: CTA test_drop_cta of the */
-  int32_t test_drop_cta;    /*   single-launch kernel never publishes its residual rows of layer L-1, so the
-                                 other CTAs' bounded waits run out and err_word reports MOE_ERR_TIMEOUT */
+                          the shapes are not eligible); 3: the first-generation single-launch kernel (kept for
+                          comparison) */
+  int32_t test_drop_layer;  /* test hook for the timeout path, 0 = off; L > 0: on the single-launch path CTA */
+  int32_t test_drop_cta;    /*   test_drop_cta never publishes its residual rows of layer L-1, so the other CTAs'
+                                 bounded waits run out; on the per-layer path the CTA test_drop_cta of layer L-1's
+                                 gate/up grouped GEMM (tensor-core path only) never marks its first operand stage
+                                 full, so the MMA's bounded wait runs out.  Either way err_word reports
+                                 MOE_ERR_TIMEOUT */
   int64_t* trace;           /* optional device buffer [n_layers][moe_stack_grid()][16] of int64 %globaltimer
-                               stamps (ns) per CTA of the single-launch kernel, written by its thread 0:
-                               0 residual received, 1 router rows published, 2 logits received, 3 routed
-                               copies issued (after the block barrier), 4 hidden vector published, 5 hidden
-                               vector received, 6 residual rows published, 7 layer end, 8 RMSNorm done,
-                               9 token-independent weights landed, 10 top-K done, 11 copy barriers armed,
-                               12 copies issued, 13 first routed pair landed (if thread 0 waits for it),
-                               14 down prologue done, 15 routed down rows landed */
+                               stamps (ns) per CTA of the single-launch kernel (paths 0 and 2), written by its
+                               thread 0: 0 x received, 1 RMSNorm done and layer weights landed, 2 router /
+                               shared-gate / LoRA-A rows published, 3 shared (gate, up) dots and Prerouter u part
+                               done, 4 logits received, 5 top-K done, 6 routed copies issued, 7 (gate, up) pairs
+                               done, 8 hidden values published and previous head's output rows done, 9 hidden
+                               vector received, 10 down rows landed, 11 down sub-rows done, 12 x rows published,
+                               15 first routed pair landed (if thread 0's warp computes it) */
 } moe_stack_opts;
 
 /* Grid size (CTAs) the single-launch stack kernel uses on the current device (host). */
@@ -238,9 +255,11 @@ int32_t moe_stack_grid(void);
  * K_next == K, the whole stack runs as ONE cooperative kernel launch (one CTA
  * per SM; layer-internal exchanges through device memory with bounded waits);
  * otherwise as per-layer launches of the kernels behind the per-layer entry
- * points.  err_word (device, optional): set to 0 at the start of the call and
- * to MOE_ERR_TIMEOUT if a wait of the single-launch kernel gave up (its
- * outputs are then undefined); read it after synchronising the stream.
+ * points.  err_word (device, optional): set to 0 at the start of the call,
+ * then collects the device-side status of every launch of the stack (see
+ * Errors): MOE_ERR_TIMEOUT if a bounded wait of the single-launch kernel or of
+ * a per-layer grouped GEMM gave up (the outputs are then undefined); read it
+ * after synchronising the stream.
  * workspace >= moe_stack_workspace_size(...) bytes, 256-byte aligned; contents
  * on entry do not matter.
  */
@@ -272,8 +291,11 @@ size_t moe_stack_workspace_size(const moe_layer* layers, const moe_prerouter* he
  *   MOE_NOALLOC_SCRATCH_BYTES (nothing is enqueued); otherwise as
  *   moe_expert_forward.
  * Set-up: the first call on a device (with that device current) looks up the
- *   array's device address once; make that first call before any stream
- *   capture on that device.
+ *   array's device address once and keeps it for the life of the process (a
+ *   failed lookup is retried by the next call); make that first call before
+ *   any stream capture on that device.  A process that calls cudaDeviceReset
+ *   must not use this entry point afterwards: the library's module is then
+ *   reloaded, possibly elsewhere, and the kept address is stale.
  * Sharing: all calls in the process share the one array per device and it
  *   keeps the previous call's contents.  Every scratch word the kernels read
  *   is written earlier in the same call, so nothing needs clearing; but calls
@@ -284,7 +306,7 @@ size_t moe_stack_workspace_size(const moe_layer* layers, const moe_prerouter* he
 
 moe_status moe_expert_forward_noalloc(const moe_layer* L, const uint16_t* u, int32_t T, int32_t K,
                                       const int32_t* idx, const float* w, void* out, int32_t out_mode,
-                                      int32_t* perm_out, void* stream);
+                                      int32_t* perm_out, int32_t* err_word, void* stream);
 
 /* MOE_NOALLOC_SCRATCH_BYTES as compiled into the library (host). */
 size_t moe_noalloc_scratch_bytes(void);

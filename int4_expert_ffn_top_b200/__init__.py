@@ -109,11 +109,12 @@ def moe_rmsnorm_bf16(x: torch.Tensor, eps: float, u: torch.Tensor, stream=None):
 
 
 def moe_route_topk(layer: DeviceLayer, u: torch.Tensor, K: int, logits: torch.Tensor, idx: torch.Tensor,
-                   w: torch.Tensor, stream=None):
+                   w: torch.Tensor, err_word: torch.Tensor | None = None, stream=None):
     fn, L = "moe_route_topk", layer.struct
     T = _rows(fn, "u", u, L.H, BF16_BITS)
     args = (_arg(fn, "logits", logits, F32, T * L.E), _arg(fn, "idx", idx, I32, T * K), _arg(fn, "w", w, F32, T * K))
-    _check(fn, lib().moe_route_topk(ctypes.byref(L), _p(u), T, K, *args, _stream(stream)))
+    err = _arg(fn, "err_word", err_word, I32, 1, optional=True)
+    _check(fn, lib().moe_route_topk(ctypes.byref(L), _p(u), T, K, *args, err, _stream(stream)))
 
 
 def moe_workspace_size(layer: DeviceLayer, T: int, K: int) -> int:
@@ -130,10 +131,11 @@ def _expert_args(fn: str, layer: DeviceLayer, u, K: int, idx, w, out, out_mode: 
 
 def moe_expert_forward(layer: DeviceLayer, u: torch.Tensor, K: int, idx: torch.Tensor, w: torch.Tensor,
                        out: torch.Tensor, out_mode: int, workspace: torch.Tensor, perm_out: torch.Tensor | None = None,
-                       stream=None):
+                       err_word: torch.Tensor | None = None, stream=None):
     fn = "moe_expert_forward"
     T, args = _expert_args(fn, layer, u, K, idx, w, out, out_mode, perm_out)
-    _check(fn, lib().moe_expert_forward(ctypes.byref(layer.struct), _p(u), T, K, *args, *_ws(fn, workspace),
+    err = _arg(fn, "err_word", err_word, I32, 1, optional=True)
+    _check(fn, lib().moe_expert_forward(ctypes.byref(layer.struct), _p(u), T, K, *args, *_ws(fn, workspace), err,
                                         _stream(stream)))
 
 
@@ -142,7 +144,8 @@ def moe_noalloc_scratch_bytes() -> int:
 
 
 def moe_expert_forward_noalloc(layer: DeviceLayer, u: torch.Tensor, K: int, idx: torch.Tensor, w: torch.Tensor,
-                               out: torch.Tensor, out_mode: int, perm_out: torch.Tensor | None = None, stream=None):
+                               out: torch.Tensor, out_mode: int, perm_out: torch.Tensor | None = None,
+                               err_word: torch.Tensor | None = None, stream=None):
     """moe_expert_forward without a workspace: scratch is the library's fixed per-device array.
 
     For callers that cannot allocate device memory.  Calls share that array, so
@@ -151,7 +154,8 @@ def moe_expert_forward_noalloc(layer: DeviceLayer, u: torch.Tensor, K: int, idx:
     """
     fn = "moe_expert_forward_noalloc"
     T, args = _expert_args(fn, layer, u, K, idx, w, out, out_mode, perm_out)
-    _check(fn, lib().moe_expert_forward_noalloc(ctypes.byref(layer.struct), _p(u), T, K, *args, _stream(stream)))
+    err = _arg(fn, "err_word", err_word, I32, 1, optional=True)
+    _check(fn, lib().moe_expert_forward_noalloc(ctypes.byref(layer.struct), _p(u), T, K, *args, err, _stream(stream)))
 
 
 def prerouter_workspace_size(head: DeviceHead, T: int) -> int:
@@ -159,7 +163,7 @@ def prerouter_workspace_size(head: DeviceHead, T: int) -> int:
 
 
 def prerouter_predict(head: DeviceHead, u: torch.Tensor, sel: torch.Tensor, K_next: int, pred: torch.Tensor,
-                      scores: torch.Tensor, workspace: torch.Tensor, stream=None):
+                      scores: torch.Tensor, workspace: torch.Tensor, err_word: torch.Tensor | None = None, stream=None):
     fn, P = "prerouter_predict", head.struct
     if not isinstance(sel, torch.Tensor) or sel.dim() != 2:
         raise ValueError(f"{fn}: sel must be [T, K]")
@@ -168,7 +172,8 @@ def prerouter_predict(head: DeviceHead, u: torch.Tensor, sel: torch.Tensor, K_ne
         raise ValueError(f"{fn}: u has {u.shape[0]} rows, sel has {T}")
     args = (_arg(fn, "sel", sel, I32), K_next, _arg(fn, "pred", pred, I32, T * K_next),
             _arg(fn, "scores", scores, F32, T * P.E_next))
-    _check(fn, lib().prerouter_predict(ctypes.byref(P), _p(u), args[0], T, K, *args[1:], *_ws(fn, workspace),
+    err = _arg(fn, "err_word", err_word, I32, 1, optional=True)
+    _check(fn, lib().prerouter_predict(ctypes.byref(P), _p(u), args[0], T, K, *args[1:], *_ws(fn, workspace), err,
                                        _stream(stream)))
 
 

@@ -8,7 +8,7 @@ from ctypes import POINTER, c_char_p, c_float, c_int32, c_int64, c_size_t, c_voi
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libmoe.so")
 
-MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = range(6)
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_RANGE = range(7)
 MOE_MAX_TOKENS = 524280  # most tokens one call takes
 
 
@@ -41,19 +41,19 @@ SIGNATURES = {
     "moe_expert_block_bytes": (c_size_t, [c_int32, c_int32]),
     "moe_rmsnorm_bf16": (c_int32, [c_void_p, c_int32, c_int32, c_float, c_void_p, c_void_p]),
     "moe_route_topk": (c_int32, [POINTER(moe_layer), c_void_p, c_int32, c_int32, c_void_p, c_void_p, c_void_p,
-                                 c_void_p]),
+                                 c_void_p, c_void_p]),
     "moe_expert_forward": (c_int32, [POINTER(moe_layer), c_void_p, c_int32, c_int32, c_void_p, c_void_p, c_void_p,
-                                     c_int32, c_void_p, c_void_p, c_size_t, c_void_p]),
+                                     c_int32, c_void_p, c_void_p, c_size_t, c_void_p, c_void_p]),
     "moe_workspace_size": (c_size_t, [POINTER(moe_layer), c_int32, c_int32]),
     "prerouter_predict": (c_int32, [POINTER(moe_prerouter), c_void_p, c_void_p, c_int32, c_int32, c_int32, c_void_p,
-                                    c_void_p, c_void_p, c_size_t, c_void_p]),
+                                    c_void_p, c_void_p, c_size_t, c_void_p, c_void_p]),
     "prerouter_workspace_size": (c_size_t, [POINTER(moe_prerouter), c_int32]),
     "moe_stack_decode": (c_int32, [POINTER(moe_layer), POINTER(moe_prerouter), c_int32, c_int32, c_int32, c_int32,
                                    c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int32,
                                    c_void_p, POINTER(moe_stack_opts), c_void_p,
                                    c_size_t, c_void_p]),
     "moe_expert_forward_noalloc": (c_int32, [POINTER(moe_layer), c_void_p, c_int32, c_int32, c_void_p, c_void_p,
-                                             c_void_p, c_int32, c_void_p, c_void_p]),
+                                             c_void_p, c_int32, c_void_p, c_void_p, c_void_p]),
     "moe_noalloc_scratch_bytes": (c_size_t, []),
     "moe_stack_grid": (c_int32, []),
     "moe_stack_workspace_size": (c_size_t, [POINTER(moe_layer), POINTER(moe_prerouter), c_int32, c_int32, c_int32,

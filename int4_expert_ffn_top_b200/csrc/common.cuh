@@ -80,19 +80,22 @@ MOE_DEV void int8_word_to_h2(uint32_t w, uint32_t (&o)[2]) {
 
 // 32 nibbles (one 16-byte chunk = half a group) dotted with 32 activations held
 // as 16 half2 in "pair order" (for each 8-block: (u_j, u_{j+4}), j = 0..3).
+// Two independent accumulation chains (words 0-1 and 2-3), added at the end.
 MOE_DEV float dot_chunk_int4(const uint4& wq, const uint4* up, float acc) {
   const uint32_t ws[4] = {wq.x, wq.y, wq.z, wq.w};
+  float a2[2] = {acc, 0.f};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     uint32_t q[4];
     int4_word_to_h2(ws[i], q);
     const uint4 u = up[i];
-    acc = dot2_mix(q[0], u.x, acc);
-    acc = dot2_mix(q[1], u.y, acc);
-    acc = dot2_mix(q[2], u.z, acc);
-    acc = dot2_mix(q[3], u.w, acc);
+    float& a = a2[i >> 1];
+    a = dot2_mix(q[0], u.x, a);
+    a = dot2_mix(q[1], u.y, a);
+    a = dot2_mix(q[2], u.z, a);
+    a = dot2_mix(q[3], u.w, a);
   }
-  return acc;
+  return a2[0] + a2[1];
 }
 
 // 16 bytes (a quarter group) of an 8-bit matrix dotted with 16 activations held
@@ -127,6 +130,15 @@ MOE_DEV uint4 ldg_stream(const void* p) {
                : "l"(p));
   return v;
 }
+
+// Device-side status report into an optional error word: the first nonzero status wins.
+MOE_DEV void report(int* err, int code) {
+  if (err) atomicCAS(err, 0, code);
+}
+
+// Largest finite fp16 value: bf16 activations above it in magnitude (or not finite) cannot be
+// multiplied as fp16 (moe_status MOE_ERR_RANGE).
+constexpr float kF16Max = 65504.0f;
 
 MOE_DEV float half_bits_to_float(uint16_t h) { return __half2float(__ushort_as_half(h)); }
 MOE_DEV float bf16_bits_to_float(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }

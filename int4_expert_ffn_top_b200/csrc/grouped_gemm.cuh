@@ -15,7 +15,9 @@
 //  * warps 0-3 then read the accumulator with tcgen05.ld and run the epilogue
 //    (SwiGLU for gate/up, gating-weight scaling for down, unmerged LoRA
 //    deltas), staging through shared memory for coalesced stores.
-// Every wait is bounded; on timeout the kernel records MOE_ERR_TIMEOUT.
+// Every wait is bounded; a wait that runs out stops the CTA from issuing more
+// copies or MMAs, lets what it issued finish (bounded) and records
+// MOE_ERR_TIMEOUT in the error word.
 #pragma once
 
 #include <cuda.h>
@@ -72,6 +74,7 @@ struct Args {
   float lora_scale;
   int* err;
   long long timeout_ns;
+  int drop_tile;  // test hook: the CTA of this tile never marks its first operand stage full (-1: off)
 };
 
 MOE_DEV uint32_t sa(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
@@ -238,25 +241,37 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         s_raw = sc[kt + 1];
         b_raw = bi[kt + 1];
       }
-      if (!bar_wait(empty + s, ph ^ 1u, a.timeout_ns)) fail = 1;
+      if (!bar_wait(empty + s, ph ^ 1u, a.timeout_ns)) {  // never overwrite a stage the MMA may still read
+        fail = 1;
+        break;
+      }
       uint8_t* d = dst_row + s * A_STAGE;
       const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
       for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(d + ((c ^ (r & 7)) << 4)) = dequant_word(ws[c], s2, b2);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      bar_arrive(full_a + s);
+      if (!(kt == 0 && r == 0 && static_cast<int>(blockIdx.x) == a.drop_tile)) bar_arrive(full_a + s);
     }
   } else if (warp == 4) {
     // ---------------------------------------------------------------- token tiles by TMA
     if (lane == 0) {
+      int issued = 0;
 #pragma unroll 1
       for (int kt = 0; kt < KT; ++kt) {
         const int s = kt % STAGES;
         const uint32_t ph = (kt / STAGES) & 1u;
-        if (!bar_wait(empty + s, ph ^ 1u, a.timeout_ns)) fail = 1;
+        if (!bar_wait(empty + s, ph ^ 1u, a.timeout_ns)) {
+          fail = 1;
+          break;
+        }
         bar_expect_tx(full_b + s, B_STAGE);
         tma_load_2d(smB + s * B_STAGE, &tmap_b, kt * BK, tile.row0, full_b + s);
+        issued = kt + 1;
       }
+      if (fail)  // let the loads already issued land before the CTA can exit
+#pragma unroll 1
+        for (int kt = issued - STAGES > 0 ? issued - STAGES : 0; kt < issued; ++kt)
+          bar_wait(full_b + kt % STAGES, (kt / STAGES) & 1u, a.timeout_ns);
     }
   } else {
     // ---------------------------------------------------------------- MMA issue (one thread)
@@ -267,8 +282,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       for (int kt = 0; kt < KT; ++kt) {
         const int s = kt % STAGES;
         const uint32_t ph = (kt / STAGES) & 1u;
-        if (!bar_wait(full_a + s, ph, a.timeout_ns)) fail = 1;
-        if (!bar_wait(full_b + s, ph, a.timeout_ns)) fail = 1;
+        if (!bar_wait(full_a + s, ph, a.timeout_ns) || !bar_wait(full_b + s, ph, a.timeout_ns)) {
+          fail = 1;  // issue nothing more; the commit below still tracks what was issued
+          break;
+        }
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const uint32_t a0 = sa(smA + s * A_STAGE), b0 = sa(smB + s * B_STAGE);
 #pragma unroll
@@ -289,6 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
     uint16_t* stage = reinterpret_cast<uint16_t*>(sm);  // reuse the pipeline buffers (all MMAs are done)
     const int r = a.lora_r;
     if (a.epi == EPI_SWIGLU) {
+      bool range_bad = false;  // a SwiGLU output fp16 cannot hold: MOE_ERR_RANGE
       const bool up = (L & 1) != 0;
       const int j = o >> 1;
       // LoRA B row of this output row (gate or up), r <= 32 values
@@ -312,10 +330,14 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
             x = fmaf(a.lora_scale, d, x);
           }
           const float partner = __shfl_xor_sync(0xffffffffu, x, 1);
-          if (!up && c0 + t < tile.n)
-            stage[(c0 + t) * 64 + (L >> 1)] = __half_as_ushort(__float2half_rn(silu(x) * partner));
+          if (!up && c0 + t < tile.n) {
+            const float hv = silu(x) * partner;
+            range_bad |= !(fabsf(hv) <= kF16Max);
+            stage[(c0 + t) * 64 + (L >> 1)] = __half_as_ushort(__float2half_rn(hv));
+          }
         }
       }
+      if (range_bad) report(a.err, 6);
       asm volatile("bar.sync 1, 128;" ::: "memory");
       // coalesced stores: row (row0 + t), columns [mt*64, mt*64 + 64)
       for (int i = tid; i < tile.n * 8; i += 128) {
@@ -357,7 +379,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       }
     }
   }
-  if (fail) atomicExch(a.err, 5);
+  if (fail) report(a.err, 5);
+  if (warp == 5 && lane == 0 && fail)  // the accumulator must be idle before its columns are released
+    bar_wait(acc_full, 0, a.timeout_ns);
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   if (warp == 5) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));

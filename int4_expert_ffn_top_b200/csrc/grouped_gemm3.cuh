@@ -1,0 +1,470 @@
+// Grouped GEMM on the 5th-generation tensor cores (tcgen05) for many-token
+// batches: persistent, warp-specialised, int4 weight stream by TMA.
+//
+// Per expert bucket D[o][t] = sum_k W[o][k] * X[t][k] ("swap AB": 128 weight
+// rows are the MMA M side, the bucket's tokens the N side).  A tile is 128
+// weight rows x up to 128 tokens; K advances one quantisation group (64) per
+// step.  One CTA per SM walks the device-built tile list (tiles c, c + grid,
+// ...), and every role runs the same sequence of (tile, step), so the pipeline
+// stays full across tiles:
+//  * warp 0, one lane (TMA): per tile the fp16 scales and biases of its 128 rows
+//    (a box of a 3-D byte map {record bytes, rows, experts} over the expert
+//    pool, two buffers); per step the 32 code bytes of each row (a box of a
+//    second map over the same bytes: 4 KB, dense [row][32 B], eight stages) and
+//    the step's token rows (2-D map, 128-byte swizzle, boxes of 32 rows, only as
+//    many as the tile has tokens);
+//  * warps 2..9 dequantise: thread (row r, half h) reads 16 code bytes (a warp
+//    reads 512 contiguous bytes), forms w = q*s + b in fp16 (one rounding) and
+//    stores four 16-byte chunks into the 128-byte-swizzled K-major A stage.  K
+//    inside each 8-element block is in "pair order" (q_j, q_{j+4}), the order
+//    the magic-exponent unpacking produces; the token operand is stored in the
+//    same order, so the products are those of the plain order;
+//  * warp 1, one lane (MMA): tcgen05.mma kind::f16 into one of two 128-column
+//    TMEM accumulators (tiles alternate), committing stage releases and
+//    accumulator-ready barriers;
+//  * warps 10..13 (epilogue, TMEM lane quadrant = warp % 4): drain the finished
+//    accumulator with tcgen05.ld while the next tile's main loop runs: SwiGLU of
+//    interleaved gate/up rows (output in pair order, the next GEMM's token
+//    operand) or the down projection's LoRA delta and gating weight; staged in
+//    shared memory for coalesced fp16 stores; then the accumulator is released.
+// Every wait is bounded: a role whose wait runs out stops issuing copies or
+// MMAs and records MOE_ERR_TIMEOUT; before the CTA leaves, the copies and MMAs
+// it issued are waited for (bounded).
+#pragma once
+
+#include "grouped_gemm.cuh"
+
+namespace moe {
+namespace gg3 {
+
+using gg::bar_arrive;
+using gg::bar_expect_tx;
+using gg::bar_init;
+using gg::bar_test;
+using gg::bar_wait;
+using gg::EPI_DOWN;
+using gg::EPI_SWIGLU;
+using gg::instr_desc;
+using gg::mma_commit;
+using gg::mma_f16;
+using gg::sa;
+using gg::smem_desc;
+using gg::tma_load_2d;
+using gg::tmem_ld32;
+using gg::Tile;
+
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int BK = 64;
+constexpr int BROWS = 32;   // token rows per TMA box
+constexpr int RSTAGES = 8;  // raw code stages (4 KB each): the weight bytes in flight per SM
+constexpr int BSTAGES = 3;  // token stages (16 KB each)
+constexpr int ASTAGES = 3;  // dequantised weight stages (16 KB each)
+constexpr int kDqWarps = 8;
+constexpr int kDq = 32 * kDqWarps;
+constexpr int kEpi = 128;
+constexpr int kThreads = 64 + kDq + kEpi;  // TMA warp, MMA warp, dequant warps, epilogue warps
+constexpr int RAW_STAGE = BM * 32;
+constexpr int A_STAGE = BM * BK * 2;
+constexpr int B_STAGE = BN * BK * 2;
+constexpr int SB_MAX = BM * 256;           // scales + biases of 128 rows, K <= 4096
+constexpr int STAGE_OUT = BN * BM * 2;     // epilogue staging: up to 128 tokens x 128 fp16
+constexpr uint32_t TMEM_COLS = 256;        // two 128-column accumulators
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + ASTAGES * A_STAGE;
+constexpr int OFF_RAW = OFF_B + BSTAGES * B_STAGE;
+constexpr int OFF_OUT = OFF_RAW + RSTAGES * RAW_STAGE;
+constexpr int OFF_SB = OFF_OUT + STAGE_OUT;
+
+// Bytes per row of the scale/bias box: the K/64 scales and K/64 biases (4*K/64 bytes), at least one 16-byte
+// TMA unit (the row record's zero padding covers the rest).
+__host__ __device__ constexpr int sb_row_bytes(int K) { return (4 * (K / 64) + 15) / 16 * 16; }
+// Dynamic shared memory for reduction length K (two scale/bias buffers, barriers, alignment slack).
+__host__ __device__ constexpr int smem_bytes(int K) { return OFF_SB + 2 * BM * sb_row_bytes(K) + 512 + 1024; }
+
+struct Args {
+  const Tile* tiles;
+  const int* n_tiles;
+  int E;
+  int K;
+  int epi;
+  uint16_t* out;
+  int out_ld;
+  const float* row_scale;
+  const uint16_t* lora_B1;
+  const float* lora_t1;
+  const uint16_t* lora_B2;
+  const float* lora_t2;
+  const uint16_t* lora_Bex;
+  int lora_r;
+  float lora_scale;
+  int* err;
+  long long timeout_ns;
+  int drop_tile;  // test hook: the CTA working on this tile never marks its first weight stage full (-1: off)
+};
+
+// 3-D byte maps {record bytes, rows, experts} over the weight matrix of every expert block (pool) and of the
+// shared expert's block (one expert): boxes of the 32 code bytes of one group x 128 rows, and of the
+// scale/bias bytes x 128 rows.  2-D fp16 map of the token operand [rows][K], boxes of 64 x 32, 128-byte swizzle.
+struct Maps {
+  CUtensorMap pool_codes, pool_sb, shared_codes, shared_sb, tokens;
+};
+
+MOE_DEV void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(sa(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(sa(bar))
+      : "memory");
+}
+
+// One int4 word -> 8 fp16 weights q*s + b in pair order ((w_j, w_{j+4}) for j = 0..3).  The codes come out of
+// the magic-exponent unpacking exactly (lo nibbles: (1024 + q) - 1024; hi nibbles: (1024 + 16 q) / 16 - 64).
+MOE_DEV uint4 dequant_pair_order(uint32_t w, __half2 s2, __half2 b2) {
+  const uint32_t kMagic = 0x64006400u;
+  const uint32_t lo0 = lop_and_or(w, 0x000F000Fu, kMagic);
+  const uint32_t hi0 = lop_and_or(w, 0x00F000F0u, kMagic);
+  const uint32_t w8 = w >> 8;
+  const uint32_t lo1 = lop_and_or(w8, 0x000F000Fu, kMagic);
+  const uint32_t hi1 = lop_and_or(w8, 0x00F000F0u, kMagic);
+  const __half2 k1024 = __half2half2(__ushort_as_half(0x6400));  // 1024
+  const __half2 k16th = __half2half2(__ushort_as_half(0x2C00));  // 1/16
+  const __half2 km64 = __half2half2(__ushort_as_half(0xD400));   // -64
+  const __half2 q0 = __hsub2(as_h2(lo0), k1024), q1 = __hfma2(as_h2(hi0), k16th, km64);
+  const __half2 q2 = __hsub2(as_h2(lo1), k1024), q3 = __hfma2(as_h2(hi1), k16th, km64);
+  return make_uint4(h2_bits(__hfma2(q0, s2, b2)), h2_bits(__hfma2(q1, s2, b2)), h2_bits(__hfma2(q2, s2, b2)),
+                    h2_bits(__hfma2(q3, s2, b2)));
+}
+
+MOE_DEV uint32_t parity(int count, int stages) { return static_cast<uint32_t>(count / stages) & 1u; }
+
+// OR of v over the 128 epilogue threads (named barrier 1), so that they take the same branch.
+MOE_DEV bool epi_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n barrier.cta.red.or.pred q, 1, 128, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return r != 0;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid_constant__ Maps maps,
+                                                                    const __grid_constant__ Args a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int KT = a.K / BK;
+  const int SB_ROW = sb_row_bytes(a.K);  // scales at byte 0, biases at byte 2*KT of a row
+  uint8_t* smA = sm + OFF_A;
+  uint8_t* smB = sm + OFF_B;
+  uint8_t* smRaw = sm + OFF_RAW;
+  uint16_t* stage = reinterpret_cast<uint16_t*>(sm + OFF_OUT);
+  uint8_t* smSB = sm + OFF_SB;  // two buffers of BM * SB_ROW bytes
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smSB + 2 * BM * SB_ROW);
+  uint64_t* raw_full = bars;
+  uint64_t* raw_empty = raw_full + RSTAGES;
+  uint64_t* b_full = raw_empty + RSTAGES;
+  uint64_t* b_empty = b_full + BSTAGES;
+  uint64_t* a_full = b_empty + BSTAGES;
+  uint64_t* a_empty = a_full + ASTAGES;
+  uint64_t* sb_full = a_empty + ASTAGES;  // [2]
+  uint64_t* sb_empty = sb_full + 2;       // [2]
+  uint64_t* acc_full = sb_empty + 2;      // [2]
+  uint64_t* acc_empty = acc_full + 2;     // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+
+  const int n_tiles = *a.n_tiles;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < RSTAGES; ++s) {
+      bar_init(raw_full + s, 1);
+      bar_init(raw_empty + s, kDq);
+    }
+    for (int s = 0; s < BSTAGES; ++s) {
+      bar_init(b_full + s, 1);
+      bar_init(b_empty + s, 1);
+    }
+    for (int s = 0; s < ASTAGES; ++s) {
+      bar_init(a_full + s, kDq);
+      bar_init(a_empty + s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      bar_init(sb_full + s, 1);
+      bar_init(sb_empty + s, kDq);
+      bar_init(acc_full + s, 1);
+      bar_init(acc_empty + s, kEpi);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(sa(tmem_slot)),
+                 "r"(TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tmem_slot;
+  int fail = 0;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int n_raw = 0, n_b = 0, n_sb = 0;  // copies issued so far (stage counters)
+#pragma unroll 1
+      for (int ti = blockIdx.x; ti < n_tiles && !fail; ti += gridDim.x) {
+        const Tile tile = a.tiles[ti];
+        const bool sh = tile.e >= a.E;
+        const CUtensorMap* cmap = sh ? &maps.shared_codes : &maps.pool_codes;
+        const CUtensorMap* smap = sh ? &maps.shared_sb : &maps.pool_sb;
+        const int ez = sh ? 0 : tile.e, y = tile.mt * BM;
+        const int tb = n_sb & 1;
+        if (!bar_wait(sb_empty + tb, parity(n_sb, 2) ^ 1u, a.timeout_ns)) {
+          fail = 1;
+          break;
+        }
+        bar_expect_tx(sb_full + tb, static_cast<uint32_t>(BM * SB_ROW));
+        tma_load_3d(smSB + tb * BM * SB_ROW, smap, a.K / 2, y, ez, sb_full + tb);
+        ++n_sb;
+        const int nb = (tile.n + BROWS - 1) / BROWS;
+#pragma unroll 1
+        for (int kt = 0; kt < KT; ++kt) {
+          const int rs = n_raw % RSTAGES, bs = n_b % BSTAGES;
+          if (!bar_wait(raw_empty + rs, parity(n_raw, RSTAGES) ^ 1u, a.timeout_ns)) {
+            fail = 1;
+            break;
+          }
+          bar_expect_tx(raw_full + rs, RAW_STAGE);
+          tma_load_3d(smRaw + rs * RAW_STAGE, cmap, kt * 32, y, ez, raw_full + rs);
+          ++n_raw;
+          if (!bar_wait(b_empty + bs, parity(n_b, BSTAGES) ^ 1u, a.timeout_ns)) {
+            fail = 1;
+            break;
+          }
+          bar_expect_tx(b_full + bs, static_cast<uint32_t>(nb * BROWS * BK * 2));
+#pragma unroll 1
+          for (int i = 0; i < nb; ++i)
+            tma_load_2d(smB + bs * B_STAGE + i * BROWS * BK * 2, &maps.tokens, kt * BK, tile.row0 + i * BROWS,
+                        b_full + bs);
+          ++n_b;
+        }
+      }
+      if (fail) {  // let the copies already issued land before the CTA can leave
+#pragma unroll 1
+        for (int q = n_raw > RSTAGES ? n_raw - RSTAGES : 0; q < n_raw; ++q)
+          bar_wait(raw_full + q % RSTAGES, parity(q, RSTAGES), a.timeout_ns);
+#pragma unroll 1
+        for (int q = n_b > BSTAGES ? n_b - BSTAGES : 0; q < n_b; ++q)
+          bar_wait(b_full + q % BSTAGES, parity(q, BSTAGES), a.timeout_ns);
+#pragma unroll 1
+        for (int q = n_sb > 2 ? n_sb - 2 : 0; q < n_sb; ++q) bar_wait(sb_full + (q & 1), parity(q, 2), a.timeout_ns);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issue (one thread)
+    if (lane == 0) {
+      int g = 0, it = 0, last_ab = -1;
+      uint32_t last_par = 0;
+#pragma unroll 1
+      for (int ti = blockIdx.x; ti < n_tiles && !fail; ti += gridDim.x, ++it) {
+        const Tile tile = a.tiles[ti];
+        const int ab = it & 1;
+        if (!bar_wait(acc_empty + ab, parity(it, 2) ^ 1u, a.timeout_ns)) {
+          fail = 1;
+          break;
+        }
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t d = tmem + static_cast<uint32_t>(ab * BM);
+        const uint32_t idesc = instr_desc((tile.n + 15) & ~15);
+#pragma unroll 1
+        for (int kt = 0; kt < KT; ++kt, ++g) {
+          const int as = g % ASTAGES, bs = g % BSTAGES;
+          if (!bar_wait(a_full + as, parity(g, ASTAGES), a.timeout_ns) ||
+              !bar_wait(b_full + bs, parity(g, BSTAGES), a.timeout_ns)) {
+            fail = 1;
+            break;
+          }
+          asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+          const uint32_t a0 = sa(smA + as * A_STAGE), b0 = sa(smB + bs * B_STAGE);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_f16(d, smem_desc(a0 + kk * 32), smem_desc(b0 + kk * 32), idesc, (kt | kk) != 0);
+          mma_commit(a_empty + as);
+          mma_commit(b_empty + bs);
+        }
+        mma_commit(acc_full + ab);  // also on failure: completes once every MMA issued into this buffer has
+        last_ab = ab;
+        last_par = parity(it, 2);
+      }
+      // never release TMEM with MMAs in flight: wait for the last commit
+      if (fail && last_ab >= 0) bar_wait(acc_full + last_ab, last_par, a.timeout_ns);
+    }
+  } else if (warp < 2 + kDqWarps) {
+    // ---------------------------------------------------------------- dequantising warps
+    const int d = tid - 64;
+    const int r = d >> 1, h = d & 1;
+    const bool vec8 = (KT & 7) == 0;
+    int g = 0, it = 0;
+#pragma unroll 1
+    for (int ti = blockIdx.x; ti < n_tiles && !fail; ti += gridDim.x, ++it) {
+      const int tb = it & 1;
+      const uint16_t* sbr = reinterpret_cast<const uint16_t*>(smSB + tb * BM * SB_ROW + r * SB_ROW);
+      if (!bar_wait(sb_full + tb, parity(it, 2), a.timeout_ns)) {
+        fail = 1;
+        break;
+      }
+      // a row's scale/bias run sits in one bank for all rows: read them 8 groups at a time
+      uint4 s8 = make_uint4(0, 0, 0, 0), b8 = s8;
+#pragma unroll 1
+      for (int kt = 0; kt < KT; ++kt, ++g) {
+        const int rs = g % RSTAGES, as = g % ASTAGES;
+        if (vec8 && (kt & 7) == 0) {
+          s8 = reinterpret_cast<const uint4*>(sbr)[kt >> 3];
+          b8 = reinterpret_cast<const uint4*>(sbr + KT)[kt >> 3];
+        }
+        uint16_t sv, bv;
+        if (vec8) {
+          const int j = (kt & 7) >> 1, shf = 16 * (kt & 1);
+          const uint32_t sw = j == 0 ? s8.x : j == 1 ? s8.y : j == 2 ? s8.z : s8.w;
+          const uint32_t bw = j == 0 ? b8.x : j == 1 ? b8.y : j == 2 ? b8.z : b8.w;
+          sv = static_cast<uint16_t>(sw >> shf);
+          bv = static_cast<uint16_t>(bw >> shf);
+        } else {
+          sv = sbr[kt];
+          bv = sbr[KT + kt];
+        }
+        if (!bar_wait(raw_full + rs, parity(g, RSTAGES), a.timeout_ns)) {
+          fail = 1;
+          break;
+        }
+        const uint4 q = *reinterpret_cast<const uint4*>(smRaw + rs * RAW_STAGE + r * 32 + h * 16);
+        bar_arrive(raw_empty + rs);
+        const __half2 s2 = __half2half2(__ushort_as_half(sv)), b2 = __half2half2(__ushort_as_half(bv));
+        const uint4 w0 = dequant_pair_order(q.x, s2, b2), w1 = dequant_pair_order(q.y, s2, b2);
+        const uint4 w2 = dequant_pair_order(q.z, s2, b2), w3 = dequant_pair_order(q.w, s2, b2);
+        if (!bar_wait(a_empty + as, parity(g, ASTAGES) ^ 1u, a.timeout_ns)) {  // the MMA may still read it
+          fail = 1;
+          break;
+        }
+        uint8_t* dd = smA + as * A_STAGE + (r >> 3) * 1024 + (r & 7) * 128;
+        const int c0 = 4 * h, x = r & 7;
+        *reinterpret_cast<uint4*>(dd + (((c0 + 0) ^ x) << 4)) = w0;
+        *reinterpret_cast<uint4*>(dd + (((c0 + 1) ^ x) << 4)) = w1;
+        *reinterpret_cast<uint4*>(dd + (((c0 + 2) ^ x) << 4)) = w2;
+        *reinterpret_cast<uint4*>(dd + (((c0 + 3) ^ x) << 4)) = w3;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (!(g == 0 && d == 0 && ti == a.drop_tile)) bar_arrive(a_full + as);
+      }
+      if (fail) break;
+      bar_arrive(sb_empty + tb);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue (TMEM lane quadrant = warp % 4)
+    const int quad = warp & 3;
+    const int L = quad * 32 + lane;  // TMEM lane = tile row
+    const int et = tid - (64 + kDq);  // 0..127 among the epilogue threads
+    const int r = a.lora_r;
+    int it = 0;
+#pragma unroll 1
+    for (int ti = blockIdx.x; ti < n_tiles && !fail; ti += gridDim.x, ++it) {
+      const Tile tile = a.tiles[ti];
+      const int ab = it & 1;
+      // the four epilogue warps leave together (they meet at named barriers below)
+      if (epi_any(!bar_wait(acc_full + ab, parity(it, 2), a.timeout_ns))) {
+        fail = 1;
+        break;
+      }
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t taddr = tmem + static_cast<uint32_t>(ab * BM) + ((static_cast<uint32_t>(quad) * 32u) << 16);
+      const int o = tile.mt * BM + L;
+      if (a.epi == EPI_SWIGLU) {
+        bool range_bad = false;  // a SwiGLU output fp16 cannot hold: MOE_ERR_RANGE
+        const bool up = (L & 1) != 0;
+        const int j = o >> 1;
+        const bool sh = tile.e == a.E;  // the shared expert's gate/up carry LoRA deltas
+        const uint16_t* Bsrc = sh ? (up ? a.lora_B2 : a.lora_B1) : nullptr;
+        const float* tsrc = up ? a.lora_t2 : a.lora_t1;
+        const int col = pair_pos(L >> 1);  // SwiGLU outputs in pair order (the down GEMM's token operand)
+#pragma unroll 1
+        for (int c0 = 0; c0 < tile.n; c0 += 32) {
+          float v[32];
+          tmem_ld32(taddr + c0, v);
+          if (Bsrc) {  // unmerged LoRA: + scale * B[j] . t[token]
+#pragma unroll 1
+            for (int i = 0; i < r; ++i) {
+              const float bj = half_bits_to_float(Bsrc[static_cast<size_t>(j) * r + i]);
+#pragma unroll
+              for (int t = 0; t < 32; ++t) {
+                const int tt = c0 + t < tile.n ? c0 + t : tile.n - 1;
+                v[t] = fmaf(a.lora_scale * bj, tsrc[static_cast<size_t>(tile.row0 + tt) * r + i], v[t]);
+              }
+            }
+          }
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            const float partner = __shfl_xor_sync(0xffffffffu, v[t], 1);
+            if (!up && c0 + t < tile.n) {
+              const float hv = silu(v[t]) * partner;
+              range_bad |= !(fabsf(hv) <= kF16Max);
+              stage[(c0 + t) * 64 + col] = __half_as_ushort(__float2half_rn(hv));
+            }
+          }
+        }
+        // the accumulator is read: release it for the tile after next
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        bar_arrive(acc_empty + ab);
+        if (range_bad) report(a.err, 6);
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        for (int i = et; i < tile.n * 8; i += kEpi) {
+          const int t = i >> 3, ch = i & 7;
+          *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(tile.row0 + t) * a.out_ld + tile.mt * 64 + ch * 8) =
+              reinterpret_cast<const uint4*>(stage + t * 64)[ch];
+        }
+      } else {
+        const uint16_t* Bsrc = tile.e < a.E ? (a.lora_Bex ? a.lora_Bex + static_cast<size_t>(tile.e) * (a.out_ld) * r
+                                                          : nullptr)
+                                            : a.lora_B1;
+#pragma unroll 1
+        for (int c0 = 0; c0 < tile.n; c0 += 32) {
+          float v[32];
+          tmem_ld32(taddr + c0, v);
+          if (Bsrc) {
+#pragma unroll 1
+            for (int i = 0; i < r; ++i) {
+              const float bo = half_bits_to_float(Bsrc[static_cast<size_t>(o) * r + i]);
+#pragma unroll
+              for (int t = 0; t < 32; ++t) {
+                const int tt = c0 + t < tile.n ? c0 + t : tile.n - 1;
+                v[t] = fmaf(a.lora_scale * bo, a.lora_t1[static_cast<size_t>(tile.row0 + tt) * r + i], v[t]);
+              }
+            }
+          }
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            if (c0 + t < tile.n) {
+              float xv = v[t];
+              if (tile.e < a.E && a.row_scale) xv *= a.row_scale[tile.row0 + c0 + t];
+              stage[(c0 + t) * 128 + L] = __half_as_ushort(__float2half_rn(xv));
+            }
+          }
+        }
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        bar_arrive(acc_empty + ab);
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        for (int i = et; i < tile.n * 16; i += kEpi) {
+          const int t = i >> 4, ch = i & 15;
+          *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(tile.row0 + t) * a.out_ld + tile.mt * BM + ch * 8) =
+              reinterpret_cast<const uint4*>(stage + t * 128)[ch];
+        }
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");  // the staging buffer is free for the next tile
+    }
+  }
+  if (fail) report(a.err, 5);
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+}
+
+}  // namespace gg3
+}  // namespace moe

@@ -22,10 +22,12 @@ constexpr int TB = 8;  // tokens per pass of a GEMV kernel
 // Stage tokens tok[0..nt) of u (bf16 [.][H]) into shared memory as fp16:
 // natural order (8 consecutive values per uint4) or pair order (per 8-block:
 // (u_j, u_{j+4}) for j = 0..3).  sum32[t][c] / sum16[t][c] are fp32 sums of the
-// bf16 values over 32- / 16-element chunks (may be null).
+// bf16 values over 32- / 16-element chunks (may be null).  A value fp16 cannot
+// hold (|u| > 65504 or not finite) reports MOE_ERR_RANGE into err (may be null).
 MOE_DEV void stage_tokens(const uint16_t* __restrict__ u, int H, const int* tok, int nt, uint4* dst,
-                          float* sum32, float* sum16, bool pair_order) {
+                          float* sum32, float* sum16, bool pair_order, int* err) {
   const int n32 = H / 32;
+  bool bad = false;
   for (int wi = threadIdx.x; wi < nt * n32; wi += blockDim.x) {
     const int t = wi / n32, c = wi - t * n32;
     const uint4* src = reinterpret_cast<const uint4*>(u + static_cast<size_t>(tok[t]) * H + c * 32);
@@ -38,8 +40,10 @@ MOE_DEV void stage_tokens(const uint16_t* __restrict__ u, int H, const int* tok,
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const uint16_t lo = static_cast<uint16_t>(vw[i] & 0xffffu), hi = static_cast<uint16_t>(vw[i] >> 16);
-        s[blk >> 1] += bf16_bits_to_float(lo);
-        s[blk >> 1] += bf16_bits_to_float(hi);
+        const float flo = bf16_bits_to_float(lo), fhi = bf16_bits_to_float(hi);
+        bad |= !(fabsf(flo) <= kF16Max) || !(fabsf(fhi) <= kF16Max);
+        s[blk >> 1] += flo;
+        s[blk >> 1] += fhi;
         e[2 * i] = bf16_to_f16_bits(lo);
         e[2 * i + 1] = bf16_to_f16_bits(hi);
       }
@@ -63,6 +67,7 @@ MOE_DEV void stage_tokens(const uint16_t* __restrict__ u, int H, const int* tok,
       sum16[t * 2 * n32 + 2 * c + 1] = s[1];
     }
   }
+  if (bad) report(err, 6);
 }
 
 
@@ -113,7 +118,7 @@ MOE_DEV void row_int8(const uint32_t* __restrict__ q, const uint16_t* __restrict
 template <int NCH>  // H / 16
 __global__ void __launch_bounds__(kThreads) router_kernel(const uint16_t* __restrict__ u, int T,
                                                           const uint8_t* __restrict__ rows, const float* __restrict__ rbias,
-                                                          int E, float* __restrict__ logits) {
+                                                          int E, float* __restrict__ logits, int* err) {
   constexpr int SEG = NCH < 32 ? NCH : 32;
   constexpr int RPW = 32 / SEG;
   constexpr int H = NCH * 16;
@@ -125,7 +130,7 @@ __global__ void __launch_bounds__(kThreads) router_kernel(const uint16_t* __rest
   const int t0 = blockIdx.y * TB, nt = min(TB, T - t0);
   if (threadIdx.x < TB) tok[threadIdx.x] = t0 + min(static_cast<int>(threadIdx.x), nt - 1);
   __syncthreads();
-  stage_tokens(u, H, tok, nt, us, nullptr, sum16, false);
+  stage_tokens(u, H, tok, nt, us, nullptr, sum16, false, blockIdx.x == 0 ? err : nullptr);
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, sl = lane % SEG;
   const int e = (blockIdx.x * kWarps + warp) * RPW + lane / SEG;
@@ -316,6 +321,7 @@ struct PreArgs {
   const uint16_t* A_up;
   float* g;     // [T]
   float* t_gu;  // [T][2][r]
+  int* err;     // optional error word
 };
 
 // Block 0: buckets.  Blocks >= 1: shared-expert gate and the shared LoRA A u
@@ -345,7 +351,7 @@ __global__ void __launch_bounds__(kThreads) pre_kernel(PreArgs a) {
     __syncthreads();
     if (threadIdx.x < TB) tok[threadIdx.x] = t0 + min(static_cast<int>(threadIdx.x), nt - 1);
     __syncthreads();
-    stage_tokens(a.u, H, tok, nt, us, nullptr, sum16, false);
+    stage_tokens(a.u, H, tok, nt, us, nullptr, sum16, false, blockIdx.x == 1 ? a.err : nullptr);
     __syncthreads();
     float acc[TB];
 #pragma unroll
@@ -387,6 +393,7 @@ struct GateUpArgs {
   int r;
   float lora_scale;
   uint16_t* h16;  // [T*K + T][I] fp16, pair order
+  int* err;       // optional error word: a SwiGLU output fp16 cannot hold reports MOE_ERR_RANGE
 };
 
 // grid (ceil(I / pairs per CTA), T*K + 1).  Unit y < T*K is the sorted slot
@@ -431,7 +438,7 @@ __global__ void __launch_bounds__(kThreads) gate_up_kernel(GateUpArgs a) {
       tok[threadIdx.x] = shared ? p0 + i : s / a.K;
     }
     __syncthreads();
-    stage_tokens(a.u, H, tok, nt, up, sum32, nullptr, true);
+    stage_tokens(a.u, H, tok, nt, up, sum32, nullptr, true, nullptr);
     __syncthreads();
     float ag[TB], au[TB];
 #pragma unroll
@@ -490,6 +497,7 @@ __global__ void __launch_bounds__(kThreads) gate_up_kernel(GateUpArgs a) {
           }
         }
         const float h = silu(gv) * uv;
+        if (!(fabsf(h) <= kF16Max)) report(a.err, 6);
         a.h16[static_cast<size_t>(slot[t]) * a.I + pair_pos(j)] = __half_as_ushort(__float2half_rn(h));
       }
     }
@@ -666,6 +674,7 @@ struct PreW1Args {
   const int32_t* sel;
   const uint16_t *W1, *b1;
   float* z;  // [T][P]
+  int* err;  // optional error word
 };
 
 // z[t][p] = silu(W1[p][:H] . u[t] + sum_k W1[p][H + sel[t][k]] + b1[p]); one row per warp.
@@ -681,7 +690,7 @@ __global__ void __launch_bounds__(kThreads) prerouter_w1_kernel(PreW1Args a) {
   const int t0 = blockIdx.y * TB, nt = min(TB, a.T - t0);
   if (threadIdx.x < TB) tok[threadIdx.x] = t0 + min(static_cast<int>(threadIdx.x), nt - 1);
   __syncthreads();
-  stage_tokens(a.u, H, tok, nt, us, nullptr, nullptr, false);
+  stage_tokens(a.u, H, tok, nt, us, nullptr, nullptr, false, blockIdx.x == 0 ? a.err : nullptr);
   __syncthreads();
   if (p >= a.P) return;
   float acc[TB];

@@ -10,6 +10,7 @@
 #include "layer_kernels.cuh"
 #include "prefill_kernels.cuh"
 #include "stack_kernel.cuh"
+#include "stack2_kernel.cuh"
 
 namespace {
 
@@ -123,7 +124,7 @@ void allow_smem(KernelT k, size_t bytes) {
 
 template <int H>
 moe_status route_h(const moe_layer* L, const uint16_t* u, int T, int K, float* logits, int32_t* idx, float* w,
-                   cudaStream_t st) {
+                   int* err, cudaStream_t st) {
   constexpr int NCH = H / 16;
   constexpr int SEG = NCH < 32 ? NCH : 32;
   const int rows_per_cta = kWarps * (32 / SEG);
@@ -131,14 +132,14 @@ moe_status route_h(const moe_layer* L, const uint16_t* u, int T, int K, float* l
   allow_smem(router_kernel<NCH>, smem);
   dim3 grid((L->E + rows_per_cta - 1) / rows_per_cta, (T + TB - 1) / TB);
   router_kernel<NCH><<<grid, kThreads, smem, st>>>(u, T, static_cast<const uint8_t*>(L->router.rows),
-                                                   L->router_bias, L->E, logits);
+                                                   L->router_bias, L->E, logits, err);
   topk_kernel<<<(T + kWarps - 1) / kWarps, kThreads, 0, st>>>(logits, T, L->E, K, idx, w);
   return launch_status();
 }
 
 template <int H, int I>
 moe_status expert_forward_hi(const moe_layer* L, const uint16_t* u, int T, int K, const int32_t* idx, const float* w,
-                             void* out, int out_mode, int32_t* perm_out, const Ws& ws, cudaStream_t st) {
+                             void* out, int out_mode, int32_t* perm_out, const Ws& ws, int* err, cudaStream_t st) {
   const int TK = T * K;
   // 1) buckets, shared gate, shared LoRA A u
   PreArgs pa{};
@@ -159,6 +160,7 @@ moe_status expert_forward_hi(const moe_layer* L, const uint16_t* u, int T, int K
   pa.A_up = L->r > 0 ? L->sh_lora_A[1] : nullptr;
   pa.g = ws.g;
   pa.t_gu = ws.t_gu;
+  pa.err = err;
   const int nrows = 1 + (pa.A_gate ? L->r : 0) + (pa.A_up ? L->r : 0);
   const size_t smem_pre = gemv_smem(H, false, true);
   allow_smem(pre_kernel<H / 8>, smem_pre);
@@ -181,6 +183,7 @@ moe_status expert_forward_hi(const moe_layer* L, const uint16_t* u, int T, int K
   ga.r = L->r;
   ga.lora_scale = L->lora_scale;
   ga.h16 = ws.h16;
+  ga.err = err;
   {
     constexpr int NCH = H / 32;
     constexpr int SEG = NCH < 32 ? NCH : 32;
@@ -231,6 +234,7 @@ moe_status expert_forward_hi(const moe_layer* L, const uint16_t* u, int T, int K
 
 // ----------------------------------------------------------------------------- grouped-GEMM path (many slots)
 constexpr int kGemmMinSlots = 128;  // T*K from which moe_expert_forward uses the tensor-core path
+constexpr long long kGemmTimeoutNs = 2000000000LL;  // bound of every wait of the grouped GEMMs
 
 struct GWs {
   int32_t *idx, *count, *offset, *perm, *inv, *blockhist;
@@ -299,31 +303,64 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// Row-major fp16 matrix [rows][cols] as a TMA source of [128 rows x 64 cols] boxes, 128-byte swizzle.
+// Row-major fp16 matrix [rows][cols] as a TMA source of [32 rows x 64 cols] boxes, 128-byte swizzle.
 bool token_map(CUtensorMap* m, const uint16_t* X, int cols, int rows) {
   const EncodeTiledFn f = encode_tiled();
   if (!f) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(gg::BK), static_cast<cuuint32_t>(gg::BN)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(gg3::BK), static_cast<cuuint32_t>(gg3::BROWS)};
   const cuuint32_t estr[2] = {1, 1};
   return f(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(X), dims, strides, box, estr,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The row records of one weight matrix in n_exp expert blocks (expert_stride bytes apart) as a 3-D byte map
+// {record bytes, rows, experts}, boxes of box_x bytes x 128 rows x 1 expert, no swizzle.
+bool weight_map(CUtensorMap* m, const uint8_t* base, int rec, int rows, int n_exp, int64_t expert_stride, int box_x) {
+  const EncodeTiledFn f = encode_tiled();
+  if (!f) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(rec), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(n_exp)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(rec), static_cast<cuuint64_t>(expert_stride)};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_x), static_cast<cuuint32_t>(gg3::BM), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The tensor maps of one grouped GEMM over the matrix at byte a_off of every expert block (records of rec
+// bytes, rows of them per expert, reduction length K).
+bool gemm_maps(gg3::Maps* m, const moe_layer* L, int64_t a_off, int rec, int rows, int K, const uint16_t* tokens,
+               int n_token_rows) {
+  const uint8_t* pool = static_cast<const uint8_t*>(L->pool) + a_off;
+  const uint8_t* sh = static_cast<const uint8_t*>(L->shared_block) + a_off;
+  const int sb = gg3::sb_row_bytes(K);
+  const int64_t sh_stride = static_cast<int64_t>(rec) * rows;
+  return weight_map(&m->pool_codes, pool, rec, rows, L->E, L->expert_stride, 32) &&
+         weight_map(&m->pool_sb, pool, rec, rows, L->E, L->expert_stride, sb) &&
+         weight_map(&m->shared_codes, sh, rec, rows, 1, sh_stride, 32) &&
+         weight_map(&m->shared_sb, sh, rec, rows, 1, sh_stride, sb) &&
+         token_map(&m->tokens, tokens, K, n_token_rows);
+}
+
 template <int H>
+// Bounded waits give up after timeout_ns; drop_tile >= 0 arms the gate/up GEMM's test hook (gg3::Args).
 moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int K, const int32_t* idx, const float* w,
-                               void* out, int out_mode, int32_t* perm_out, void* workspace, cudaStream_t st) {
+                               void* out, int out_mode, int32_t* perm_out, void* workspace, int* err,
+                               long long timeout_ns, int drop_tile, cudaStream_t st) {
   const int E = L->E, I = L->I, TK = T * K, R = TK + T;
   const bool lora = L->r > 0 && L->sh_lora_A[0];
   const int r = L->r > 0 ? L->r : 0;
   const GWs ws = carve_gemm(workspace, T, K, E, H, I, L->r);
-  if (cudaMemsetAsync(ws.err, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+  int* err_dev = err ? err : ws.err;  // without a caller's word, reports go to the workspace's own (unread) word
+  if (!err && cudaMemsetAsync(ws.err, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
   pf::bucket_count_kernel<<<ws.nblk, pf::kChunk, 0, st>>>(idx, TK, E, ws.idx, ws.blockhist);
   pf::bucket_scan_kernel<<<1, 256, 0, st>>>(ws.nblk, E, ws.blockhist, ws.count, ws.offset);
   pf::bucket_place_kernel<<<ws.nblk, pf::kChunk, 0, st>>>(ws.idx, TK, E, ws.blockhist, ws.perm, ws.inv, perm_out);
-  pf::permute_kernel<<<R, 256, 0, st>>>(u, T, K, H, ws.perm, w, ws.X, ws.w_pos);
+  pf::permute_kernel<<<R, 256, 0, st>>>(u, T, K, H, ws.perm, w, ws.X, ws.w_pos, err_dev);
   pf::tile_list_kernel<<<1, 288, 0, st>>>(ws.count, ws.offset, E, T, K, 2 * I / gg::BM, H / gg::BM, ws.tiles_gu,
                                           ws.tiles_dn, ws.n_tiles);
   // The GEMMs trust the device-built tile list: stop here if any launch so far failed.
@@ -337,32 +374,37 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
         u, T, TK, r, static_cast<const uint8_t*>(L->shared_gate.rows), lora ? L->sh_lora_A[0] : nullptr,
         lora ? L->sh_lora_A[1] : nullptr, ws.g, ws.t1, ws.t2);
   }
-  CUtensorMap mx, mh;
-  if (!token_map(&mx, ws.X, H, R) || !token_map(&mh, ws.Hh, I, R)) return MOE_ERR_CUDA;
   const int RGU = qrow_bytes(H, 4), RDN = qrow_bytes(I, 4);
+  const int64_t dn_off = static_cast<int64_t>(2 * I) * RGU;
+  gg3::Maps m_gu, m_dn;
+  if (!gemm_maps(&m_gu, L, 0, RGU, 2 * I, H, ws.X, R) || !gemm_maps(&m_dn, L, dn_off, RDN, H, I, ws.Hh, R))
+    return MOE_ERR_CUDA;
   auto base_args = [&]() {
-    gg::Args a{};
+    gg3::Args a{};
     a.n_tiles = ws.n_tiles;
-    a.pool = static_cast<const uint8_t*>(L->pool);
-    a.stride = L->expert_stride;
-    a.shared_block = static_cast<const uint8_t*>(L->shared_block);
     a.E = E;
     a.lora_r = r;
     a.lora_scale = L->lora_scale;
-    a.err = ws.err;
-    a.timeout_ns = 2000000000LL;
+    a.err = err_dev;
+    a.timeout_ns = timeout_ns;
+    a.drop_tile = -1;
     return a;
   };
-  if (cudaFuncSetAttribute(gg::grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gg::SMEM_BYTES) !=
-      cudaSuccess)
+  const int smem_gu = gg3::smem_bytes(H), smem_dn = gg3::smem_bytes(I);
+  if (cudaFuncSetAttribute(gg3::grouped_gemm3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem_gu > smem_dn ? smem_gu : smem_dn) != cudaSuccess)
     return MOE_ERR_CUDA;
+  int dev = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  // persistent: one CTA per SM walks the tile list (the tile count is known only on the device)
+  const int grid_gu = ws.max_gu < nsm ? ws.max_gu : nsm, grid_dn = ws.max_dn < nsm ? ws.max_dn : nsm;
   {  // gate/up + SwiGLU for every bucket and the shared expert
-    gg::Args a = base_args();
+    gg3::Args a = base_args();
     a.tiles = ws.tiles_gu;
     a.K = H;
-    a.a_off = 0;
-    a.a_rec = RGU;
     a.epi = gg::EPI_SWIGLU;
+    a.drop_tile = drop_tile;
     a.out = ws.Hh;
     a.out_ld = I;
     if (lora) {
@@ -371,7 +413,7 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
       a.lora_B2 = L->sh_lora_B[1];
       a.lora_t2 = ws.t2;
     }
-    gg::grouped_gemm_kernel<<<ws.max_gu, gg::kThreads, gg::SMEM_BYTES, st>>>(mx, a);
+    gg3::grouped_gemm3_kernel<<<grid_gu, gg3::kThreads, smem_gu, st>>>(m_gu, a);
   }
   const bool ex = r > 0 && L->ex_lora_A;
   if (lora || ex) {  // LoRA A products on the SwiGLU output (shared down, routed down)
@@ -381,12 +423,10 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
         ws.perm, ws.t1);
   }
   {  // down (+ LoRA), routed rows scaled by their gating weight
-    gg::Args a = base_args();
+    gg3::Args a = base_args();
     a.tiles = ws.tiles_dn;
     a.n_tiles = ws.n_tiles + 1;
     a.K = I;
-    a.a_off = static_cast<int64_t>(2 * I) * RGU;
-    a.a_rec = RDN;
     a.epi = gg::EPI_DOWN;
     a.out = ws.Y;
     a.out_ld = H;
@@ -394,7 +434,7 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
     a.lora_B1 = lora ? L->sh_lora_B[2] : nullptr;
     a.lora_t1 = ws.t1;
     a.lora_Bex = ex ? L->ex_lora_B : nullptr;
-    gg::grouped_gemm_kernel<<<ws.max_dn, gg::kThreads, gg::SMEM_BYTES, st>>>(mh, a);
+    gg3::grouped_gemm3_kernel<<<grid_dn, gg3::kThreads, smem_dn, st>>>(m_dn, a);
   }
   pf::combine_kernel<<<T, 256, 0, st>>>(ws.Y, T, K, H, ws.inv, ws.g, out, out_mode);
   return launch_status();
@@ -402,21 +442,23 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
 
 template <int H>
 moe_status expert_forward_h(const moe_layer* L, const uint16_t* u, int T, int K, const int32_t* idx, const float* w,
-                            void* out, int out_mode, int32_t* perm_out, const Ws& ws, cudaStream_t st) {
-  if (gemm_path(L, T, K)) return expert_forward_gemm<H>(L, u, T, K, idx, w, out, out_mode, perm_out, ws.base, st);
+                            void* out, int out_mode, int32_t* perm_out, const Ws& ws, int* err, long long timeout_ns,
+                            int drop_tile, cudaStream_t st) {
+  if (gemm_path(L, T, K))
+    return expert_forward_gemm<H>(L, u, T, K, idx, w, out, out_mode, perm_out, ws.base, err, timeout_ns, drop_tile, st);
   switch (L->I) {
-    case 128: return expert_forward_hi<H, 128>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
-    case 256: return expert_forward_hi<H, 256>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
-    case 512: return expert_forward_hi<H, 512>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
-    case 1024: return expert_forward_hi<H, 1024>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
-    case 2048: return expert_forward_hi<H, 2048>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
+    case 128: return expert_forward_hi<H, 128>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, err, st);
+    case 256: return expert_forward_hi<H, 256>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, err, st);
+    case 512: return expert_forward_hi<H, 512>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, err, st);
+    case 1024: return expert_forward_hi<H, 1024>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, err, st);
+    case 2048: return expert_forward_hi<H, 2048>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, err, st);
     default: return MOE_ERR_UNSUPPORTED;
   }
 }
 
 template <int H>
 moe_status prerouter_h(const moe_prerouter* P, const uint16_t* u, const int32_t* sel, int T, int K, int K_next,
-                       int32_t* pred, float* scores, float* z, cudaStream_t st) {
+                       int32_t* pred, float* scores, float* z, int* err, cudaStream_t st) {
   PreW1Args a{};
   a.u = u;
   a.T = T;
@@ -427,6 +469,7 @@ moe_status prerouter_h(const moe_prerouter* P, const uint16_t* u, const int32_t*
   a.W1 = P->W1;
   a.b1 = P->b1;
   a.z = z;
+  a.err = err;
   const size_t smem = gemv_smem(H, false, false);
   allow_smem(prerouter_w1_kernel<H / 8>, smem);
   dim3 g1((P->P + kWarps - 1) / kWarps, (T + TB - 1) / TB);
@@ -453,6 +496,7 @@ const char* moe_status_string(moe_status s) {
     case MOE_ERR_WORKSPACE: return "workspace too small";
     case MOE_ERR_CUDA: return "CUDA launch failed";
     case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+    case MOE_ERR_RANGE: return "activation outside the fp16 range";
   }
   return "unknown status";
 }
@@ -476,18 +520,18 @@ moe_status moe_rmsnorm_bf16(const float* x, int32_t T, int32_t H, float eps, uin
 }
 
 moe_status moe_route_topk(const moe_layer* L, const uint16_t* u, int32_t T, int32_t K, float* logits, int32_t* idx,
-                          float* w, void* stream) {
+                          float* w, int32_t* err_word, void* stream) {
   const moe_status s = check_layer(L, T, K);
   if (s != MOE_OK) return s;
   if (T == 0) return MOE_OK;
   if (!u || !logits || !idx || !w || !aligned(u, 16)) return MOE_ERR_INVALID_ARG;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (L->H) {
-    case 256: return route_h<256>(L, u, T, K, logits, idx, w, st);
-    case 512: return route_h<512>(L, u, T, K, logits, idx, w, st);
-    case 1024: return route_h<1024>(L, u, T, K, logits, idx, w, st);
-    case 2048: return route_h<2048>(L, u, T, K, logits, idx, w, st);
-    case 4096: return route_h<4096>(L, u, T, K, logits, idx, w, st);
+    case 256: return route_h<256>(L, u, T, K, logits, idx, w, err_word, st);
+    case 512: return route_h<512>(L, u, T, K, logits, idx, w, err_word, st);
+    case 1024: return route_h<1024>(L, u, T, K, logits, idx, w, err_word, st);
+    case 2048: return route_h<2048>(L, u, T, K, logits, idx, w, err_word, st);
+    case 4096: return route_h<4096>(L, u, T, K, logits, idx, w, err_word, st);
     default: return MOE_ERR_UNSUPPORTED;
   }
 }
@@ -506,9 +550,16 @@ size_t moe_workspace_size(const moe_layer* L, int32_t T, int32_t K) {
   return ws_bytes_for(L, T, K);
 }
 
-moe_status moe_expert_forward(const moe_layer* L, const uint16_t* u, int32_t T, int32_t K, const int32_t* idx,
-                              const float* w, void* out, int32_t out_mode, int32_t* perm_out, void* workspace,
-                              size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// moe_expert_forward with the grouped GEMMs' wait bound and test hook exposed (the stack's per-layer path
+// passes its options through).
+moe_status expert_forward_entry(const moe_layer* L, const uint16_t* u, int32_t T, int32_t K, const int32_t* idx,
+                                const float* w, void* out, int32_t out_mode, int32_t* perm_out, void* workspace,
+                                size_t ws_bytes, int32_t* err_word, long long timeout_ns, int drop_tile,
+                                void* stream) {
   moe_status s = check_layer(L, T, K);
   if (s != MOE_OK) return s;
   if (out_mode < 0 || out_mode > 2) return MOE_ERR_INVALID_ARG;
@@ -521,13 +572,34 @@ moe_status moe_expert_forward(const moe_layer* L, const uint16_t* u, int32_t T, 
   const Ws ws = carve(workspace, T, K, L->E, L->I, L->r);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (L->H) {
-    case 256: return expert_forward_h<256>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
-    case 512: return expert_forward_h<512>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
-    case 1024: return expert_forward_h<1024>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
-    case 2048: return expert_forward_h<2048>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
-    case 4096: return expert_forward_h<4096>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, st);
+    case 256:
+      return expert_forward_h<256>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, err_word, timeout_ns, drop_tile,
+                                  st);
+    case 512:
+      return expert_forward_h<512>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, err_word, timeout_ns, drop_tile,
+                                  st);
+    case 1024:
+      return expert_forward_h<1024>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, err_word, timeout_ns, drop_tile,
+                                  st);
+    case 2048:
+      return expert_forward_h<2048>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, err_word, timeout_ns, drop_tile,
+                                  st);
+    case 4096:
+      return expert_forward_h<4096>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, err_word, timeout_ns, drop_tile,
+                                  st);
     default: return MOE_ERR_UNSUPPORTED;
   }
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_expert_forward(const moe_layer* L, const uint16_t* u, int32_t T, int32_t K, const int32_t* idx,
+                              const float* w, void* out, int32_t out_mode, int32_t* perm_out, void* workspace,
+                              size_t ws_bytes, int32_t* err_word, void* stream) {
+  return expert_forward_entry(L, u, T, K, idx, w, out, out_mode, perm_out, workspace, ws_bytes, err_word,
+                              kGemmTimeoutNs, -1, stream);
 }
 
 size_t prerouter_workspace_size(const moe_prerouter* head, int32_t T) {
@@ -537,7 +609,7 @@ size_t prerouter_workspace_size(const moe_prerouter* head, int32_t T) {
 
 moe_status prerouter_predict(const moe_prerouter* head, const uint16_t* u, const int32_t* sel, int32_t T, int32_t K,
                              int32_t K_next, int32_t* pred, float* scores, void* workspace, size_t ws_bytes,
-                             void* stream) {
+                             int32_t* err_word, void* stream) {
   if (!head) return MOE_ERR_INVALID_ARG;
   if (T < 0 || T > MOE_MAX_TOKENS) return MOE_ERR_UNSUPPORTED;
   moe_status s = check_head_shape(head, K, K_next);
@@ -551,11 +623,11 @@ moe_status prerouter_predict(const moe_prerouter* head, const uint16_t* u, const
   float* z = static_cast<float*>(workspace);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (head->H) {
-    case 256: return prerouter_h<256>(head, u, sel, T, K, K_next, pred, scores, z, st);
-    case 512: return prerouter_h<512>(head, u, sel, T, K, K_next, pred, scores, z, st);
-    case 1024: return prerouter_h<1024>(head, u, sel, T, K, K_next, pred, scores, z, st);
-    case 2048: return prerouter_h<2048>(head, u, sel, T, K, K_next, pred, scores, z, st);
-    case 4096: return prerouter_h<4096>(head, u, sel, T, K, K_next, pred, scores, z, st);
+    case 256: return prerouter_h<256>(head, u, sel, T, K, K_next, pred, scores, z, err_word, st);
+    case 512: return prerouter_h<512>(head, u, sel, T, K, K_next, pred, scores, z, err_word, st);
+    case 1024: return prerouter_h<1024>(head, u, sel, T, K, K_next, pred, scores, z, err_word, st);
+    case 2048: return prerouter_h<2048>(head, u, sel, T, K, K_next, pred, scores, z, err_word, st);
+    case 4096: return prerouter_h<4096>(head, u, sel, T, K, K_next, pred, scores, z, err_word, st);
     default: return MOE_ERR_UNSUPPORTED;
   }
 }
@@ -733,6 +805,175 @@ cudaError_t launch_persistent(const Persist& pl, const moe_layer* Ls, const moe_
                                     pl.sm.total, st);
 }
 
+// Layout of the second-generation single-launch kernel (same eligibility as plan_persistent).
+struct Persist2 {
+  bool ok = false;
+  stk2::Smem sm{};
+  int NA = 0, grid = 0;
+  int ll_x = 0, ll_a = 0, ll_h = 0, ll_z = 0, ll_p = 0, ll_stride = 0, st_bytes = 0;
+  size_t ll_bytes = 0;
+};
+
+Persist2 plan_persistent2(const moe_layer* Ls, const moe_prerouter* Ps, int n, int T, int K, int K_next, int use_pred) {
+  Persist2 pl;
+  const moe_layer& L0 = Ls[0];
+  const int H = L0.H, E = L0.E, I = L0.I, r = L0.r;
+  if (T != 1 || use_pred || n > stk::kMaxLayers || (H != 1024 && H != 2048) || I != 512 || E % 8 || K > stk2::kMaxK)
+    return pl;
+  const bool lora = r > 0 && L0.sh_lora_A[0];
+  if (lora && (r % 8 || r > 32)) return pl;
+  for (int l = 0; l < n; ++l) {
+    const moe_layer& L = Ls[l];
+    if (L.ex_lora_A) return pl;
+    for (int q = 0; q < 3; ++q)
+      if ((L.sh_lora_A[q] != nullptr) != lora || (L.sh_lora_B[q] != nullptr) != lora) return pl;
+    if (!L.shared_block || !aligned(L.shared_block, 16) || !qrows_ok(L.shared_gate, 1, H, 8)) return pl;
+    if (!L.pool || !aligned(L.pool, 256) || L.expert_stride != L0.expert_stride || L.expert_stride % 256) return pl;
+    if (Ps && (!Ps[l].W1 || !Ps[l].b1 || !Ps[l].W2 || !Ps[l].b2 || !aligned(Ps[l].W1, 16) || !aligned(Ps[l].W2, 16)))
+      return pl;
+  }
+  const int P = Ps ? Ps[0].P : 0, En = Ps ? Ps[0].E_next : 0;
+  if (Ps && (P % 8 || P > 2048 || En > 256 || En < K || K_next != K)) return pl;
+  int dev = 0, nsm = 0, optin = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess || nsm <= 0)
+    return pl;
+  const int N = nsm;
+  const int NA = E + 1 + (lora ? 2 * r : 0);
+  auto cdiv = [](int a, int b) { return (a + b - 1) / b; };
+  stk2::Smem& S = pl.sm;
+  S.maxA = cdiv(NA, N);
+  S.maxS = cdiv(I / 2, N);
+  S.maxR = cdiv(K * I / 2, N);
+  S.maxD = cdiv(H, N);
+  S.maxZ = P ? cdiv(P, N) : 0;
+  // per-thread roles of the kernel: SwiGLU words by threads < 480, Prerouter words by the last warp's
+  // lanes, 16 combine lanes per output row
+  if (S.maxS + S.maxR > stk2::kThreads - 32 || S.maxZ > 32 || S.maxD > 2 * stk2::kWarps) return pl;
+  const int RGU = qrow_bytes(H, 4), RDN = qrow_bytes(I, 4), R8 = qrow_bytes(H, 8), UNIT = 4 * RGU;
+  S.item_bytes = static_cast<int>(align_up(static_cast<size_t>(R8 > 2 * H ? R8 : 2 * H), 16));
+  size_t o = 0;
+  auto put = [&](size_t bytes) {
+    const uint32_t at = al128(o);
+    o = at + bytes;
+    return at;
+  };
+  S.o_items = put(static_cast<size_t>(S.maxA) * S.item_bytes);
+  S.o_shu = put(static_cast<size_t>(S.maxS) * UNIT);
+  S.o_shB = put(static_cast<size_t>(S.maxS) * 8 * r);
+  S.o_sdn = put(static_cast<size_t>(S.maxD) * RDN);
+  S.o_Bd = put(static_cast<size_t>(S.maxD) * 2 * r);
+  S.o_Ad = put(static_cast<size_t>(r) * I * 2);
+  S.o_W1 = put(static_cast<size_t>(S.maxZ) * 2 * H);
+  const uint32_t st_bytes = al128(o);
+  o = 0;
+  S.st[0] = put(st_bytes);
+  S.st[1] = put(st_bytes);
+  S.units = put(static_cast<size_t>(S.maxR) * UNIT);
+  S.down = put(static_cast<size_t>(K) * S.maxD * RDN);
+  S.xs = put(4 * H);
+  S.un = put(2 * H);
+  S.up = put(2 * H);
+  S.s16 = put(4 * H / 16);
+  S.s32 = put(4 * H / 32);
+  S.hs = put(2 * (K + 1) * I);
+  S.hsum = put(4 * (K + 1) * I / 32);
+  S.logit = put(4 * ((E > En ? E : En) + 1 + 2 * r));
+  S.td = put(4 * (r + 1));
+  S.yd = put(4 * S.maxD * (K + 1));
+  S.red = put(4 * 64);
+  S.zx = put(4 * (S.maxZ + 1));
+  S.hloc = put(4 * 2 * (S.maxS + S.maxR));
+  S.shacc = put(4 * 4 * (S.maxS + 1));
+  S.bar = put(8 * (2 + S.maxR + stk2::kMaxK));
+  S.total = al128(o);
+  if (static_cast<int>(S.total) > optin) return pl;
+  pl.NA = NA;
+  pl.ll_x = 0;
+  pl.ll_a = H;
+  pl.ll_h = pl.ll_a + NA;
+  pl.ll_stride = (pl.ll_h + (K + 1) * I / 2 + 31) / 32 * 32;
+  pl.ll_z = 2 * pl.ll_stride;
+  pl.ll_p = pl.ll_z + n * P;
+  pl.ll_bytes = (static_cast<size_t>(pl.ll_p) + static_cast<size_t>(n) * En) * 8;
+  pl.st_bytes = static_cast<int>(st_bytes);
+  pl.grid = N;
+  pl.ok = true;
+  return pl;
+}
+
+template <int H>
+cudaError_t launch_persistent2(const Persist2& pl, const moe_layer* Ls, const moe_prerouter* Ps, int n, int K,
+                               float eps, float* x, float* x_trace, uint16_t* u_trace, int32_t* idx_all,
+                               int32_t* true_idx_all, int32_t* pred_all, int32_t* err, unsigned long long* ll,
+                               const moe_stack_opts* opts, cudaStream_t st) {
+  auto kern = stk2::stack_decode2_kernel<H, 512>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(pl.sm.total));
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, stk2::kThreads, pl.sm.total);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorCooperativeLaunchTooLarge;
+  stk2::Params p{};
+  const moe_layer& L0 = Ls[0];
+  p.n_layers = n;
+  p.E = L0.E;
+  p.K = K;
+  p.r = (L0.r > 0 && L0.sh_lora_A[0]) ? L0.r : 0;
+  p.P = Ps ? Ps[0].P : 0;
+  p.En = Ps ? Ps[0].E_next : 0;
+  p.NA = pl.NA;
+  p.stride = L0.expert_stride;
+  p.eps = eps;
+  p.lora_scale = L0.lora_scale;
+  p.x = x;
+  p.x_trace = x_trace;
+  p.u_trace = u_trace;
+  p.idx_all = idx_all;
+  p.true_idx_all = true_idx_all;
+  p.pred_all = pred_all;
+  p.err = err;
+  p.ll = ll;
+  p.ll_x = pl.ll_x;
+  p.ll_a = pl.ll_a;
+  p.ll_h = pl.ll_h;
+  p.ll_z = pl.ll_z;
+  p.ll_p = pl.ll_p;
+  p.ll_stride = pl.ll_stride;
+  p.st_bytes = pl.st_bytes;
+  p.timeout_ns = (opts && opts->timeout_ns > 0) ? opts->timeout_ns : 1000000000LL;
+  p.drop_layer = (opts && opts->test_drop_layer > 0) ? opts->test_drop_layer - 1 : -1;
+  p.drop_cta = opts ? opts->test_drop_cta : -1;
+  p.trace = opts ? reinterpret_cast<long long*>(opts->trace) : nullptr;
+  p.sm = pl.sm;
+  for (int l = 0; l < n; ++l) {
+    const moe_layer& L = Ls[l];
+    stk::LayerPtrs& d = p.L[l];
+    d.router = static_cast<const uint8_t*>(L.router.rows);
+    d.rbias = L.router_bias;
+    d.sgate = static_cast<const uint8_t*>(L.shared_gate.rows);
+    d.shared = static_cast<const uint8_t*>(L.shared_block);
+    if (p.r) {
+      d.Ag = L.sh_lora_A[0];
+      d.Bg = L.sh_lora_B[0];
+      d.Au = L.sh_lora_A[1];
+      d.Bu = L.sh_lora_B[1];
+      d.Ad = L.sh_lora_A[2];
+      d.Bd = L.sh_lora_B[2];
+    }
+    d.pool = static_cast<const uint8_t*>(L.pool);
+    if (Ps) {
+      d.W1 = Ps[l].W1;
+      d.b1 = Ps[l].b1;
+      d.W2 = Ps[l].W2;
+      d.b2 = Ps[l].b2;
+    }
+  }
+  void* args[] = {&p};
+  return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(kern), dim3(pl.grid), dim3(stk2::kThreads), args,
+                                    pl.sm.total, st);
+}
+
 struct StackWs {
   uint16_t* u;
   float *logits, *w, *scores;
@@ -771,11 +1012,11 @@ StackWs carve_stack(void* base, const moe_layer* L0, const moe_prerouter* P0, in
   return w;
 }
 
-// Upper bound of the epoch-word region (two parity halves + one score vector per layer).
+// Upper bound of the epoch-word region (two parity halves + one Prerouter hidden and score vector per layer).
 size_t ll_bound(const moe_layer* L0, const moe_prerouter* P0, int K, int n_layers) {
   const int NA = L0->E + 1 + 2 * (L0->r > 0 ? L0->r : 0);
   const size_t words = L0->H + NA + static_cast<size_t>(K + 1) * L0->I / 2 + (P0 ? P0->P : 0) + 32;
-  return (2 * words + static_cast<size_t>(n_layers) * (P0 ? P0->E_next : 0)) * 8;
+  return (2 * words + static_cast<size_t>(n_layers) * (P0 ? P0->E_next + P0->P : 0)) * 8;
 }
 
 }  // namespace
@@ -802,7 +1043,7 @@ moe_status moe_stack_decode(const moe_layer* layers, const moe_prerouter* heads,
                             void* stream) {
   if (!layers || n_layers < 1 || !x) return MOE_ERR_INVALID_ARG;
   if (use_predicted_routing && (!heads || K_next != K)) return MOE_ERR_INVALID_ARG;
-  if (opts && (opts->path < 0 || opts->path > 2)) return MOE_ERR_INVALID_ARG;
+  if (opts && (opts->path < 0 || opts->path > 3)) return MOE_ERR_INVALID_ARG;
   for (int l = 0; l < n_layers; ++l) {
     const moe_status s = check_layer(&layers[l], T, K);
     if (s != MOE_OK) return s;
@@ -835,18 +1076,29 @@ moe_status moe_stack_decode(const moe_layer* layers, const moe_prerouter* heads,
   if (cudaMemsetAsync(err, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
 
   const int want = opts ? opts->path : 0;
-  if (want != 1) {
-    const Persist pl = plan_persistent(layers, heads, n_layers, T, K, K_next, use_predicted_routing);
+  if (want == 0 || want == 2) {
+    const Persist2 pl = plan_persistent2(layers, heads, n_layers, T, K, K_next, use_predicted_routing);
     if (pl.ok && pl.ll_bytes <= llb) {
       if (cudaMemsetAsync(ws.ll, 0, pl.ll_bytes, st) != cudaSuccess) return MOE_ERR_CUDA;
       const cudaError_t e =
-          H == 2048 ? launch_persistent<2048>(pl, layers, heads, n_layers, K, eps, x, x_trace, u_trace, idx_all,
-                                              true_idx_all, pred_all, err, ws.ll, opts, st)
-                    : launch_persistent<1024>(pl, layers, heads, n_layers, K, eps, x, x_trace, u_trace, idx_all,
-                                              true_idx_all, pred_all, err, ws.ll, opts, st);
+          H == 2048 ? launch_persistent2<2048>(pl, layers, heads, n_layers, K, eps, x, x_trace, u_trace, idx_all,
+                                               true_idx_all, pred_all, err, ws.ll, opts, st)
+                    : launch_persistent2<1024>(pl, layers, heads, n_layers, K, eps, x, x_trace, u_trace, idx_all,
+                                               true_idx_all, pred_all, err, ws.ll, opts, st);
       return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
     }
     if (want == 2) return MOE_ERR_UNSUPPORTED;
+  }
+  if (want == 3) {
+    const Persist pl = plan_persistent(layers, heads, n_layers, T, K, K_next, use_predicted_routing);
+    if (!pl.ok || pl.ll_bytes > llb) return MOE_ERR_UNSUPPORTED;
+    if (cudaMemsetAsync(ws.ll, 0, pl.ll_bytes, st) != cudaSuccess) return MOE_ERR_CUDA;
+    const cudaError_t e =
+        H == 2048 ? launch_persistent<2048>(pl, layers, heads, n_layers, K, eps, x, x_trace, u_trace, idx_all,
+                                            true_idx_all, pred_all, err, ws.ll, opts, st)
+                  : launch_persistent<1024>(pl, layers, heads, n_layers, K, eps, x, x_trace, u_trace, idx_all,
+                                            true_idx_all, pred_all, err, ws.ll, opts, st);
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   }
 
   const size_t TK = static_cast<size_t>(T) * K, TKn = static_cast<size_t>(T) * K_next;
@@ -861,7 +1113,7 @@ moe_status moe_stack_decode(const moe_layer* layers, const moe_prerouter* heads,
     if (s != MOE_OK) return s;
     int32_t* idx_true = true_idx_all ? true_idx_all + l * TK : (idx_all && !use_predicted_routing ? idx_all + l * TK
                                                                                                     : ws.idx_true);
-    s = moe_route_topk(L, u, T, K, ws.logits, idx_true, ws.w, stream);
+    s = moe_route_topk(L, u, T, K, ws.logits, idx_true, ws.w, err, stream);
     if (s != MOE_OK) return s;
     const int32_t* idx_exec = idx_true;
     if (use_predicted_routing && l > 0) {
@@ -871,11 +1123,14 @@ moe_status moe_stack_decode(const moe_layer* layers, const moe_prerouter* heads,
     if (idx_all && idx_all + l * TK != idx_exec &&
         cudaMemcpyAsync(idx_all + l * TK, idx_exec, TK * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
       return MOE_ERR_CUDA;
-    s = moe_expert_forward(L, u, T, K, idx_exec, ws.w, x, 2, nullptr, ws.ews, ws.ews_bytes, stream);
+    const long long gemm_to = (opts && opts->timeout_ns > 0) ? opts->timeout_ns : kGemmTimeoutNs;
+    const int drop = (opts && opts->test_drop_layer == l + 1) ? opts->test_drop_cta : -1;
+    s = expert_forward_entry(L, u, T, K, idx_exec, ws.w, x, 2, nullptr, ws.ews, ws.ews_bytes, err, gemm_to, drop,
+                             stream);
     if (s != MOE_OK) return s;
     if (heads) {
       int32_t* pred = pred_all ? pred_all + l * TKn : ((l & 1) ? ws.pred1 : ws.pred0);
-      s = prerouter_predict(&heads[l], u, idx_exec, T, K, K_next, pred, ws.scores, ws.pws, ws.pws_bytes, stream);
+      s = prerouter_predict(&heads[l], u, idx_exec, T, K, K_next, pred, ws.scores, ws.pws, ws.pws_bytes, err, stream);
       if (s != MOE_OK) return s;
       pred_prev = pred;
     }
@@ -897,20 +1152,23 @@ constexpr size_t kStaticScratchBytes = MOE_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_scratch_once[kMaxDevices];
+std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices];
-cudaError_t g_scratch_err[kMaxDevices];
 
-// Device address of the scratch array on the current device (set up on first use).
+// Device address of the scratch array on the current device, looked up on first use.  A failed lookup is
+// not remembered: the next call tries again.
 moe_status static_scratch(void** ptr) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
-  std::call_once(g_scratch_once[dev], [dev] {
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
     void* p = nullptr;
-    g_scratch_err[dev] = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();  // leave no sticky launch status behind
+      return MOE_ERR_CUDA;
+    }
     g_scratch_ptr[dev] = p;
-  });
-  if (g_scratch_err[dev] != cudaSuccess || !g_scratch_ptr[dev]) return MOE_ERR_CUDA;
+  }
   *ptr = g_scratch_ptr[dev];
   return MOE_OK;
 }
@@ -923,7 +1181,7 @@ size_t moe_noalloc_scratch_bytes(void) { return kStaticScratchBytes; }
 
 moe_status moe_expert_forward_noalloc(const moe_layer* L, const uint16_t* u, int32_t T, int32_t K,
                                       const int32_t* idx, const float* w, void* out, int32_t out_mode,
-                                      int32_t* perm_out, void* stream) {
+                                      int32_t* perm_out, int32_t* err_word, void* stream) {
   moe_status s = check_layer(L, T, K);
   if (s != MOE_OK) return s;
   if (out_mode < 0 || out_mode > 2) return MOE_ERR_INVALID_ARG;
@@ -932,7 +1190,8 @@ moe_status moe_expert_forward_noalloc(const moe_layer* L, const uint16_t* u, int
   void* scratch = nullptr;
   s = static_scratch(&scratch);
   if (s != MOE_OK) return s;
-  return moe_expert_forward(L, u, T, K, idx, w, out, out_mode, perm_out, scratch, kStaticScratchBytes, stream);
+  return moe_expert_forward(L, u, T, K, idx, w, out, out_mode, perm_out, scratch, kStaticScratchBytes, err_word,
+                            stream);
 }
 
 }  // extern "C"

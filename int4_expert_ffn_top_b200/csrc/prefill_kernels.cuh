@@ -3,7 +3,7 @@
 // tile list, LoRA-A products for many tokens, and the gather-combine.
 #pragma once
 
-#include "grouped_gemm.cuh"
+#include "grouped_gemm3.cuh"
 #include "layer_kernels.cuh"
 
 namespace moe {
@@ -90,10 +90,13 @@ __global__ void __launch_bounds__(kChunk) bucket_place_kernel(const int32_t* __r
 
 // Token operand rows in fp16: rows [0, TK) are the slots in bucket order (the
 // slot's token), rows [TK, TK+T) the tokens in order (shared expert).  Also the
-// gating weight of each sorted slot.
+// gating weight of each sorted slot.  Each 8-element block is stored in pair
+// order (u_j, u_{j+4}), j = 0..3, the K order of the dequantised weight tiles.
+// Activations fp16 cannot hold (|u| > 65504 or not finite) report MOE_ERR_RANGE
+// into err (checked on the shared-expert rows, which hold every token once).
 __global__ void __launch_bounds__(256) permute_kernel(const uint16_t* __restrict__ u, int T, int K, int H,
                                                       const int32_t* __restrict__ perm, const float* __restrict__ w,
-                                                      uint16_t* __restrict__ X, float* __restrict__ w_pos) {
+                                                      uint16_t* __restrict__ X, float* __restrict__ w_pos, int* err) {
   const int row = blockIdx.x;
   const int TK = T * K;
   int tok;
@@ -106,16 +109,22 @@ __global__ void __launch_bounds__(256) permute_kernel(const uint16_t* __restrict
   }
   const uint4* src = reinterpret_cast<const uint4*>(u + static_cast<size_t>(tok) * H);
   uint4* dst = reinterpret_cast<uint4*>(X + static_cast<size_t>(row) * H);
+  bool bad = false;
   for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
     const uint4 v = src[c];
     const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[4];
+    uint16_t e[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      o[i] = bf16_to_f16_bits(static_cast<uint16_t>(vw[i] & 0xffffu)) |
-             (static_cast<uint32_t>(bf16_to_f16_bits(static_cast<uint16_t>(vw[i] >> 16))) << 16);
-    dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
+    for (int i = 0; i < 4; ++i) {
+      const uint16_t lo = static_cast<uint16_t>(vw[i] & 0xffffu), hi = static_cast<uint16_t>(vw[i] >> 16);
+      bad |= !(fabsf(bf16_bits_to_float(lo)) <= kF16Max) || !(fabsf(bf16_bits_to_float(hi)) <= kF16Max);
+      e[2 * i] = bf16_to_f16_bits(lo);
+      e[2 * i + 1] = bf16_to_f16_bits(hi);
+    }
+    dst[c] = make_uint4(e[0] | (static_cast<uint32_t>(e[4]) << 16), e[1] | (static_cast<uint32_t>(e[5]) << 16),
+                        e[2] | (static_cast<uint32_t>(e[6]) << 16), e[3] | (static_cast<uint32_t>(e[7]) << 16));
   }
+  if (bad && row >= TK) report(err, 6);
 }
 
 // Tile lists of both GEMMs: per expert (then the shared expert) its token
@@ -159,6 +168,7 @@ __global__ void __launch_bounds__(kThreads) lora_a_tokens_kernel(const uint16_t*
                                                                  const uint16_t* __restrict__ A_gate,
                                                                  const uint16_t* __restrict__ A_up, float* __restrict__ g,
                                                                  float* __restrict__ t1, float* __restrict__ t2) {
+  // (the activation range is checked by permute_kernel, which reads every token)
   constexpr int H = NCH8 * 8;
   constexpr int SEG8 = (H / 16) < 32 ? (H / 16) : 32;
   extern __shared__ uint4 smem[];
@@ -168,7 +178,7 @@ __global__ void __launch_bounds__(kThreads) lora_a_tokens_kernel(const uint16_t*
   const int t0 = blockIdx.x * TB, nt = min(TB, T - t0);
   if (threadIdx.x < TB) tok[threadIdx.x] = t0 + min(static_cast<int>(threadIdx.x), nt - 1);
   __syncthreads();
-  stage_tokens(u, H, tok, nt, us, nullptr, sum16, false);
+  stage_tokens(u, H, tok, nt, us, nullptr, sum16, false, nullptr);
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.y * kWarps + warp;  // 0: shared gate; 1..r: A_gate; r+1..2r: A_up
@@ -202,7 +212,7 @@ __global__ void __launch_bounds__(kThreads) lora_a_tokens_kernel(const uint16_t*
 
 // LoRA-A products on the SwiGLU output rows: t[row][i] = A_row[i] . h[row] with
 // A = A_down_shared for rows >= TK, else the routed expert's A (if any).
-// One warp per (row, i); h rows are fp16 in natural order.
+// One warp per (row, i); h rows are fp16 in pair order, A rows in natural order.
 __global__ void __launch_bounds__(kThreads) lora_a_rows_kernel(const uint16_t* __restrict__ h, int I, int TK, int nrows,
                                                                int row_begin, int r, const uint16_t* __restrict__ A_sd,
                                                                const uint16_t* __restrict__ A_ex,
@@ -216,8 +226,14 @@ __global__ void __launch_bounds__(kThreads) lora_a_rows_kernel(const uint16_t* _
   else A = A_ex + (static_cast<size_t>(idx[perm[row]]) * r + i) * I;
   const uint16_t* hr = h + static_cast<size_t>(row) * I;
   float acc = 0.f;
-  for (int c = lane; c < I / 8; c += 32)
-    acc = dot_chunk_f16(reinterpret_cast<const uint4*>(A)[c], reinterpret_cast<const uint4*>(hr)[c], acc);
+  for (int c = lane; c < I / 8; c += 32) {
+    const uint4 w = reinterpret_cast<const uint4*>(A)[c];
+    const uint4 hv = reinterpret_cast<const uint4*>(hr)[c];
+    acc = dot2_mix(prmt(w.x, w.z, 0x5410u), hv.x, acc);  // A chunk to pair order
+    acc = dot2_mix(prmt(w.x, w.z, 0x7632u), hv.y, acc);
+    acc = dot2_mix(prmt(w.y, w.w, 0x5410u), hv.z, acc);
+    acc = dot2_mix(prmt(w.y, w.w, 0x7632u), hv.w, acc);
+  }
   acc = warp_reduce(acc);
   if (lane == 0) t[static_cast<size_t>(row) * r + i] = acc;
 }

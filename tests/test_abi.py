@@ -66,26 +66,26 @@ def test_host_side_rejections(lib):
     from int4_expert_ffn_top_b200 import _lib
     L = _lib.moe_layer()
     # null layer / null pointers / bad shapes fail before any launch
-    assert lib.moe_route_topk(None, None, 1, 4, None, None, None, None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_route_topk(None, None, 1, 4, None, None, None, None, None) == _lib.MOE_ERR_INVALID_ARG
     assert lib.moe_rmsnorm_bf16(None, -1, 2048, 1e-6, None, None) == _lib.MOE_ERR_INVALID_ARG
     assert lib.moe_rmsnorm_bf16(None, 0, 2048, 1e-6, None, None) == _lib.MOE_OK
     L.H, L.E, L.I, L.I_s, L.r = 2048, 256, 512, 512, 16
-    assert lib.moe_route_topk(ctypes.byref(L), None, 1, 9, None, None, None, None) == _lib.MOE_ERR_UNSUPPORTED
+    assert lib.moe_route_topk(ctypes.byref(L), None, 1, 9, None, None, None, None, None) == _lib.MOE_ERR_UNSUPPORTED
     L.H = 2000
-    assert lib.moe_route_topk(ctypes.byref(L), None, 1, 4, None, None, None, None) == _lib.MOE_ERR_UNSUPPORTED
+    assert lib.moe_route_topk(ctypes.byref(L), None, 1, 4, None, None, None, None, None) == _lib.MOE_ERR_UNSUPPORTED
     L.H = 2048
     # router matrix missing
-    assert lib.moe_route_topk(ctypes.byref(L), None, 1, 4, None, None, None, None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_route_topk(ctypes.byref(L), None, 1, 4, None, None, None, None, None) == _lib.MOE_ERR_INVALID_ARG
     assert lib.moe_expert_forward(ctypes.byref(L), None, 1, 4, None, None, None, 0, None, None, 0,
-                                  None) == _lib.MOE_ERR_INVALID_ARG
+                                  None, None) == _lib.MOE_ERR_INVALID_ARG
     assert lib.moe_expert_forward(ctypes.byref(L), None, 1, 4, None, None, None, 7, None, None, 0,
-                                  None) == _lib.MOE_ERR_INVALID_ARG
+                                  None, None) == _lib.MOE_ERR_INVALID_ARG
     P = _lib.moe_prerouter()
     P.H, P.E, P.P, P.E_next = 2048, 256, 256, 256
     assert lib.prerouter_predict(ctypes.byref(P), None, None, 1, 4, 9, None, None, None, 0,
-                                 None) == _lib.MOE_ERR_UNSUPPORTED
+                                 None, None) == _lib.MOE_ERR_UNSUPPORTED
     assert lib.prerouter_predict(ctypes.byref(P), None, None, 1, 4, 4, None, None, None, 0,
-                                 None) == _lib.MOE_ERR_INVALID_ARG
+                                 None, None) == _lib.MOE_ERR_INVALID_ARG
     assert lib.moe_stack_decode(None, None, 0, 1, 4, 4, 1e-6, None, None, None, None, None, None, 0, None, None,
                                 None, 0, None) == _lib.MOE_ERR_INVALID_ARG
 
@@ -99,15 +99,15 @@ def test_token_limit_is_rejected_on_the_host(lib):
     L = _lib.moe_layer()
     L.H, L.E, L.I, L.I_s, L.r = 2048, 256, 512, 512, 16
     big = _lib.MOE_MAX_TOKENS + 1
-    assert lib.moe_route_topk(ctypes.byref(L), None, big, 4, None, None, None, None) == _lib.MOE_ERR_UNSUPPORTED
+    assert lib.moe_route_topk(ctypes.byref(L), None, big, 4, None, None, None, None, None) == _lib.MOE_ERR_UNSUPPORTED
     assert lib.moe_expert_forward(ctypes.byref(L), None, big, 4, None, None, None, 0, None, None, 0,
-                                  None) == _lib.MOE_ERR_UNSUPPORTED
+                                  None, None) == _lib.MOE_ERR_UNSUPPORTED
     assert lib.moe_workspace_size(ctypes.byref(L), big, 4) == 0
     assert lib.moe_workspace_size(ctypes.byref(L), _lib.MOE_MAX_TOKENS, 4) > 0
     P = _lib.moe_prerouter()
     P.H, P.E, P.P, P.E_next = 2048, 256, 256, 256
     assert lib.prerouter_predict(ctypes.byref(P), None, None, big, 4, 4, None, None, None, 0,
-                                 None) == _lib.MOE_ERR_UNSUPPORTED
+                                 None, None) == _lib.MOE_ERR_UNSUPPORTED
     assert lib.prerouter_workspace_size(ctypes.byref(P), big) == 0
     assert lib.moe_stack_workspace_size(ctypes.byref(L), None, 1, big, 4, 4) == 0
 
@@ -123,14 +123,14 @@ def test_workspace_sizes_grow_with_tokens(lib):
     assert b >= (64 * 4 + 64) * 512 * 2
 
 
-def test_stack_probe_tool_parses_its_arguments():
-    """The profiling/tracing driver named in profiles/ is importable and parses its options without a GPU."""
+def test_bench_diagnostic_mode_parses_its_arguments():
+    """The profiling/tracing mode named in profiles/ (bench.py --diag-stack) parses its options without a GPU."""
     import subprocess
     import sys
-    r = subprocess.run([sys.executable, "-m", "int4_expert_ffn_top_b200.stack_probe", "--help"],
+    r = subprocess.run([sys.executable, "bench.py", "--help"],
                        cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))), capture_output=True, text=True,
                        timeout=300)
-    assert r.returncode == 0 and "--trace" in r.stdout
+    assert r.returncode == 0 and "--diag-stack" in r.stdout and "--trace" in r.stdout
 
 
 def test_expert_block_layout_decodes_back_to_the_expert():
@@ -202,9 +202,9 @@ def test_well_formed_calls_pass_every_host_check(lib):
     L, P = _fake_layer(0x10000000), _fake_head(0x20000000)
     dev = 0x30000000
     assert lib.moe_expert_forward(ctypes.byref(L), dev, 1, 4, dev, dev, dev, 0, None, FAKE_WS, 0,
-                                  None) == _lib.MOE_ERR_WORKSPACE
+                                  None, None) == _lib.MOE_ERR_WORKSPACE
     assert lib.prerouter_predict(ctypes.byref(P), dev, dev, 1, 4, 4, dev, dev, FAKE_WS, 0,
-                                 None) == _lib.MOE_ERR_WORKSPACE
+                                 None, None) == _lib.MOE_ERR_WORKSPACE
     layers = (_lib.moe_layer * 3)(*[_fake_layer(0x10000000 * (l + 1)) for l in range(3)])
     heads = (_lib.moe_prerouter * 3)(*[_fake_head(0x40000000 * (l + 1)) for l in range(3)])
     assert lib.moe_stack_decode(layers, heads, 3, 1, 4, 4, 1e-6, dev, None, None, None, None, None, 0, None, None,
@@ -274,7 +274,7 @@ int main(void) {
   memset(&L, 0, sizeof L);
   L.H = 2048; L.E = 256; L.I = 512; L.I_s = 512; L.r = 16;
   printf("%s|%zu|%zu|%d|%zu\n", moe_status_string(MOE_ERR_WORKSPACE), moe_expert_block_bytes(2048, 512),
-         moe_qrow_bytes(2048, 8), (int)moe_route_topk(&L, NULL, 1, 4, NULL, NULL, NULL, NULL),
+         moe_qrow_bytes(2048, 8), (int)moe_route_topk(&L, NULL, 1, 4, NULL, NULL, NULL, NULL, NULL),
          moe_workspace_size(&L, MOE_MAX_TOKENS + 1, 4));
   return 0;
 }

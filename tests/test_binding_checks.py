@@ -82,12 +82,15 @@ def test_expert_forward_passes_arguments_in_abi_order(rec):
     name, a = rec.calls[-1]
     assert name == "moe_expert_forward"
     assert a[1:] == (u.data_ptr(), T, K, idx.data_ptr(), w.data_ptr(), out.data_ptr(), 0, perm.data_ptr(),
-                     work.data_ptr(), 4096, 0)
+                     work.data_ptr(), 4096, None, 0)
+    err = i32(1)
+    M.moe_expert_forward(FakeLayer(), u, K, idx, w, out, M.OUT_F32, work, err_word=err, stream=0)
+    assert rec.calls[-1][1][-2:] == (err.data_ptr(), 0)
     out16 = u16()
     M.moe_expert_forward_noalloc(FakeLayer(), u, K, idx, w, out16, M.OUT_BF16, stream=0)
     name, a = rec.calls[-1]
     assert name == "moe_expert_forward_noalloc"
-    assert a[1:] == (u.data_ptr(), T, K, idx.data_ptr(), w.data_ptr(), out16.data_ptr(), 1, None, 0)
+    assert a[1:] == (u.data_ptr(), T, K, idx.data_ptr(), w.data_ptr(), out16.data_ptr(), 1, None, None, 0)
 
 
 def test_zero_tokens_and_a_larger_output_are_accepted(rec):
@@ -98,14 +101,14 @@ def test_zero_tokens_and_a_larger_output_are_accepted(rec):
 def test_route_rmsnorm_prerouter_argument_order(rec):
     u, logits, idx, w = u16(), f32(T, E), i32(T, K), f32(T, K)
     M.moe_route_topk(FakeLayer(), u, K, logits, idx, w, stream=0)
-    assert rec.calls[-1][1][1:] == (u.data_ptr(), T, K, logits.data_ptr(), idx.data_ptr(), w.data_ptr(), 0)
+    assert rec.calls[-1][1][1:] == (u.data_ptr(), T, K, logits.data_ptr(), idx.data_ptr(), w.data_ptr(), None, 0)
     x = f32(T, H)
     M.moe_rmsnorm_bf16(x, 1e-6, u, stream=0)
     assert rec.calls[-1] == ("moe_rmsnorm_bf16", (x.data_ptr(), T, H, 1e-6, u.data_ptr(), 0))
     sel, pred, scores, work = i32(T, K), i32(T, 3), f32(T, E), ws()
     M.prerouter_predict(FakeHead(), u, sel, 3, pred, scores, work, stream=0)
     assert rec.calls[-1][1][1:] == (u.data_ptr(), sel.data_ptr(), T, K, 3, pred.data_ptr(), scores.data_ptr(),
-                                    work.data_ptr(), 4096, 0)
+                                    work.data_ptr(), 4096, None, 0)
 
 
 def test_stack_decode_argument_order_and_trace_size(rec):

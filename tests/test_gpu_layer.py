@@ -493,3 +493,79 @@ def test_expert_forward_grouped_gemm_full_size_layer(cuda_ok):
     sample = np.arange(0, T, 37)
     ref = oracle_out(lay, u[sample], idx[sample], w[sample])
     assert_close_inf(out[sample], ref)
+
+
+# ----------------------------------------------------------------------------- device-side status (error word)
+def _status_calls(layer: Layer, ub, K):
+    """Run the three per-layer entry points on u with one error word each; returns their statuses."""
+    m = M()
+    T, cfg = ub.shape[0], layer.cfg
+    errs = [torch.zeros((1,), dtype=torch.int32, device=DEV) for _ in range(3)]
+    u = dev_bits(ub)
+    logits = torch.empty((T, cfg.E), device=DEV)
+    idx = torch.empty((T, K), dtype=torch.int32, device=DEV)
+    w = torch.empty((T, K), device=DEV)
+    m.moe_route_topk(layer.dev, u, K, logits, idx, w, err_word=errs[0])
+    sel = torch.from_numpy(np.tile(np.arange(K, dtype=np.int32), (T, 1))).to(DEV)
+    wfix = torch.full((T, K), 1.0 / K, device=DEV)
+    out = torch.empty((T, cfg.H), device=DEV)
+    ws = m.workspace(m.moe_workspace_size(layer.dev, T, K))
+    m.moe_expert_forward(layer.dev, u, K, sel, wfix, out, 0, ws, err_word=errs[1])
+    pred = torch.empty((T, K), dtype=torch.int32, device=DEV)
+    scores = torch.empty((T, cfg.E_next), device=DEV)
+    pws = m.workspace(m.prerouter_workspace_size(layer.head, T))
+    m.prerouter_predict(layer.head, u, sel, K, pred, scores, pws, err_word=errs[2])
+    torch.cuda.synchronize()
+    return [int(e.item()) for e in errs], out.cpu().numpy().astype(np.float64)
+
+
+@pytest.mark.parametrize("T", [4, 64])  # GEMV path and grouped-GEMM path (64 x 2 slots)
+def test_activation_beyond_fp16_range_is_reported(c0, T):
+    """An activation fp16 cannot hold (|u| > 65504) sets MOE_ERR_RANGE in every entry point's error word."""
+    ub = inputs.activations(c0.cfg, step=41, T=T)
+    ok, _ = _status_calls(c0, ub, c0.cfg.K)
+    assert ok == [0, 0, 0]
+    bad = ub.copy()
+    bad[T // 2, 17] = inputs.f32_to_bf16_bits(np.array([7.0e4], np.float32))[0]
+    st, _ = _status_calls(c0, bad, c0.cfg.K)
+    assert st == [6, 6, 6]
+
+
+@pytest.mark.parametrize("T", [4, 64])
+@pytest.mark.parametrize("scale", [2.0 ** -4, 8.0])
+def test_expert_forward_parity_across_activation_scales(c0, T, scale):
+    """Activations below and above unit scale whose SwiGLU outputs stay in fp16's normal range (the envelope the
+    kernels compute in, see moe.h, Errors): parity with the oracle on both expert paths, and no status."""
+    cfg = c0.cfg
+    ub = inputs.f32_to_bf16_bits(inputs.bf16_bits_to_f32(inputs.activations(cfg, step=43, T=T)) * np.float32(scale))
+    u = u_vals(ub)
+    st, out = _status_calls(c0, ub, cfg.K)
+    assert st == [0, 0, 0]
+    idx = np.tile(np.arange(cfg.K), (T, 1))
+    w = np.full((T, cfg.K), 1.0 / cfg.K)
+    assert_close_inf(out, oracle_out(c0, u, idx, w), what=f"scale {scale}")
+
+
+@pytest.mark.parametrize("T", [4, 64])
+def test_swiglu_output_beyond_fp16_range_is_reported(c0, T):
+    """At 1000x unit-scale activations the SwiGLU outputs exceed fp16's range (both paths keep h in fp16): the
+    expert forward reports MOE_ERR_RANGE instead of returning silent infinities."""
+    ub = inputs.f32_to_bf16_bits(inputs.bf16_bits_to_f32(inputs.activations(c0.cfg, step=44, T=T)) * np.float32(1e3))
+    st, _ = _status_calls(c0, ub, c0.cfg.K)
+    assert st[0] == 0 and st[1] == 6
+
+
+def test_grouped_gemm_bounded_wait_reports_timeout(cuda_ok):
+    """A grouped-GEMM CTA whose first operand stage is never marked full (test hook): its waits run out, the
+    stack's error word says MOE_ERR_TIMEOUT, and the next call on the same context succeeds."""
+    m = M()
+    cfg = dataclasses.replace(CONFIGS[0], layers=2)
+    stack = m.DeviceStack(cfg, lambda l: inputs.layer(cfg, l))
+    T = 64  # 64 x 2 slots: the tensor-core path
+    x0 = inputs.bf16_bits_to_f32(inputs.activations(cfg, step=45, T=T))
+    res = run_stack(stack, cfg, T, x0, False,
+                    opts=m.stack_opts(path=m.PATH_LAYERS, timeout_ns=20_000_000, drop_layer=1, drop_cta=0))
+    assert res["err"] == 5
+    res2 = run_stack(stack, cfg, T, x0, False, opts=m.stack_opts(path=m.PATH_LAYERS))
+    assert res2["err"] == 0
+    _check_stack(cfg, lambda l: inputs.layer(cfg, l), T, res2, x0, range(cfg.layers))

@@ -66,6 +66,32 @@ def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row(cuda_ok):
             assert np.array_equal(pgot, pref)
 
 
+def _oracle_out(host, ub, idx, w):
+    u = inputs.bf16_bits_to_f32(ub).astype(np.float64)
+    y = O.routed_outputs(u, host["experts"], idx)
+    return O.combine(w, y, O.shared_gate(u, host["shared"]), O.shared_expert(u, host["shared"]))
+
+
+def test_noalloc_tensor_core_path_on_two_calls_in_a_row(cuda_ok):
+    """64 tokens x top-2 (128 slots) take the grouped-GEMM path, whose tensor maps, tile lists and bucket
+    histograms then live in the shared scratch array: two calls in a row with different routing agree with the
+    workspace entry point bit for bit and with the oracle."""
+    import int4_expert_ffn_top_b200 as M
+    cfg = CONFIGS[0]
+    host = inputs.layer(cfg, 3)
+    layer = M.DeviceLayer(cfg, host)
+    T = 64
+    assert M.moe_workspace_size(layer, T, cfg.K) <= M.moe_noalloc_scratch_bytes()
+    for call in range(2):
+        ub = inputs.activations(cfg, step=400 + call, T=T)
+        idx, w = _routing(host, ub, cfg.K)
+        if call:
+            idx = (idx + 5) % cfg.E  # different buckets from the first call
+        (ref, got), (pref, pgot) = _both(M, layer, ub, cfg.K, idx, w, 0)
+        assert np.array_equal(got, ref) and np.array_equal(pgot, pref)
+        assert_close_inf(got, _oracle_out(host, ub, idx, w), what=f"call {call}")
+
+
 def test_noalloc_rejects_requests_beyond_its_scratch(cuda_ok):
     import int4_expert_ffn_top_b200 as M
     cfg = CONFIGS[0]
