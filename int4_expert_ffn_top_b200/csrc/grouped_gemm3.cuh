@@ -3,84 +3,108 @@
 //
 // Per expert bucket D[o][t] = sum_k W[o][k] * X[t][k] ("swap AB": 128 weight
 // rows are the MMA M side, the bucket's tokens the N side).  A tile is 128
-// weight rows x up to 128 tokens; K advances one quantisation group (64) per
+// weight rows x up to 64 tokens; K advances one quantisation group (64) per
 // step.  One CTA per SM walks the device-built tile list (tiles c, c + grid,
 // ...), and every role runs the same sequence of (tile, step), so the pipeline
 // stays full across tiles:
 //  * warp 0, one lane (TMA): per tile the fp16 scales and biases of its 128 rows
 //    (a box of a 3-D byte map {record bytes, rows, experts} over the expert
-//    pool, two buffers); per step the 32 code bytes of each row (a box of a
-//    second map over the same bytes: 4 KB, dense [row][32 B], eight stages) and
-//    the step's token rows (2-D map, 128-byte swizzle, boxes of 32 rows, only as
-//    many as the tile has tokens);
-//  * warps 2..9 dequantise: thread (row r, half h) reads 16 code bytes (a warp
-//    reads 512 contiguous bytes), forms w = q*s + b in fp16 (one rounding) and
-//    stores four 16-byte chunks into the 128-byte-swizzled K-major A stage.  K
-//    inside each 8-element block is in "pair order" (q_j, q_{j+4}), the order
-//    the magic-exponent unpacking produces; the token operand is stored in the
-//    same order, so the products are those of the plain order;
-//  * warp 1, one lane (MMA): tcgen05.mma kind::f16 into one of two 128-column
-//    TMEM accumulators (tiles alternate), committing stage releases and
-//    accumulator-ready barriers;
-//  * warps 10..13 (epilogue, TMEM lane quadrant = warp % 4): drain the finished
-//    accumulator with tcgen05.ld while the next tile's main loop runs: SwiGLU of
+//    pool, two buffers when they fit); every four steps the 128 code bytes of
+//    each row (a box of a second map over the same bytes, 128-byte swizzle,
+//    16 KB, three stages); per step the step's token rows (2-D map, 128-byte
+//    swizzle, boxes of 32 rows, only as many as the tile has tokens);
+//  * warps 2..9 dequantise, two K steps per pass: thread (row r, half h) reads
+//    16 code bytes per step (lanes of a warp take 8 consecutive rows per
+//    128-byte wavefront, conflict-free under the swizzle), forms w = q*s + b in
+//    fp16 (one rounding) and stores four 16-byte chunks into the
+//    128-byte-swizzled K-major A stage.  K inside each 8-element block is in
+//    "pair order" (q_j, q_{j+4}), the order the magic-exponent unpacking
+//    produces; the token operand is stored in the same order, so the products
+//    are those of the plain order;
+//  * warp 1, one lane (MMA): tcgen05.mma kind::f16 into one of two sets of four
+//    64-column TMEM accumulators (tiles alternate); K slice c (16 wide) of
+//    every step goes to accumulator c, so four independent accumulation chains
+//    keep the tensor core busy at ~64 tokens per MMA; each commit releases the
+//    step's operand stages and, after a tile, its accumulators;
+//  * warps 10..17 (epilogue, TMEM lane quadrant = warp % 4, two warps per
+//    quadrant splitting the token columns): drain and add the finished
+//    accumulators with tcgen05.ld while the next tile's main loop runs: SwiGLU of
 //    interleaved gate/up rows (output in pair order, the next GEMM's token
 //    operand) or the down projection's LoRA delta and gating weight; staged in
 //    shared memory for coalesced fp16 stores; then the accumulator is released.
+// K must be a multiple of 128 (an even number of steps).
 // Every wait is bounded: a role whose wait runs out stops issuing copies or
 // MMAs and records MOE_ERR_TIMEOUT; before the CTA leaves, the copies and MMAs
 // it issued are waited for (bounded).
 #pragma once
 
-#include "grouped_gemm.cuh"
+#include "tc_primitives.cuh"
 
 namespace moe {
 namespace gg3 {
 
-using gg::bar_arrive;
-using gg::bar_expect_tx;
-using gg::bar_init;
-using gg::bar_test;
-using gg::bar_wait;
-using gg::EPI_DOWN;
-using gg::EPI_SWIGLU;
-using gg::instr_desc;
-using gg::mma_commit;
-using gg::mma_f16;
-using gg::sa;
-using gg::smem_desc;
-using gg::tma_load_2d;
-using gg::tmem_ld32;
-using gg::Tile;
+using tc::bar_arrive;
+using tc::bar_expect_tx;
+using tc::bar_init;
+using tc::bar_test;
+using tc::bar_wait;
+using tc::EPI_DOWN;
+using tc::EPI_SWIGLU;
+using tc::instr_desc;
+using tc::mma_commit;
+using tc::mma_f16;
+using tc::sa;
+using tc::smem_desc;
+using tc::tma_load_2d;
+using tc::tmem_ld32;
+using tc::Tile;
 
 constexpr int BM = 128;
-constexpr int BN = 128;
+constexpr int BN = 64;   // tokens per tile: buckets average ~50 tokens at prefill; keeps the token ring deep
 constexpr int BK = 64;
 constexpr int BROWS = 32;   // token rows per TMA box
-constexpr int RSTAGES = 8;  // raw code stages (4 KB each): the weight bytes in flight per SM
-constexpr int BSTAGES = 3;  // token stages (16 KB each)
-constexpr int ASTAGES = 3;  // dequantised weight stages (16 KB each)
+constexpr int RGROUPS = 4;  // quantisation groups per raw code load: 128-byte TMA rows (narrower rows cap the
+                            // TMA request rate well below the HBM bandwidth)
+constexpr int RSTAGES = 3;  // raw code stages (16 KB each): the weight bytes in flight per SM
+// Operand stages: a dequantised weight stage (16 KB) and a token stage (8 KB) per K step, released together by
+// the MMA warps' commits.
+constexpr int STAGES = 4;
+constexpr int BSTAGES = STAGES;
+constexpr int ASTAGES = STAGES;
 constexpr int kDqWarps = 8;
 constexpr int kDq = 32 * kDqWarps;
-constexpr int kEpi = 128;
-constexpr int kThreads = 64 + kDq + kEpi;  // TMA warp, MMA warp, dequant warps, epilogue warps
-constexpr int RAW_STAGE = BM * 32;
+constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant, splitting the tile's token columns
+constexpr int kEpi = 32 * kEpiWarps;
+constexpr int kMmaWarps = 1;  // MMA-issuing warps; warp 1 + w issues the chains w, w + kMmaWarps, ...
+constexpr int kThreads = 32 * (1 + kMmaWarps) + kDq + kEpi;  // TMA warp, MMA warps, dequant warps, epilogue warps
+constexpr int kWarpDq0 = 1 + kMmaWarps;                         // first dequantising warp
+constexpr int kWarpEpi0 = kWarpDq0 + kDqWarps;                  // first epilogue warp
+constexpr int RAW_STAGE = BM * 32 * RGROUPS;
 constexpr int A_STAGE = BM * BK * 2;
 constexpr int B_STAGE = BN * BK * 2;
 constexpr int SB_MAX = BM * 256;           // scales + biases of 128 rows, K <= 4096
-constexpr int STAGE_OUT = BN * BM * 2;     // epilogue staging: up to 128 tokens x 128 fp16
-constexpr uint32_t TMEM_COLS = 256;        // two 128-column accumulators
+constexpr int STAGE_OUT = BN * BM * 2;     // epilogue staging: up to BN tokens x 128 fp16
+// MMAs that accumulate into one TMEM accumulator run one after another (each waits for the previous sum), so a
+// tile's K steps are spread over ACC_CHAINS accumulators (MMA kk of every step into accumulator kk) that the
+// tensor core works on concurrently, and the epilogue adds them.  Two tiles in flight: 2 x ACC_CHAINS x BN columns.
+constexpr int ACC_CHAINS = 4;
+constexpr uint32_t TMEM_COLS = 2 * ACC_CHAINS * BN;
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + ASTAGES * A_STAGE;
 constexpr int OFF_RAW = OFF_B + BSTAGES * B_STAGE;
+constexpr int LORA_T = 2 * BN * 32 * 4;    // epilogue staging of the tile's LoRA t vectors (two sets, r <= 32) ...
 constexpr int OFF_OUT = OFF_RAW + RSTAGES * RAW_STAGE;
-constexpr int OFF_SB = OFF_OUT + STAGE_OUT;
+constexpr int OFF_LT = OFF_OUT + STAGE_OUT;
+constexpr int OFF_RS = OFF_LT + LORA_T;    // ... and of its gating weights
+constexpr int OFF_SB = OFF_RS + BN * 4;
 
 // Bytes per row of the scale/bias box: the K/64 scales and K/64 biases (4*K/64 bytes), at least one 16-byte
 // TMA unit (the row record's zero padding covers the rest).
 __host__ __device__ constexpr int sb_row_bytes(int K) { return (4 * (K / 64) + 15) / 16 * 16; }
-// Dynamic shared memory for reduction length K (two scale/bias buffers, barriers, alignment slack).
-__host__ __device__ constexpr int smem_bytes(int K) { return OFF_SB + 2 * BM * sb_row_bytes(K) + 512 + 1024; }
+// Dynamic shared memory for reduction length K with nsb scale/bias buffers (+ barriers, alignment slack).
+__host__ __device__ constexpr int smem_bytes(int K, int nsb) { return OFF_SB + nsb * BM * sb_row_bytes(K) + 512 + 1024; }
+// Scale/bias buffers for reduction length K: two (the next tile's scales load during this tile) when they fit.
+__host__ __device__ constexpr int sb_buffers(int K) { return smem_bytes(K, 2) <= 227 * 1024 ? 2 : 1; }
 
 struct Args {
   const Tile* tiles;
@@ -101,11 +125,13 @@ struct Args {
   int* err;
   long long timeout_ns;
   int drop_tile;  // test hook: the CTA working on this tile never marks its first weight stage full (-1: off)
+  int nsb;        // scale/bias buffers (sb_buffers(K))
 };
 
 // 3-D byte maps {record bytes, rows, experts} over the weight matrix of every expert block (pool) and of the
-// shared expert's block (one expert): boxes of the 32 code bytes of one group x 128 rows, and of the
-// scale/bias bytes x 128 rows.  2-D fp16 map of the token operand [rows][K], boxes of 64 x 32, 128-byte swizzle.
+// shared expert's block (one expert): boxes of the 128 code bytes of four groups x 128 rows (128-byte swizzle),
+// and of the scale/bias bytes x 128 rows.  2-D fp16 map of the token operand [rows][K], boxes of 64 x 32,
+// 128-byte swizzle.
 struct Maps {
   CUtensorMap pool_codes, pool_sb, shared_codes, shared_sb, tokens;
 };
@@ -136,13 +162,15 @@ MOE_DEV uint4 dequant_pair_order(uint32_t w, __half2 s2, __half2 b2) {
                     h2_bits(__hfma2(q3, s2, b2)));
 }
 
+static_assert(BK / 16 == ACC_CHAINS && ACC_CHAINS % kMmaWarps == 0 && TMEM_COLS <= 512, "accumulator chains");
+
 MOE_DEV uint32_t parity(int count, int stages) { return static_cast<uint32_t>(count / stages) & 1u; }
 
-// OR of v over the 128 epilogue threads (named barrier 1), so that they take the same branch.
+// OR of v over the 256 epilogue threads (named barrier 1), so that they take the same branch.
 MOE_DEV bool epi_any(bool v) {
   uint32_t r;
   asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n barrier.cta.red.or.pred q, 1, 128, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n barrier.cta.red.or.pred q, 1, 256, p;\n selp.u32 %0, 1, 0, q;\n}\n"
       : "=r"(r)
       : "r"(static_cast<uint32_t>(v))
       : "memory");
@@ -159,15 +187,15 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
   uint8_t* smB = sm + OFF_B;
   uint8_t* smRaw = sm + OFF_RAW;
   uint16_t* stage = reinterpret_cast<uint16_t*>(sm + OFF_OUT);
-  uint8_t* smSB = sm + OFF_SB;  // two buffers of BM * SB_ROW bytes
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smSB + 2 * BM * SB_ROW);
+  uint8_t* smSB = sm + OFF_SB;  // nsb buffers of BM * SB_ROW bytes
+  const int nsb = a.nsb;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smSB + nsb * BM * SB_ROW);
   uint64_t* raw_full = bars;
   uint64_t* raw_empty = raw_full + RSTAGES;
   uint64_t* b_full = raw_empty + RSTAGES;
-  uint64_t* b_empty = b_full + BSTAGES;
-  uint64_t* a_full = b_empty + BSTAGES;
-  uint64_t* a_empty = a_full + ASTAGES;
-  uint64_t* sb_full = a_empty + ASTAGES;  // [2]
+  uint64_t* a_full = b_full + STAGES;
+  uint64_t* st_empty = a_full + STAGES;   // both operand stages of a step are free (one commit per MMA warp)
+  uint64_t* sb_full = st_empty + STAGES;  // [2]
   uint64_t* sb_empty = sb_full + 2;       // [2]
   uint64_t* acc_full = sb_empty + 2;      // [2]
   uint64_t* acc_empty = acc_full + 2;     // [2]
@@ -178,25 +206,22 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
   if (tid == 0) {
     for (int s = 0; s < RSTAGES; ++s) {
       bar_init(raw_full + s, 1);
-      bar_init(raw_empty + s, kDq);
+      bar_init(raw_empty + s, kDqWarps);  // one elected arrival per warp
     }
-    for (int s = 0; s < BSTAGES; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       bar_init(b_full + s, 1);
-      bar_init(b_empty + s, 1);
-    }
-    for (int s = 0; s < ASTAGES; ++s) {
-      bar_init(a_full + s, kDq);
-      bar_init(a_empty + s, 1);
+      bar_init(a_full + s, kDqWarps);
+      bar_init(st_empty + s, kMmaWarps);
     }
     for (int s = 0; s < 2; ++s) {
       bar_init(sb_full + s, 1);
-      bar_init(sb_empty + s, kDq);
-      bar_init(acc_full + s, 1);
-      bar_init(acc_empty + s, kEpi);
+      bar_init(sb_empty + s, kDqWarps);
+      bar_init(acc_full + s, kMmaWarps);
+      bar_init(acc_empty + s, kEpiWarps);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) {
+  if (warp == 1) {  // the first MMA warp owns the TMEM allocation
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(sa(tmem_slot)),
                  "r"(TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -218,8 +243,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
         const CUtensorMap* cmap = sh ? &maps.shared_codes : &maps.pool_codes;
         const CUtensorMap* smap = sh ? &maps.shared_sb : &maps.pool_sb;
         const int ez = sh ? 0 : tile.e, y = tile.mt * BM;
-        const int tb = n_sb & 1;
-        if (!bar_wait(sb_empty + tb, parity(n_sb, 2) ^ 1u, a.timeout_ns)) {
+        const int tb = n_sb % nsb;
+        if (!bar_wait(sb_empty + tb, parity(n_sb, nsb) ^ 1u, a.timeout_ns)) {
           fail = 1;
           break;
         }
@@ -230,14 +255,16 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
 #pragma unroll 1
         for (int kt = 0; kt < KT; ++kt) {
           const int rs = n_raw % RSTAGES, bs = n_b % BSTAGES;
-          if (!bar_wait(raw_empty + rs, parity(n_raw, RSTAGES) ^ 1u, a.timeout_ns)) {
-            fail = 1;
-            break;
+          if (kt % RGROUPS == 0) {
+            if (!bar_wait(raw_empty + rs, parity(n_raw, RSTAGES) ^ 1u, a.timeout_ns)) {
+              fail = 1;
+              break;
+            }
+            bar_expect_tx(raw_full + rs, RAW_STAGE);
+            tma_load_3d(smRaw + rs * RAW_STAGE, cmap, kt * 32, y, ez, raw_full + rs);
+            ++n_raw;
           }
-          bar_expect_tx(raw_full + rs, RAW_STAGE);
-          tma_load_3d(smRaw + rs * RAW_STAGE, cmap, kt * 32, y, ez, raw_full + rs);
-          ++n_raw;
-          if (!bar_wait(b_empty + bs, parity(n_b, BSTAGES) ^ 1u, a.timeout_ns)) {
+          if (!bar_wait(st_empty + bs, parity(n_b, STAGES) ^ 1u, a.timeout_ns)) {
             fail = 1;
             break;
           }
@@ -257,11 +284,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
         for (int q = n_b > BSTAGES ? n_b - BSTAGES : 0; q < n_b; ++q)
           bar_wait(b_full + q % BSTAGES, parity(q, BSTAGES), a.timeout_ns);
 #pragma unroll 1
-        for (int q = n_sb > 2 ? n_sb - 2 : 0; q < n_sb; ++q) bar_wait(sb_full + (q & 1), parity(q, 2), a.timeout_ns);
+        for (int q = n_sb > nsb ? n_sb - nsb : 0; q < n_sb; ++q) bar_wait(sb_full + q % nsb, parity(q, nsb), a.timeout_ns);
       }
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issue (one thread)
+  } else if (warp < kWarpDq0) {
+    // ---------------------------------------------------------------- MMA issue
+    const int ch = warp - 1;
     if (lane == 0) {
       int g = 0, it = 0, last_ab = -1;
       uint32_t last_par = 0;
@@ -274,190 +302,225 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
           break;
         }
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const uint32_t d = tmem + static_cast<uint32_t>(ab * BM);
+        const uint32_t d = tmem + static_cast<uint32_t>(ab * ACC_CHAINS * BN);
         const uint32_t idesc = instr_desc((tile.n + 15) & ~15);
 #pragma unroll 1
         for (int kt = 0; kt < KT; ++kt, ++g) {
-          const int as = g % ASTAGES, bs = g % BSTAGES;
-          if (!bar_wait(a_full + as, parity(g, ASTAGES), a.timeout_ns) ||
-              !bar_wait(b_full + bs, parity(g, BSTAGES), a.timeout_ns)) {
+          const int s = g % STAGES;
+          if (!bar_wait(a_full + s, parity(g, STAGES), a.timeout_ns) ||
+              !bar_wait(b_full + s, parity(g, STAGES), a.timeout_ns)) {
             fail = 1;
             break;
           }
           asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-          const uint32_t a0 = sa(smA + as * A_STAGE), b0 = sa(smB + bs * B_STAGE);
+          const uint32_t a0 = sa(smA + s * A_STAGE), b0 = sa(smB + s * B_STAGE);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            mma_f16(d, smem_desc(a0 + kk * 32), smem_desc(b0 + kk * 32), idesc, (kt | kk) != 0);
-          mma_commit(a_empty + as);
-          mma_commit(b_empty + bs);
+          for (int c = ch; c < ACC_CHAINS; c += kMmaWarps)  // K slice c of the step into accumulator c
+            mma_f16(d + c * BN, smem_desc(a0 + c * 32), smem_desc(b0 + c * 32), idesc, kt != 0);
+          mma_commit(st_empty + s);
         }
         mma_commit(acc_full + ab);  // also on failure: completes once every MMA issued into this buffer has
         last_ab = ab;
         last_par = parity(it, 2);
       }
-      // never release TMEM with MMAs in flight: wait for the last commit
+      // never release TMEM with MMAs in flight: wait for the last commit (this chain's part of it)
       if (fail && last_ab >= 0) bar_wait(acc_full + last_ab, last_par, a.timeout_ns);
     }
-  } else if (warp < 2 + kDqWarps) {
+  } else if (warp < kWarpEpi0) {
     // ---------------------------------------------------------------- dequantising warps
-    const int d = tid - 64;
-    const int r = d >> 1, h = d & 1;
+    const int d = tid - 32 * kWarpDq0;
+    // lanes l and l+8 take the two halves of one row; a 128-byte wavefront covers 8 consecutive rows
+    const int r = 16 * (d >> 5) + (lane & 7) + 8 * (lane >> 4), h = (lane >> 3) & 1;
     const bool vec8 = (KT & 7) == 0;
-    int g = 0, it = 0;
+    int g = 0, it = 0, nr = 0;
 #pragma unroll 1
     for (int ti = blockIdx.x; ti < n_tiles && !fail; ti += gridDim.x, ++it) {
-      const int tb = it & 1;
+      const int tb = it % nsb;
       const uint16_t* sbr = reinterpret_cast<const uint16_t*>(smSB + tb * BM * SB_ROW + r * SB_ROW);
-      if (!bar_wait(sb_full + tb, parity(it, 2), a.timeout_ns)) {
+      if (__any_sync(0xffffffffu, !bar_wait(sb_full + tb, parity(it, nsb), a.timeout_ns))) {
         fail = 1;
         break;
       }
       // a row's scale/bias run sits in one bank for all rows: read them 8 groups at a time
       uint4 s8 = make_uint4(0, 0, 0, 0), b8 = s8;
 #pragma unroll 1
-      for (int kt = 0; kt < KT; ++kt, ++g) {
-        const int rs = g % RSTAGES, as = g % ASTAGES;
+      for (int kt = 0; kt < KT; kt += 2, g += 2) {  // two K steps per pass (KT is even): more independent work per
+                                                   // hand-off
         if (vec8 && (kt & 7) == 0) {
           s8 = reinterpret_cast<const uint4*>(sbr)[kt >> 3];
           b8 = reinterpret_cast<const uint4*>(sbr + KT)[kt >> 3];
         }
-        uint16_t sv, bv;
+        uint32_t sw, bw;  // low half: step kt, high half: step kt + 1
         if (vec8) {
-          const int j = (kt & 7) >> 1, shf = 16 * (kt & 1);
-          const uint32_t sw = j == 0 ? s8.x : j == 1 ? s8.y : j == 2 ? s8.z : s8.w;
-          const uint32_t bw = j == 0 ? b8.x : j == 1 ? b8.y : j == 2 ? b8.z : b8.w;
-          sv = static_cast<uint16_t>(sw >> shf);
-          bv = static_cast<uint16_t>(bw >> shf);
+          const int j = (kt & 7) >> 1;
+          sw = j == 0 ? s8.x : j == 1 ? s8.y : j == 2 ? s8.z : s8.w;
+          bw = j == 0 ? b8.x : j == 1 ? b8.y : j == 2 ? b8.z : b8.w;
         } else {
-          sv = sbr[kt];
-          bv = sbr[KT + kt];
+          sw = sbr[kt] | (static_cast<uint32_t>(sbr[kt + 1]) << 16);
+          bw = sbr[KT + kt] | (static_cast<uint32_t>(sbr[KT + kt + 1]) << 16);
         }
-        if (!bar_wait(raw_full + rs, parity(g, RSTAGES), a.timeout_ns)) {
+        const int rs = nr % RSTAGES, grp = kt % RGROUPS;  // grp is even: groups grp and grp + 1 of the raw stage
+        if (__any_sync(0xffffffffu, grp == 0 && !bar_wait(raw_full + rs, parity(nr, RSTAGES), a.timeout_ns))) {
           fail = 1;
           break;
         }
-        const uint4 q = *reinterpret_cast<const uint4*>(smRaw + rs * RAW_STAGE + r * 32 + h * 16);
-        bar_arrive(raw_empty + rs);
-        const __half2 s2 = __half2half2(__ushort_as_half(sv)), b2 = __half2half2(__ushort_as_half(bv));
-        const uint4 w0 = dequant_pair_order(q.x, s2, b2), w1 = dequant_pair_order(q.y, s2, b2);
-        const uint4 w2 = dequant_pair_order(q.z, s2, b2), w3 = dequant_pair_order(q.w, s2, b2);
-        if (!bar_wait(a_empty + as, parity(g, ASTAGES) ^ 1u, a.timeout_ns)) {  // the MMA may still read it
-          fail = 1;
-          break;
+        // chunk (2 grp + h) of row r, 128-byte swizzle: 16-byte chunk c of a row sits at c ^ (r % 8)
+        const uint8_t* rrow = smRaw + rs * RAW_STAGE + r * 128;
+        const uint4 q0 = *reinterpret_cast<const uint4*>(rrow + (((2 * grp + h) ^ (r & 7)) << 4));
+        const uint4 q1 = *reinterpret_cast<const uint4*>(rrow + (((2 * grp + 2 + h) ^ (r & 7)) << 4));
+        if (grp + 1 == RGROUPS - 1 || kt + 1 == KT - 1) {
+          __syncwarp();
+          if (lane == 0) bar_arrive(raw_empty + rs);
+          ++nr;
         }
-        uint8_t* dd = smA + as * A_STAGE + (r >> 3) * 1024 + (r & 7) * 128;
+        const __half2 s0 = __half2half2(__ushort_as_half(static_cast<uint16_t>(sw))),
+                      b0 = __half2half2(__ushort_as_half(static_cast<uint16_t>(bw)));
+        const __half2 s1 = __half2half2(__ushort_as_half(static_cast<uint16_t>(sw >> 16))),
+                      b1 = __half2half2(__ushort_as_half(static_cast<uint16_t>(bw >> 16)));
+        uint4 w[8];
+        w[0] = dequant_pair_order(q0.x, s0, b0);
+        w[1] = dequant_pair_order(q0.y, s0, b0);
+        w[2] = dequant_pair_order(q0.z, s0, b0);
+        w[3] = dequant_pair_order(q0.w, s0, b0);
+        w[4] = dequant_pair_order(q1.x, s1, b1);
+        w[5] = dequant_pair_order(q1.y, s1, b1);
+        w[6] = dequant_pair_order(q1.z, s1, b1);
+        w[7] = dequant_pair_order(q1.w, s1, b1);
         const int c0 = 4 * h, x = r & 7;
-        *reinterpret_cast<uint4*>(dd + (((c0 + 0) ^ x) << 4)) = w0;
-        *reinterpret_cast<uint4*>(dd + (((c0 + 1) ^ x) << 4)) = w1;
-        *reinterpret_cast<uint4*>(dd + (((c0 + 2) ^ x) << 4)) = w2;
-        *reinterpret_cast<uint4*>(dd + (((c0 + 3) ^ x) << 4)) = w3;
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        if (!(g == 0 && d == 0 && ti == a.drop_tile)) bar_arrive(a_full + as);
+#pragma unroll
+        for (int st = 0; st < 2; ++st) {
+          const int as = (g + st) % STAGES;
+          if (__any_sync(0xffffffffu, !bar_wait(st_empty + as, parity(g + st, STAGES) ^ 1u, a.timeout_ns))) {
+            fail = 1;  // the MMA may still read this stage
+            break;
+          }
+          uint8_t* dd = smA + as * A_STAGE + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(dd + (((c0 + j) ^ x) << 4)) = w[4 * st + j];
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0 && !(g + st == 0 && d == 0 && ti == a.drop_tile)) bar_arrive(a_full + as);
+        }
+        if (fail) break;
       }
       if (fail) break;
-      bar_arrive(sb_empty + tb);
+      __syncwarp();
+      if (lane == 0) bar_arrive(sb_empty + tb);
     }
   } else {
     // ---------------------------------------------------------------- epilogue (TMEM lane quadrant = warp % 4)
+    const int ew = warp - kWarpEpi0;  // 0..7
     const int quad = warp & 3;
-    const int L = quad * 32 + lane;  // TMEM lane = tile row
-    const int et = tid - (64 + kDq);  // 0..127 among the epilogue threads
+    const int chalf = ew >> 2;             // token columns [32 chalf, 32 chalf + 32)
+    const int L = quad * 32 + lane;        // TMEM lane = tile row
+    const int et = tid - 32 * kWarpEpi0;  // 0..255 among the epilogue threads
     const int r = a.lora_r;
+    float* lt = reinterpret_cast<float*>(sm + OFF_LT);   // [token][r] LoRA t vectors of the tile (two sets)
+    float* rsc = reinterpret_cast<float*>(sm + OFF_RS);  // [token] gating weights of the tile
     int it = 0;
 #pragma unroll 1
     for (int ti = blockIdx.x; ti < n_tiles && !fail; ti += gridDim.x, ++it) {
       const Tile tile = a.tiles[ti];
       const int ab = it & 1;
-      // the four epilogue warps leave together (they meet at named barriers below)
+      const int o = tile.mt * BM + L;
+      const int c0 = 32 * chalf;
+      // per-tile inputs of the epilogue, staged once while the accumulator is still being written
+      const bool swiglu = a.epi == EPI_SWIGLU;
+      const bool up = swiglu && (L & 1) != 0;
+      const uint16_t* Bsrc;
+      if (swiglu)
+        Bsrc = tile.e == a.E ? (up ? a.lora_B2 : a.lora_B1) : nullptr;  // LoRA on the shared expert's gate/up
+      else
+        Bsrc = tile.e < a.E ? (a.lora_Bex ? a.lora_Bex + static_cast<size_t>(tile.e) * a.out_ld * r : nullptr)
+                            : a.lora_B1;
+      const int brow = swiglu ? (o >> 1) : o;
+      const bool any_lora = swiglu ? tile.e == a.E && (a.lora_B1 || a.lora_B2)
+                                   : (tile.e < a.E ? a.lora_Bex != nullptr : a.lora_B1 != nullptr);
+      if (any_lora) {  // gate and up rows read different t arrays on SwiGLU tiles: even rows t1, odd rows t2
+        const int tn = tile.n * r;
+        for (int i = et; i < tn; i += kEpi) {
+          lt[i] = a.lora_t1[static_cast<size_t>(tile.row0) * r + i];
+          if (swiglu) lt[BN * 32 + i] = a.lora_t2 ? a.lora_t2[static_cast<size_t>(tile.row0) * r + i] : 0.f;
+        }
+      }
+      if (!swiglu && tile.e < a.E && a.row_scale)
+        for (int i = et; i < tile.n; i += kEpi) rsc[i] = a.row_scale[tile.row0 + i];
+      // the epilogue warps leave together (they meet at named barriers below)
       if (epi_any(!bar_wait(acc_full + ab, parity(it, 2), a.timeout_ns))) {
         fail = 1;
         break;
       }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t taddr = tmem + static_cast<uint32_t>(ab * BM) + ((static_cast<uint32_t>(quad) * 32u) << 16);
-      const int o = tile.mt * BM + L;
-      if (a.epi == EPI_SWIGLU) {
-        bool range_bad = false;  // a SwiGLU output fp16 cannot hold: MOE_ERR_RANGE
-        const bool up = (L & 1) != 0;
-        const int j = o >> 1;
-        const bool sh = tile.e == a.E;  // the shared expert's gate/up carry LoRA deltas
-        const uint16_t* Bsrc = sh ? (up ? a.lora_B2 : a.lora_B1) : nullptr;
-        const float* tsrc = up ? a.lora_t2 : a.lora_t1;
-        const int col = pair_pos(L >> 1);  // SwiGLU outputs in pair order (the down GEMM's token operand)
+      const uint32_t taddr =
+          tmem + static_cast<uint32_t>(ab * ACC_CHAINS * BN) + ((static_cast<uint32_t>(quad) * 32u) << 16);
+      const float* ltr = lt + (up ? BN * 32 : 0);
+      float v[32];
+      const bool live = c0 < tile.n;
+      if (live) {  // the sum of the accumulator chains
+        tmem_ld32(taddr + c0, v);
 #pragma unroll 1
-        for (int c0 = 0; c0 < tile.n; c0 += 32) {
-          float v[32];
-          tmem_ld32(taddr + c0, v);
-          if (Bsrc) {  // unmerged LoRA: + scale * B[j] . t[token]
-#pragma unroll 1
-            for (int i = 0; i < r; ++i) {
-              const float bj = half_bits_to_float(Bsrc[static_cast<size_t>(j) * r + i]);
+        for (int ch = 1; ch < ACC_CHAINS; ++ch) {
+          float w[32];
+          tmem_ld32(taddr + ch * BN + c0, w);
 #pragma unroll
-              for (int t = 0; t < 32; ++t) {
-                const int tt = c0 + t < tile.n ? c0 + t : tile.n - 1;
-                v[t] = fmaf(a.lora_scale * bj, tsrc[static_cast<size_t>(tile.row0 + tt) * r + i], v[t]);
-              }
-            }
+          for (int t = 0; t < 32; ++t) v[t] += w[t];
+        }
+      }
+      // the accumulator is read: release it for the tile after next
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) bar_arrive(acc_empty + ab);
+      if (live && Bsrc) {  // unmerged LoRA: + scale * B[row] . t[token]
+#pragma unroll 1
+        for (int i = 0; i < r; ++i) {
+          const float bi = a.lora_scale * half_bits_to_float(Bsrc[static_cast<size_t>(brow) * r + i]);
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            const int tt = c0 + t < tile.n ? c0 + t : tile.n - 1;
+            v[t] = fmaf(bi, ltr[tt * r + i], v[t]);
           }
+        }
+      }
+      if (swiglu) {
+        bool range_bad = false;  // a SwiGLU output fp16 cannot hold: MOE_ERR_RANGE
+        const int col = pair_pos(L >> 1);  // SwiGLU outputs in pair order (the down GEMM's token operand)
+        if (live) {
 #pragma unroll
           for (int t = 0; t < 32; ++t) {
             const float partner = __shfl_xor_sync(0xffffffffu, v[t], 1);
             if (!up && c0 + t < tile.n) {
-              const float hv = silu(v[t]) * partner;
+              const float hv = __fdividef(v[t], 1.0f + __expf(-v[t])) * partner;  // fp16 result: fast SiLU suffices
               range_bad |= !(fabsf(hv) <= kF16Max);
               stage[(c0 + t) * 64 + col] = __half_as_ushort(__float2half_rn(hv));
             }
           }
         }
-        // the accumulator is read: release it for the tile after next
-        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-        bar_arrive(acc_empty + ab);
         if (range_bad) report(a.err, 6);
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        asm volatile("bar.sync 1, 256;" ::: "memory");
         for (int i = et; i < tile.n * 8; i += kEpi) {
           const int t = i >> 3, ch = i & 7;
           *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(tile.row0 + t) * a.out_ld + tile.mt * 64 + ch * 8) =
               reinterpret_cast<const uint4*>(stage + t * 64)[ch];
         }
       } else {
-        const uint16_t* Bsrc = tile.e < a.E ? (a.lora_Bex ? a.lora_Bex + static_cast<size_t>(tile.e) * (a.out_ld) * r
-                                                          : nullptr)
-                                            : a.lora_B1;
-#pragma unroll 1
-        for (int c0 = 0; c0 < tile.n; c0 += 32) {
-          float v[32];
-          tmem_ld32(taddr + c0, v);
-          if (Bsrc) {
-#pragma unroll 1
-            for (int i = 0; i < r; ++i) {
-              const float bo = half_bits_to_float(Bsrc[static_cast<size_t>(o) * r + i]);
-#pragma unroll
-              for (int t = 0; t < 32; ++t) {
-                const int tt = c0 + t < tile.n ? c0 + t : tile.n - 1;
-                v[t] = fmaf(a.lora_scale * bo, a.lora_t1[static_cast<size_t>(tile.row0 + tt) * r + i], v[t]);
-              }
-            }
-          }
+        const bool scaled = tile.e < a.E && a.row_scale;
+        if (live) {
 #pragma unroll
           for (int t = 0; t < 32; ++t) {
             if (c0 + t < tile.n) {
-              float xv = v[t];
-              if (tile.e < a.E && a.row_scale) xv *= a.row_scale[tile.row0 + c0 + t];
+              const float xv = scaled ? v[t] * rsc[c0 + t] : v[t];
               stage[(c0 + t) * 128 + L] = __half_as_ushort(__float2half_rn(xv));
             }
           }
         }
-        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-        bar_arrive(acc_empty + ab);
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        asm volatile("bar.sync 1, 256;" ::: "memory");
         for (int i = et; i < tile.n * 16; i += kEpi) {
           const int t = i >> 4, ch = i & 15;
           *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(tile.row0 + t) * a.out_ld + tile.mt * BM + ch * 8) =
               reinterpret_cast<const uint4*>(stage + t * 128)[ch];
         }
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");  // the staging buffer is free for the next tile
+      asm volatile("bar.sync 1, 256;" ::: "memory");  // staging buffers are free for the next tile
     }
   }
   if (fail) report(a.err, 5);

@@ -240,7 +240,7 @@ struct GWs {
   int32_t *idx, *count, *offset, *perm, *inv, *blockhist;
   float *w_pos, *t1, *t2, *g;
   uint16_t *X, *Hh, *Y;
-  gg::Tile *tiles_gu, *tiles_dn;
+  tc::Tile *tiles_gu, *tiles_dn;
   int* n_tiles;
   int* err;
   int max_gu, max_dn, nblk;
@@ -258,9 +258,9 @@ GWs carve_gemm(void* base, int T, int K, int E, int H, int I, int r) {
   const size_t TK = static_cast<size_t>(T) * K, R = TK + T;
   const int rr = r > 0 ? r : 1;
   w.nblk = static_cast<int>((TK + pf::kChunk - 1) / pf::kChunk);
-  const int nt_max = static_cast<int>((TK + static_cast<size_t>(E) * (gg::BN - 1)) / gg::BN) + (T + gg::BN - 1) / gg::BN + 1;
-  w.max_gu = nt_max * (2 * I / gg::BM);
-  w.max_dn = nt_max * (H / gg::BM);
+  const int nt_max = static_cast<int>((TK + static_cast<size_t>(E) * (gg3::BN - 1)) / gg3::BN) + (T + gg3::BN - 1) / gg3::BN + 1;
+  w.max_gu = nt_max * (2 * I / gg3::BM);
+  w.max_dn = nt_max * (H / gg3::BM);
   w.idx = reinterpret_cast<int32_t*>(take(TK * 4));
   w.count = reinterpret_cast<int32_t*>(take(static_cast<size_t>(E) * 4));
   w.offset = reinterpret_cast<int32_t*>(take(static_cast<size_t>(E + 1) * 4));
@@ -274,8 +274,8 @@ GWs carve_gemm(void* base, int T, int K, int E, int H, int I, int r) {
   w.X = reinterpret_cast<uint16_t*>(take(R * H * 2));
   w.Hh = reinterpret_cast<uint16_t*>(take(R * I * 2));
   w.Y = reinterpret_cast<uint16_t*>(take(R * H * 2));
-  w.tiles_gu = reinterpret_cast<gg::Tile*>(take(static_cast<size_t>(w.max_gu) * sizeof(gg::Tile)));
-  w.tiles_dn = reinterpret_cast<gg::Tile*>(take(static_cast<size_t>(w.max_dn) * sizeof(gg::Tile)));
+  w.tiles_gu = reinterpret_cast<tc::Tile*>(take(static_cast<size_t>(w.max_gu) * sizeof(tc::Tile)));
+  w.tiles_dn = reinterpret_cast<tc::Tile*>(take(static_cast<size_t>(w.max_dn) * sizeof(tc::Tile)));
   w.n_tiles = reinterpret_cast<int*>(take(2 * 4));
   w.err = reinterpret_cast<int*>(take(4));
   w.bytes = off;
@@ -283,8 +283,8 @@ GWs carve_gemm(void* base, int T, int K, int E, int H, int I, int r) {
 }
 
 bool gemm_path(const moe_layer* L, int T, int K) {
-  return static_cast<long long>(T) * K >= kGemmMinSlots && L->H % gg::BM == 0 && (2 * L->I) % gg::BM == 0 &&
-         L->I % gg::BK == 0;
+  return static_cast<long long>(T) * K >= kGemmMinSlots && L->H % gg3::BM == 0 && (2 * L->I) % gg3::BM == 0 &&
+         L->I % (2 * gg3::BK) == 0;  // the dequantising warps take two K steps per pass
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -317,8 +317,9 @@ bool token_map(CUtensorMap* m, const uint16_t* X, int cols, int rows) {
 }
 
 // The row records of one weight matrix in n_exp expert blocks (expert_stride bytes apart) as a 3-D byte map
-// {record bytes, rows, experts}, boxes of box_x bytes x 128 rows x 1 expert, no swizzle.
-bool weight_map(CUtensorMap* m, const uint8_t* base, int rec, int rows, int n_exp, int64_t expert_stride, int box_x) {
+// {record bytes, rows, experts}, boxes of box_x bytes x 128 rows x 1 expert (128-byte swizzle if asked).
+bool weight_map(CUtensorMap* m, const uint8_t* base, int rec, int rows, int n_exp, int64_t expert_stride, int box_x,
+                bool swizzle = false) {
   const EncodeTiledFn f = encode_tiled();
   if (!f) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(rec), static_cast<cuuint64_t>(rows),
@@ -327,8 +328,8 @@ bool weight_map(CUtensorMap* m, const uint8_t* base, int rec, int rows, int n_ex
   const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_x), static_cast<cuuint32_t>(gg3::BM), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims, strides, box, estr,
-           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+           CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // The tensor maps of one grouped GEMM over the matrix at byte a_off of every expert block (records of rec
@@ -339,9 +340,9 @@ bool gemm_maps(gg3::Maps* m, const moe_layer* L, int64_t a_off, int rec, int row
   const uint8_t* sh = static_cast<const uint8_t*>(L->shared_block) + a_off;
   const int sb = gg3::sb_row_bytes(K);
   const int64_t sh_stride = static_cast<int64_t>(rec) * rows;
-  return weight_map(&m->pool_codes, pool, rec, rows, L->E, L->expert_stride, 32) &&
+  return weight_map(&m->pool_codes, pool, rec, rows, L->E, L->expert_stride, 32 * gg3::RGROUPS, true) &&
          weight_map(&m->pool_sb, pool, rec, rows, L->E, L->expert_stride, sb) &&
-         weight_map(&m->shared_codes, sh, rec, rows, 1, sh_stride, 32) &&
+         weight_map(&m->shared_codes, sh, rec, rows, 1, sh_stride, 32 * gg3::RGROUPS, true) &&
          weight_map(&m->shared_sb, sh, rec, rows, 1, sh_stride, sb) &&
          token_map(&m->tokens, tokens, K, n_token_rows);
 }
@@ -361,8 +362,8 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
   pf::bucket_scan_kernel<<<1, 256, 0, st>>>(ws.nblk, E, ws.blockhist, ws.count, ws.offset);
   pf::bucket_place_kernel<<<ws.nblk, pf::kChunk, 0, st>>>(ws.idx, TK, E, ws.blockhist, ws.perm, ws.inv, perm_out);
   pf::permute_kernel<<<R, 256, 0, st>>>(u, T, K, H, ws.perm, w, ws.X, ws.w_pos, err_dev);
-  pf::tile_list_kernel<<<1, 288, 0, st>>>(ws.count, ws.offset, E, T, K, 2 * I / gg::BM, H / gg::BM, ws.tiles_gu,
-                                          ws.tiles_dn, ws.n_tiles);
+  pf::tile_list_kernel<<<E + 1, 128, 0, st>>>(ws.count, ws.offset, E, T, K, 2 * I / gg3::BM, H / gg3::BM, ws.tiles_gu,
+                                              ws.tiles_dn, ws.n_tiles);
   // The GEMMs trust the device-built tile list: stop here if any launch so far failed.
   if (launch_status() != MOE_OK) return MOE_ERR_CUDA;
   {
@@ -388,9 +389,10 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
     a.err = err_dev;
     a.timeout_ns = timeout_ns;
     a.drop_tile = -1;
+    a.nsb = 2;
     return a;
   };
-  const int smem_gu = gg3::smem_bytes(H), smem_dn = gg3::smem_bytes(I);
+  const int smem_gu = gg3::smem_bytes(H, gg3::sb_buffers(H)), smem_dn = gg3::smem_bytes(I, gg3::sb_buffers(I));
   if (cudaFuncSetAttribute(gg3::grouped_gemm3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smem_gu > smem_dn ? smem_gu : smem_dn) != cudaSuccess)
     return MOE_ERR_CUDA;
@@ -403,7 +405,8 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
     gg3::Args a = base_args();
     a.tiles = ws.tiles_gu;
     a.K = H;
-    a.epi = gg::EPI_SWIGLU;
+    a.nsb = gg3::sb_buffers(H);
+    a.epi = tc::EPI_SWIGLU;
     a.drop_tile = drop_tile;
     a.out = ws.Hh;
     a.out_ld = I;
@@ -427,7 +430,8 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
     a.tiles = ws.tiles_dn;
     a.n_tiles = ws.n_tiles + 1;
     a.K = I;
-    a.epi = gg::EPI_DOWN;
+    a.nsb = gg3::sb_buffers(I);
+    a.epi = tc::EPI_DOWN;
     a.out = ws.Y;
     a.out_ld = H;
     a.row_scale = ws.w_pos;

@@ -37,6 +37,7 @@ __global__ void __launch_bounds__(256) bucket_scan_kernel(int nblk, int E, int32
   const int e = threadIdx.x;
   if (e < E) {
     int t = 0;
+#pragma unroll 8
     for (int b = 0; b < nblk; ++b) t += blockhist[static_cast<size_t>(b) * E + e];
     tot[e] = t;
   }
@@ -129,34 +130,33 @@ __global__ void __launch_bounds__(256) permute_kernel(const uint16_t* __restrict
 
 // Tile lists of both GEMMs: per expert (then the shared expert) its token
 // n-tiles, m-tiles innermost, so CTAs that share a token tile run together.
-__global__ void __launch_bounds__(288) tile_list_kernel(const int32_t* __restrict__ count,
+// One block per expert (block E: the shared expert): the block sums the n-tile
+// counts of the experts before it, then writes its tiles with all threads.
+__global__ void __launch_bounds__(128) tile_list_kernel(const int32_t* __restrict__ count,
                                                         const int32_t* __restrict__ offset, int E, int T, int K,
-                                                        int mt_gu, int mt_dn, gg::Tile* __restrict__ tiles_gu,
-                                                        gg::Tile* __restrict__ tiles_dn, int* __restrict__ n_tiles) {
-  __shared__ int nt[257];
-  __shared__ int start[258];
-  const int e = threadIdx.x;  // 0..E (E = shared)
-  if (e <= E) nt[e] = e < E ? (count[e] + gg::BN - 1) / gg::BN : (T + gg::BN - 1) / gg::BN;
+                                                        int mt_gu, int mt_dn, tc::Tile* __restrict__ tiles_gu,
+                                                        tc::Tile* __restrict__ tiles_dn, int* __restrict__ n_tiles) {
+  constexpr int BN = gg3::BN;
+  __shared__ int red[4];
+  const int e = blockIdx.x;  // 0..E
+  int before = 0;
+  for (int i = threadIdx.x; i < e; i += blockDim.x) before += (count[i] + BN - 1) / BN;
+  before = __reduce_add_sync(0xffffffffu, before);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = before;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int run = 0;
-    for (int i = 0; i <= E; ++i) {
-      start[i] = run;
-      run += nt[i];
-    }
-    start[E + 1] = run;
-    n_tiles[0] = run * mt_gu;
-    n_tiles[1] = run * mt_dn;
+  const int start = red[0] + red[1] + red[2] + red[3];
+  const int n = e < E ? count[e] : T;
+  const int nt = (n + BN - 1) / BN;
+  const int base = e < E ? offset[e] : T * K;
+  if (e == E && threadIdx.x == 0) {
+    n_tiles[0] = (start + nt) * mt_gu;
+    n_tiles[1] = (start + nt) * mt_dn;
   }
-  __syncthreads();
-  if (e <= E) {
-    const int base = e < E ? offset[e] : T * K;
-    const int n = e < E ? count[e] : T;
-    for (int q = 0; q < nt[e]; ++q) {
-      const int n0 = q * gg::BN, nn = min(gg::BN, n - n0), t = start[e] + q;
-      for (int m = 0; m < mt_gu; ++m) tiles_gu[t * mt_gu + m] = gg::Tile{e, m, base + n0, nn};
-      for (int m = 0; m < mt_dn; ++m) tiles_dn[t * mt_dn + m] = gg::Tile{e, m, base + n0, nn};
-    }
+  const int mt = mt_gu > mt_dn ? mt_gu : mt_dn;
+  for (int i = threadIdx.x; i < nt * mt; i += blockDim.x) {
+    const int q = i / mt, m = i % mt, n0 = q * BN, nn = min(BN, n - n0), t = start + q;
+    if (m < mt_dn) tiles_dn[t * mt_dn + m] = tc::Tile{e, m, base + n0, nn};
+    if (m < mt_gu) tiles_gu[t * mt_gu + m] = tc::Tile{e, m, base + n0, nn};
   }
 }
 
