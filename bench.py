@@ -629,6 +629,44 @@ def diag_expert(args):
           f"({expert_flops(cfg, T) / (ms / 1000.0) / 1e12:.1f} TFLOP/s)")
 
 
+def diag_route(args):
+    """Diagnostic run of one layer's router + top-K and Prerouter (no JSON line): layer 1 of --cfg (default: the
+    35B-shaped prefill) on --tokens tokens, --runs calls of each; for profilers."""
+    import torch
+    import int4_expert_ffn_top_b200 as M
+    cfg = CONFIGS[args.cfg if args.cfg != CFG_ID else PREFILL_CFG_ID]
+    T, K = args.tokens, cfg.K
+    host = inputs.layer(cfg, 1, experts=[])
+    lay = M.DeviceLayer(cfg, host)
+    head = M.DeviceHead(cfg, host["prerouter"])
+    u = torch.from_numpy(inputs.activations(cfg, step=9, T=T).view(np.int16)).cuda()
+    logits = torch.empty((T, cfg.E), device="cuda")
+    idx = torch.empty((T, K), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, K), device="cuda")
+    pred = torch.empty((T, K), dtype=torch.int32, device="cuda")
+    scores = torch.empty((T, cfg.E), device="cuda")
+    pws = M.workspace(M.prerouter_workspace_size(head, T))
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    M.moe_route_topk(lay, u, K, logits, idx, w, err_word=err)
+    M.prerouter_predict(head, u, idx, K, pred, scores, pws, err_word=err)
+    e0.record()
+    for _ in range(args.runs):
+        M.moe_route_topk(lay, u, K, logits, idx, w, err_word=err)
+    e1.record()
+    for _ in range(args.runs):
+        M.prerouter_predict(head, u, idx, K, pred, scores, pws, err_word=err)
+    e2.record()
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise SystemExit(f"status {int(err.item())}")
+    ms_r, ms_p = e0.elapsed_time(e1) / args.runs, e1.elapsed_time(e2) / args.runs
+    fr = 2.0 * T * cfg.H * cfg.E
+    fp = 2.0 * T * ((cfg.H + cfg.E) * cfg.P + cfg.P * cfg.E_next)
+    print(f"{cfg.name}, {T} tokens: router + top-K {ms_r * 1e3:.1f} us ({fr / (ms_r / 1e3) / 1e12:.1f} TFLOP/s), "
+          f"Prerouter {ms_p * 1e3:.1f} us ({fp / (ms_p / 1e3) / 1e12:.1f} TFLOP/s)")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -647,13 +685,17 @@ def main():
     ap.add_argument("--trace", action="store_true", help="--diag-stack: print per-phase times")
     ap.add_argument("--diag-expert", action="store_true",
                     help="diagnostic run of one layer's expert forward (for profilers); prints no JSON line")
-    ap.add_argument("--tokens", type=int, default=3328, help="--diag-expert: tokens per call")
+    ap.add_argument("--diag-route", action="store_true",
+                    help="diagnostic run of one layer's router + top-K and Prerouter; prints no JSON line")
+    ap.add_argument("--tokens", type=int, default=3328, help="--diag-expert / --diag-route: tokens per call")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.diag_stack:
         return diag_stack(args)
     if args.diag_expert:
         return diag_expert(args)
+    if args.diag_route:
+        return diag_route(args)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -154,6 +154,13 @@ moe_status moe_rmsnorm_bf16(const float* x, int32_t T, int32_t H, float eps, uin
  *   w[t][k]  = exp(l_k - l_0) / sum_j exp(l_j - l_0) over the K selected
  * u [T][H] bf16; logits [T][E] fp32 (required output); idx [T][K] int32;
  * w [T][K] fp32.  Two launches.
+ * Paths (chosen by shape and alignment only): from 256 tokens on, with E a
+ *   multiple of 128 and u 16-byte aligned, the logits come from a tcgen05
+ *   GEMM with bf16 operands: per 64-input group the exact products of the
+ *   codes minus 128 with u accumulate in fp32 in tensor memory, and each group
+ *   is folded in as s*D + (b + 128 s)*sum(u) in fp32 (no weight is rounded;
+ *   any finite bf16 u is taken).  Otherwise a dequant-fused GEMV on the CUDA
+ *   cores multiplies u rounded to fp16 (see MOE_ERR_RANGE).
  */
 moe_status moe_route_topk(const moe_layer* L, const uint16_t* u, int32_t T, int32_t K,
                           float* logits, int32_t* idx, float* w, int32_t* err_word, void* stream);
@@ -199,6 +206,11 @@ size_t moe_workspace_size(const moe_layer* L, int32_t T, int32_t K);
  * outside [0,E) is clamped to 0 or E-1); pred [T][K_next] int32 (same ordering and
  * tie rule as moe_route_topk); scores [T][E_next] fp32 (required output, the
  * p vector); workspace >= prerouter_workspace_size(head, T) bytes.
+ * Paths (chosen by shape and alignment only): from 256 tokens on, with P a
+ *   multiple of 128, E of 64 and u 16-byte aligned, the first layer is a
+ *   tcgen05 GEMM over [u ; multi_hot(sel)] with W1 split exactly into two bf16
+ *   parts (fp32 accumulation, no input rounded); otherwise a GEMV on the CUDA
+ *   cores with u rounded to fp16.  The second layer is a CUDA-core GEMV.
  */
 moe_status prerouter_predict(const moe_prerouter* head, const uint16_t* u, const int32_t* sel,
                              int32_t T, int32_t K, int32_t K_next, int32_t* pred, float* scores,

@@ -13,7 +13,7 @@
 //    each row (a box of a second map over the same bytes, 128-byte swizzle,
 //    16 KB, three stages); per step the step's token rows (2-D map, 128-byte
 //    swizzle, boxes of 32 rows, only as many as the tile has tokens);
-//  * warps 2..9 dequantise, two K steps per pass: thread (row r, half h) reads
+//  * 8 warps dequantise, two K steps per pass: thread (row r, half h) reads
 //    16 code bytes per step (lanes of a warp take 8 consecutive rows per
 //    128-byte wavefront, conflict-free under the swizzle), forms w = q*s + b in
 //    fp16 (one rounding) and stores four 16-byte chunks into the
@@ -21,12 +21,12 @@
 //    "pair order" (q_j, q_{j+4}), the order the magic-exponent unpacking
 //    produces; the token operand is stored in the same order, so the products
 //    are those of the plain order;
-//  * warp 1, one lane (MMA): tcgen05.mma kind::f16 into one of two sets of four
-//    64-column TMEM accumulators (tiles alternate); K slice c (16 wide) of
-//    every step goes to accumulator c, so four independent accumulation chains
-//    keep the tensor core busy at ~64 tokens per MMA; each commit releases the
-//    step's operand stages and, after a tile, its accumulators;
-//  * warps 10..17 (epilogue, TMEM lane quadrant = warp % 4, two warps per
+//  * warps 1 and 2, one lane each (MMA): tcgen05.mma kind::f16 into one of two sets of
+//    four 64-column TMEM accumulators (tiles alternate); K slice c (16 wide) of every step goes to
+//    accumulator c, issued by MMA warp c % 2 -- four independent accumulation chains, and two issuing
+//    threads, since one thread issues an MMA only every ~175 cycles; each commit releases the step's
+//    operand stages and, after a tile, its accumulators;
+//  * 8 epilogue warps (TMEM lane quadrant = warp % 4, two warps per
 //    quadrant splitting the token columns): drain and add the finished
 //    accumulators with tcgen05.ld while the next tile's main loop runs: SwiGLU of
 //    interleaved gate/up rows (output in pair order, the next GEMM's token
@@ -75,7 +75,8 @@ constexpr int kDqWarps = 8;
 constexpr int kDq = 32 * kDqWarps;
 constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant, splitting the tile's token columns
 constexpr int kEpi = 32 * kEpiWarps;
-constexpr int kMmaWarps = 1;  // MMA-issuing warps; warp 1 + w issues the chains w, w + kMmaWarps, ...
+constexpr int kMmaWarps = 2;  // MMA-issuing warps (one thread issues an MMA only every ~175 cycles); warp 1 + w
+                              // issues the chains w, w + kMmaWarps, ...
 constexpr int kThreads = 32 * (1 + kMmaWarps) + kDq + kEpi;  // TMA warp, MMA warps, dequant warps, epilogue warps
 constexpr int kWarpDq0 = 1 + kMmaWarps;                         // first dequantising warp
 constexpr int kWarpEpi0 = kWarpDq0 + kDqWarps;                  // first epilogue warp

@@ -7,6 +7,7 @@
 #include <mutex>
 
 #include "../../include/moe.h"
+#include "dense_gemm.cuh"
 #include "layer_kernels.cuh"
 #include "prefill_kernels.cuh"
 #include "stack_kernel.cuh"
@@ -122,9 +123,24 @@ void allow_smem(KernelT k, size_t bytes) {
   if (bytes > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
 }
 
+// Many-token batches of the router and the Prerouter's first layer run on the tensor cores (dense::dense_kernel)
+// from this many tokens on; fewer take the CUDA-core GEMVs.
+constexpr int kDenseMinTokens = 256;
+bool dense_router_ok(const moe_layer* L, const uint16_t* u, int T);
+moe_status dense_router(const moe_layer* L, const uint16_t* u, int T, float* logits, int* err, cudaStream_t st);
+bool dense_w1_ok(const moe_prerouter* P, const uint16_t* u, int T);
+moe_status dense_w1(const moe_prerouter* P, const uint16_t* u, const int32_t* sel, int T, int K, float* z, int* err,
+                    cudaStream_t st);
+
 template <int H>
 moe_status route_h(const moe_layer* L, const uint16_t* u, int T, int K, float* logits, int32_t* idx, float* w,
                    int* err, cudaStream_t st) {
+  if (dense_router_ok(L, u, T)) {
+    const moe_status s = dense_router(L, u, T, logits, err, st);
+    if (s != MOE_OK) return s;
+    topk_kernel<<<(T + kWarps - 1) / kWarps, kThreads, 0, st>>>(logits, T, L->E, K, idx, w);
+    return launch_status();
+  }
   constexpr int NCH = H / 16;
   constexpr int SEG = NCH < 32 ? NCH : 32;
   const int rows_per_cta = kWarps * (32 / SEG);
@@ -347,6 +363,102 @@ bool gemm_maps(gg3::Maps* m, const moe_layer* L, int64_t a_off, int rec, int row
          token_map(&m->tokens, tokens, K, n_token_rows);
 }
 
+// Row-major bf16 activations u [T][H] as a TMA source of [64 rows x 64 cols] boxes, 128-byte swizzle.
+bool u_map(CUtensorMap* m, const uint16_t* u, int H, int T) {
+  const EncodeTiledFn f = encode_tiled();
+  if (!f) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(H) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(dense::BK), static_cast<cuuint32_t>(dense::BN)};
+  const cuuint32_t estr[2] = {1, 1};
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(u), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A row-major matrix of `rows` rows, `cols` elements of elem_bytes each per row, row_bytes apart, as a TMA source
+// of [128 rows x 128 bytes] boxes, 128-byte swizzle.
+bool rows_map(CUtensorMap* m, const void* base, CUtensorMapDataType type, int elem_bytes, int cols, int rows,
+              int64_t row_bytes) {
+  const EncodeTiledFn f = encode_tiled();
+  if (!f) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(dense::BM)};
+  const cuuint32_t estr[2] = {1, 1};
+  return f(m, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE>
+moe_status launch_dense(const dense::Maps& m, dense::Args a, cudaStream_t st) {
+  using C = dense::Cfg<MODE>;
+  a.n_tiles = a.m_tiles * ((a.T + dense::BN - 1) / dense::BN);
+  a.timeout_ns = kGemmTimeoutNs;
+  int dev = 0, nsm = 0;
+  if (cudaFuncSetAttribute(dense::dense_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+          cudaSuccess ||
+      cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int grid = a.n_tiles < nsm ? a.n_tiles : nsm;
+  dense::dense_kernel<MODE><<<grid, C::kThreads, C::SMEM_BYTES, st>>>(m, a);
+  return launch_status();
+}
+
+bool dense_router_ok(const moe_layer* L, const uint16_t* u, int T) {
+  return T >= kDenseMinTokens && L->E % dense::BM == 0 && L->router.bits == 8 && aligned(u, 16);
+}
+
+// logits [T][E] of the 8-bit router on the tensor cores.
+moe_status dense_router(const moe_layer* L, const uint16_t* u, int T, float* logits, int* err, cudaStream_t st) {
+  const int H = L->H, rec = qrow_bytes(H, 8);
+  dense::Maps m;
+  if (!u_map(&m.u, u, H, T) ||
+      !rows_map(&m.a, L->router.rows, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, H, L->E, rec))
+    return MOE_ERR_CUDA;
+  dense::Args a{};
+  a.T = T;
+  a.H = H;
+  a.KT = a.KTu = H / dense::BK;
+  a.M = L->E;
+  a.m_tiles = L->E / dense::BM;
+  a.rows = static_cast<const uint8_t*>(L->router.rows);
+  a.rec = rec;
+  a.beta = L->router_bias;
+  a.logits = logits;
+  a.err = err;
+  return launch_dense<dense::MODE_ROUTER>(m, a, st);
+}
+
+bool dense_w1_ok(const moe_prerouter* P, const uint16_t* u, int T) {
+  return T >= kDenseMinTokens && P->P % dense::BM == 0 && P->E % dense::BK == 0 && aligned(u, 16);
+}
+
+// z [T][P] = silu(W1 [u ; multi_hot(sel)] + b1) on the tensor cores.
+moe_status dense_w1(const moe_prerouter* P, const uint16_t* u, const int32_t* sel, int T, int K, float* z, int* err,
+                    cudaStream_t st) {
+  const int H = P->H, W = P->H + P->E;
+  dense::Maps m;
+  if (!u_map(&m.u, u, H, T) ||
+      !rows_map(&m.a, P->W1, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, W, P->P, static_cast<int64_t>(W) * 2))
+    return MOE_ERR_CUDA;
+  dense::Args a{};
+  a.T = T;
+  a.H = H;
+  a.KT = W / dense::BK;
+  a.KTu = H / dense::BK;
+  a.M = P->P;
+  a.m_tiles = P->P / dense::BM;
+  a.sel = sel;
+  a.K = K;
+  a.E = P->E;
+  a.b1 = P->b1;
+  a.z = z;
+  a.err = err;
+  return launch_dense<dense::MODE_W1>(m, a, st);
+}
+
 template <int H>
 // Bounded waits give up after timeout_ns; drop_tile >= 0 arms the gate/up GEMM's test hook (gg3::Args).
 moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int K, const int32_t* idx, const float* w,
@@ -463,21 +575,26 @@ moe_status expert_forward_h(const moe_layer* L, const uint16_t* u, int T, int K,
 template <int H>
 moe_status prerouter_h(const moe_prerouter* P, const uint16_t* u, const int32_t* sel, int T, int K, int K_next,
                        int32_t* pred, float* scores, float* z, int* err, cudaStream_t st) {
-  PreW1Args a{};
-  a.u = u;
-  a.T = T;
-  a.K = K;
-  a.E = P->E;
-  a.P = P->P;
-  a.sel = sel;
-  a.W1 = P->W1;
-  a.b1 = P->b1;
-  a.z = z;
-  a.err = err;
-  const size_t smem = gemv_smem(H, false, false);
-  allow_smem(prerouter_w1_kernel<H / 8>, smem);
-  dim3 g1((P->P + kWarps - 1) / kWarps, (T + TB - 1) / TB);
-  prerouter_w1_kernel<H / 8><<<g1, kThreads, smem, st>>>(a);
+  if (dense_w1_ok(P, u, T)) {
+    const moe_status s = dense_w1(P, u, sel, T, K, z, err, st);
+    if (s != MOE_OK) return s;
+  } else {
+    PreW1Args a{};
+    a.u = u;
+    a.T = T;
+    a.K = K;
+    a.E = P->E;
+    a.P = P->P;
+    a.sel = sel;
+    a.W1 = P->W1;
+    a.b1 = P->b1;
+    a.z = z;
+    a.err = err;
+    const size_t smem = gemv_smem(H, false, false);
+    allow_smem(prerouter_w1_kernel<H / 8>, smem);
+    dim3 g1((P->P + kWarps - 1) / kWarps, (T + TB - 1) / TB);
+    prerouter_w1_kernel<H / 8><<<g1, kThreads, smem, st>>>(a);
+  }
   dim3 g2((P->E_next + kW2Rows - 1) / kW2Rows, (T + kW2Tok - 1) / kW2Tok);
   prerouter_w2_kernel<<<g2, kThreads, 0, st>>>(z, T, P->P, P->W2, P->b2, P->E_next, scores);
   topk_kernel<<<(T + kWarps - 1) / kWarps, kThreads, 0, st>>>(scores, T, P->E_next, K_next, pred, nullptr);

@@ -63,6 +63,53 @@ def router_tau(u: np.ndarray, router: dict, n_round: int = 64) -> np.ndarray:
             + fp16_input_error(u) @ (np.abs(q - mid) * s).T)
 
 
+def tc_chain_rounds(blocks: int) -> int:
+    """fp32 rounding units charged to a chain of ``blocks`` tensor-core MMA blocks.
+
+    One tcgen05 kind::f16 block adds 16 exact products to the fp32 accumulator.
+    The bound assumes nothing finer than this: every one of the 17 addends is
+    aligned to the largest and truncated to within one unit in the last place
+    (2 EPS32 of the largest magnitude, hence of the sum of magnitudes).
+    """
+    return 34 * blocks
+
+
+def router_tau_tc(u: np.ndarray, router: dict) -> np.ndarray:
+    """Bound [T, E] on |GPU logit - exact logit| for the tensor-core router (many-token path).
+
+    Per group: the four 16-wide MMA blocks of sum_k (q-128) u (exact products),
+    the group sum of u (16-term sums, two pairwise adds) and b + 128 s (one
+    rounding); then two fused multiply-adds per group into the fp32 logit and
+    the bias add.  u enters unrounded (bf16 operands).
+    """
+    G = u.shape[1] // 64
+    beta = np.abs(np.asarray(router["beta"], np.float64))
+    n = tc_chain_rounds(4) + 2 * G + 4
+    return n * EPS32 * (np.abs(u) @ qmat_abs_terms(router).T) + 4 * EPS32 * beta
+
+
+def prerouter_tau(u, sel, head, E, n_round=128, tc=False):
+    """Bound [T, E_next] on |fp32 GPU scores - exact| (first order through SiLU, |silu'| <= 1.1).
+
+    ``tc``: the first layer ran on the tensor cores: W1 split exactly into two
+    bf16 parts, u unrounded, four accumulation chains of 2 (H + E) / 64 MMA
+    blocks each, then three chain adds and the bias add.  Otherwise the GEMV:
+    ``n_round`` roundings per product term and u rounded to fp16.
+    """
+    W1 = np.abs(head["W1"].astype(np.float64))
+    W2 = np.abs(head["W2"].astype(np.float64))
+    xin = np.concatenate([np.abs(u), O.multi_hot(sel, E)], axis=1)
+    if tc:
+        n1 = tc_chain_rounds(2 * (u.shape[1] + E) // 64) + 8
+        a_err = n1 * EPS32 * (xin @ W1.T + np.abs(head["b1"].astype(np.float64)))
+    else:
+        a_err = n_round * EPS32 * (xin @ W1.T + np.abs(head["b1"].astype(np.float64)))
+        a_err = a_err + fp16_input_error(u) @ W1[:, :u.shape[1]].T  # u enters W1 rounded to fp16
+    z = np.abs(O.silu(np.concatenate([u, O.multi_hot(sel, E)], 1) @ head["W1"].astype(np.float64).T
+                      + head["b1"].astype(np.float64)))
+    return (1.1 * a_err + 8 * EPS32 * z) @ W2.T + n_round * EPS32 * (z @ W2.T + np.abs(head["b2"].astype(np.float64)))
+
+
 def check_topk(gpu_idx, ref, tau_row, K: int, exact_order: bool = True) -> int:
     """Check GPU top-K indices against float64 scores ``ref`` [T, E]; returns #certified near-tie rows."""
     gpu_idx = np.asarray(gpu_idx)

@@ -12,7 +12,8 @@ import torch
 
 from gen import CONFIGS, inputs
 from oracle import moe_oracle as O
-from parity import EPS32, assert_close_inf, check_bf16_rounding, check_topk, fp16_input_error, router_tau
+from parity import (EPS32, assert_close_inf, check_bf16_rounding, check_topk, prerouter_tau, router_tau,
+                    router_tau_tc)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -86,18 +87,6 @@ def prerouter(layer: Layer, u_bits, sel, K_next):
                         scores, ws)
     torch.cuda.synchronize()
     return pred.cpu().numpy(), scores.cpu().numpy().astype(np.float64)
-
-
-def prerouter_tau(u, sel, head, E, n_round=128):
-    """Bound [T, E_next] on |fp32 GPU scores - exact| (first order through SiLU, |silu'| <= 1.1)."""
-    W1 = np.abs(head["W1"].astype(np.float64))
-    W2 = np.abs(head["W2"].astype(np.float64))
-    xin = np.concatenate([np.abs(u), O.multi_hot(sel, E)], axis=1)
-    a_err = n_round * EPS32 * (xin @ W1.T + np.abs(head["b1"].astype(np.float64)))
-    a_err = a_err + fp16_input_error(u) @ W1[:, :u.shape[1]].T  # u enters W1 rounded to fp16
-    z = np.abs(O.silu(np.concatenate([u, O.multi_hot(sel, E)], 1) @ head["W1"].astype(np.float64).T
-                      + head["b1"].astype(np.float64)))
-    return (1.1 * a_err + 8 * EPS32 * z) @ W2.T + n_round * EPS32 * (z @ W2.T + np.abs(head["b2"].astype(np.float64)))
 
 
 @pytest.fixture(scope="module")
@@ -266,8 +255,9 @@ def test_full_size_layer(cuda_ok, cfg_id, l, T):
 
 
 # ----------------------------------------------------------------------------- stacks
-def _check_stack(cfg, stack_layers, T, res, x0, sample):
-    """Teacher-forced per-layer parity on the sampled layers of a stack run."""
+def _check_stack(cfg, stack_layers, T, res, x0, sample, tc=False):
+    """Teacher-forced per-layer parity on the sampled layers of a stack run (``tc``: the run's router and
+    Prerouter first layer took the tensor-core many-token path)."""
     xs = res["x_trace"]
     for l in sample:
         L = stack_layers(l)
@@ -276,7 +266,7 @@ def _check_stack(cfg, stack_layers, T, res, x0, sample):
         if l == 0:
             check_bf16_rounding(ub, O.rmsnorm(x0.astype(np.float64), 1e-6), rel_err=(cfg.H / 256 + 24) * EPS32)
         ref_logits = O.router_logits(u, L["router"])
-        tau = router_tau(u, L["router"])
+        tau = router_tau_tc(u, L["router"]) if tc else router_tau(u, L["router"])
         check_topk(res["true_idx"][l], ref_logits, tau, cfg.K)
         executed = res["idx"][l]
         if cfg.predicted_routing and l > 0:
@@ -289,7 +279,7 @@ def _check_stack(cfg, stack_layers, T, res, x0, sample):
         x_next = xs[l + 1] if l + 1 < len(xs) else res["x"]
         assert_close_inf(x_next.astype(np.float64) - xs[l].astype(np.float64), ref_out, what=f"layer {l} output")
         ref_p = O.prerouter_scores(u, executed, L["prerouter"], cfg.E)
-        check_topk(res["pred"][l], ref_p, prerouter_tau(u, executed, L["prerouter"], cfg.E), cfg.K)
+        check_topk(res["pred"][l], ref_p, prerouter_tau(u, executed, L["prerouter"], cfg.E, tc=tc), cfg.K)
 
 
 def run_stack(stack, cfg, T, x0, predicted, opts=None):
@@ -418,7 +408,7 @@ def test_prefill_stack_full_size_sampled(cuda_ok):
            if k != "err"}
     sample = [0, 1, cfg.layers // 2, cfg.layers - 1]
     needed = {l: sorted(set(sub["idx"][l].reshape(-1).tolist())) for l in sample}
-    _check_stack(cfg, lambda l: inputs.layer(cfg, l, experts=needed[l]), len(toks), sub, x0[toks], sample)
+    _check_stack(cfg, lambda l: inputs.layer(cfg, l, experts=needed[l]), len(toks), sub, x0[toks], sample, tc=True)
 
 
 # Largest supported shapes (H 4096, I 2048) on both expert paths: 4 tokens (GEMV), 64 tokens (grouped GEMM).

@@ -6,6 +6,10 @@
   butterfly reduction over the lanes of a row, the bias add), emulated here
   with one float32 rounding per operation -- including activations so small
   that their fp16 copies round.
+* ``router_tau_tc`` bounds the tensor-core router's error under a pessimistic
+  model of the MMA (each 16-product block added to the accumulator with every
+  addend truncated at the largest one's last place, the result truncated to
+  fp32), followed by the kernel's fp32 group sums and fused multiply-adds.
 * ``check_topk`` accepts the exact top-K and certified near-ties and refuses
   wrong sets, duplicates, out-of-range indices and wrong order.
 * ``check_bf16_rounding`` accepts round-to-nearest-even and, only next to a
@@ -18,7 +22,8 @@ import pytest
 
 from gen import CONFIGS, inputs
 from oracle import moe_oracle as O
-from parity import EPS32, check_bf16_rounding, check_topk, fp16_input_error, qmat_abs_terms, router_tau
+from parity import (EPS32, check_bf16_rounding, check_topk, fp16_input_error, qmat_abs_terms, router_tau,
+                    router_tau_tc)
 
 f32 = np.float32
 
@@ -80,6 +85,63 @@ def test_router_tau_bounds_an_fp32_evaluation_in_kernel_order(cfg_id, H, zipf, s
         assert np.any(err > rounding_only)
     else:
         assert np.all(fp16_input_error(u) == 0)
+
+
+def _f32_toward_zero(x):
+    m, e = np.frexp(np.asarray(x, np.float64))
+    return np.ldexp(np.trunc(m * 2.0 ** 24) / 2.0 ** 24, e)
+
+
+def _truncating_block(acc, prods):
+    """acc + sum(prods) with every addend truncated at the last place of the largest, then to fp32."""
+    add = np.concatenate([acc[..., None], prods], axis=-1)
+    mx = np.max(np.abs(add), axis=-1, keepdims=True)
+    quantum = np.where(mx > 0, np.ldexp(1.0, (np.frexp(np.where(mx > 0, mx, 1.0))[1] - 1) - 23), 1.0)
+    return _f32_toward_zero(np.sum(np.trunc(add / quantum) * quantum, axis=-1))
+
+
+def emulate_router_tc(u: np.ndarray, router: dict) -> np.ndarray:
+    """Tensor-core router logits [T, E]: per group four truncating 16-product blocks of (q - 128) u, the fp32
+    group sum of u (four 16-element runs, then pairwise), b + 128 s in fp32, two fp32 fused multiply-adds."""
+    T, H = u.shape
+    qm = O.unpack_codes(router["q"], 8).astype(np.float64) - 128.0
+    E = qm.shape[0]
+    s = router["s"].astype(np.float64)
+    bprime = (router["b"].astype(np.float32) + f32(128.0) * router["s"].astype(np.float32)).astype(np.float64)
+    acc = np.zeros((T, E), np.float64)
+    for g in range(H // 64):
+        D = np.zeros((T, E))
+        for blk in range(4):
+            k = slice(64 * g + 16 * blk, 64 * g + 16 * blk + 16)
+            D = _truncating_block(D, u[:, None, k] * qm[None, :, k])
+        quarters = []
+        for qq in range(4):
+            run = u[:, 64 * g + 16 * qq: 64 * g + 16 * qq + 16].astype(np.float32)
+            acc_q = np.zeros(T, np.float32)
+            for i in range(16):
+                acc_q = (acc_q + run[:, i]).astype(np.float32)
+            quarters.append(acc_q)
+        U = ((quarters[0] + quarters[1]).astype(np.float32) + (quarters[2] + quarters[3]).astype(np.float32))
+        U = U.astype(np.float32).astype(np.float64)
+        acc = (s[None, :, g] * D + acc).astype(np.float32).astype(np.float64)
+        acc = (bprime[None, :, g] * U[:, None] + acc).astype(np.float32).astype(np.float64)
+    beta = np.asarray(router["beta"], np.float32)
+    return (acc + beta).astype(np.float32).astype(np.float64)
+
+
+@pytest.mark.parametrize("H,zipf", [(256, 0.0), (2048, 1.1)])
+@pytest.mark.parametrize("scale", [1.0, 3e-6])
+def test_router_tau_tc_bounds_a_truncating_tensor_core_model(H, zipf, scale):
+    cfg = dataclasses.replace(CONFIGS[0], E=16, H=H, zipf_s=zipf)
+    router = inputs.router(cfg, 0)
+    rng = np.random.default_rng(int(scale * 1e6) + H + 7)
+    u = _bf16(rng.standard_normal((3, H)) * scale)
+    exact = O.router_logits(u, router)
+    err = np.abs(emulate_router_tc(u, router) - exact)
+    tau = router_tau_tc(u, router)
+    assert np.all(err <= tau), float(np.max(err / tau))
+    # the model is not trivially exact: truncation leaves a visible error
+    assert np.max(err) > 0
 
 
 # ----------------------------------------------------------------------------- check_topk
