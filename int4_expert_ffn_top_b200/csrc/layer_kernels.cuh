@@ -714,58 +714,67 @@ __global__ void __launch_bounds__(kThreads) prerouter_w1_kernel(PreW1Args a) {
   }
 }
 
-// Second Prerouter layer: scores[t][e] = b2[e] + sum_p W2[e][p] * z[t][p].
-// A CTA takes 32 tokens x 32 rows; z of its tokens is staged in shared memory
-// 256 inputs at a time (rows padded by one float against bank conflicts); lane
-// = token, each warp 4 rows, whose W2 values are warp-uniform (broadcast) loads.
-constexpr int kW2Tok = 32, kW2Rows = 32, kW2Chunk = 256;
-__global__ void __launch_bounds__(kThreads) prerouter_w2_kernel(const float* __restrict__ z, int T, int P,
-                                                                const uint16_t* __restrict__ W2,
-                                                                const uint16_t* __restrict__ b2, int En,
-                                                                float* __restrict__ scores) {
-  __shared__ float zs[kW2Tok * (kW2Chunk + 1)];
-  const int t0 = blockIdx.y * kW2Tok, e0 = blockIdx.x * kW2Rows;
-  const int nt = min(kW2Tok, T - t0);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int RPW = kW2Rows / kWarps;  // rows per warp
-  float acc[RPW];
+// Second Prerouter layer: scores[t][e] = b2[e] + sum_p W2[e][p] * z[t][p], register-tiled.  A CTA of 256
+// threads takes 64 tokens x 64 rows, each thread 4 tokens x 4 rows; z and W2 (as fp32) are staged in shared
+// memory 32 inputs at a time, input-major, so a thread reads one float4 of each per input.  A chunk's 32
+// products are summed in order and the chunk sum is added to the total: at most 32 + ceil(P/32) + 1 fp32
+// roundings on the path of any product.
+constexpr int kW2T = 64, kW2E = 64, kW2K = 32, kW2Threads = 256;
+__global__ void __launch_bounds__(kW2Threads) prerouter_w2_kernel(const float* __restrict__ z, int T, int P,
+                                                                   const uint16_t* __restrict__ W2,
+                                                                   const uint16_t* __restrict__ b2, int En,
+                                                                   float* __restrict__ scores) {
+  __shared__ __align__(16) float zs[kW2K][kW2T + 4];
+  __shared__ __align__(16) float ws[kW2K][kW2E + 4];
+  const int t0 = blockIdx.y * kW2T, e0 = blockIdx.x * kW2E;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;  // rows e0 + 4 tx + j, tokens t0 + 4 ty + i
+  float acc[4][4];
 #pragma unroll
-  for (int j = 0; j < RPW; ++j) acc[j] = 0.f;
-  for (int p0 = 0; p0 < P; p0 += kW2Chunk) {
-    const int pc = min(kW2Chunk, P - p0);
-    __syncthreads();
-    for (int i = threadIdx.x; i < kW2Tok * pc; i += blockDim.x) {
-      const int tt = i / pc, pp = i - tt * pc;
-      zs[tt * (kW2Chunk + 1) + pp] = tt < nt ? z[static_cast<size_t>(t0 + tt) * P + p0 + pp] : 0.f;
-    }
-    __syncthreads();
-    const float* zr = zs + lane * (kW2Chunk + 1);
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 #pragma unroll 1
-    for (int pp = 0; pp < pc; pp += 8) {
-      float zv[8];
-#pragma unroll
-      for (int m = 0; m < 8; ++m) zv[m] = zr[pp + m];
-#pragma unroll
-      for (int j = 0; j < RPW; ++j) {
-        const int e = e0 + warp * RPW + j;
-        if (e < En) {
-          const uint4 w = *reinterpret_cast<const uint4*>(W2 + static_cast<size_t>(e) * P + p0 + pp);
-          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const float2 f = __half22float2(as_h2(ws[m]));
-            acc[j] = fmaf(f.x, zv[2 * m], acc[j]);
-            acc[j] = fmaf(f.y, zv[2 * m + 1], acc[j]);
-          }
-        }
-      }
+  for (int p0 = 0; p0 < P; p0 += kW2K) {
+    const int pc = min(kW2K, P - p0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < kW2T * kW2K; i += kW2Threads) {
+      const int tt = i / kW2K, pp = i % kW2K, t = t0 + tt;  // consecutive threads: consecutive inputs
+      zs[pp][tt] = (t < T && pp < pc) ? z[static_cast<size_t>(t) * P + p0 + pp] : 0.f;
     }
-  }
-  if (lane < nt) {
+    for (int i = threadIdx.x; i < kW2E * kW2K; i += kW2Threads) {
+      const int ee = i / kW2K, pp = i % kW2K, e = e0 + ee;
+      ws[pp][ee] = (e < En && pp < pc) ? half_bits_to_float(W2[static_cast<size_t>(e) * P + p0 + pp]) : 0.f;
+    }
+    __syncthreads();
+    float part[4][4];
 #pragma unroll
-    for (int j = 0; j < RPW; ++j) {
-      const int e = e0 + warp * RPW + j;
-      if (e < En) scores[static_cast<size_t>(t0 + lane) * En + e] = acc[j] + half_bits_to_float(b2[e]);
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) part[i][j] = 0.f;
+#pragma unroll 8
+    for (int pp = 0; pp < kW2K; ++pp) {
+      const float4 zv = *reinterpret_cast<const float4*>(&zs[pp][4 * ty]);
+      const float4 wv = *reinterpret_cast<const float4*>(&ws[pp][4 * tx]);
+      const float zz[4] = {zv.x, zv.y, zv.z, zv.w}, ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) part[i][j] = fmaf(zz[i], ww[j], part[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] += part[i][j];
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int e = e0 + 4 * tx + j;
+    if (e >= En) continue;
+    const float b = half_bits_to_float(b2[e]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int t = t0 + 4 * ty + i;
+      if (t < T) scores[static_cast<size_t>(t) * En + e] = acc[i][j] + b;
     }
   }
 }

@@ -595,8 +595,8 @@ moe_status prerouter_h(const moe_prerouter* P, const uint16_t* u, const int32_t*
     dim3 g1((P->P + kWarps - 1) / kWarps, (T + TB - 1) / TB);
     prerouter_w1_kernel<H / 8><<<g1, kThreads, smem, st>>>(a);
   }
-  dim3 g2((P->E_next + kW2Rows - 1) / kW2Rows, (T + kW2Tok - 1) / kW2Tok);
-  prerouter_w2_kernel<<<g2, kThreads, 0, st>>>(z, T, P->P, P->W2, P->b2, P->E_next, scores);
+  dim3 g2((P->E_next + kW2E - 1) / kW2E, (T + kW2T - 1) / kW2T);
+  prerouter_w2_kernel<<<g2, kW2Threads, 0, st>>>(z, T, P->P, P->W2, P->b2, P->E_next, scores);
   topk_kernel<<<(T + kWarps - 1) / kWarps, kThreads, 0, st>>>(scores, T, P->E_next, K_next, pred, nullptr);
   return launch_status();
 }

@@ -45,12 +45,26 @@ MOE_DEV bool bar_test(uint64_t* b, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread sleeps until the phase completes or about `ns` nanoseconds
+// pass, instead of spinning and taking issue slots from the warps that do the work.
+MOE_DEV bool bar_test_sleep(uint64_t* b, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(sa(b)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
+constexpr uint32_t kSuspendNs = 20000;
+
 MOE_DEV bool bar_wait(uint64_t* b, uint32_t parity, long long timeout_ns) {
   if (bar_test(b, parity)) return true;
   const long long deadline = gtime() + timeout_ns;
-  for (int it = 1;; ++it) {
-    if (bar_test(b, parity)) return true;
-    if ((it & 63) == 0 && gtime() > deadline) return false;
+  for (;;) {
+    if (bar_test_sleep(b, parity, kSuspendNs)) return true;
+    if (gtime() > deadline) return false;
   }
 }
 

@@ -94,8 +94,13 @@ def prerouter_tau(u, sel, head, E, n_round=128, tc=False):
     ``tc``: the first layer ran on the tensor cores: W1 split exactly into two
     bf16 parts, u unrounded, four accumulation chains of 2 (H + E) / 64 MMA
     blocks each, then three chain adds and the bias add.  Otherwise the GEMV:
-    ``n_round`` roundings per product term and u rounded to fp16.
+    ``n_round`` roundings per product term and u rounded to fp16.  The second
+    layer takes at most 33 + ceil(P / 32) roundings per product (32-term chunk
+    sums added up, then the bias) on the many-token path and 8 ceil(P / 256) + 6
+    in the decode kernels; ``n_round`` must cover both.
     """
+    P = head["W2"].shape[1]
+    assert n_round >= max(33 + -(-P // 32), 8 * -(-P // 256) + 6)
     W1 = np.abs(head["W1"].astype(np.float64))
     W2 = np.abs(head["W2"].astype(np.float64))
     xin = np.concatenate([np.abs(u), O.multi_hot(sel, E)], axis=1)
