@@ -3,39 +3,44 @@
 //
 // Per expert bucket D[o][t] = sum_k W[o][k] * X[t][k] ("swap AB": 128 weight
 // rows are the MMA M side, the bucket's tokens the N side).  A tile is 128
-// weight rows x up to 64 tokens; K advances one quantisation group (64) per
-// step.  One CTA per SM walks the device-built tile list (tiles c, c + grid,
-// ...), and every role runs the same sequence of (tile, step), so the pipeline
-// stays full across tiles:
-//  * warp 0, one lane (TMA): per tile the fp16 scales and biases of its 128 rows
-//    (a box of a 3-D byte map {record bytes, rows, experts} over the expert
-//    pool, two buffers when they fit); every four steps the 128 code bytes of
-//    each row (a box of a second map over the same bytes, 128-byte swizzle,
-//    16 KB, three stages); per step the step's token rows (2-D map, 128-byte
-//    swizzle, boxes of 32 rows, only as many as the tile has tokens);
-//  * 8 warps dequantise, two K steps per pass: thread (row r, half h) reads
-//    16 code bytes per step (lanes of a warp take 8 consecutive rows per
-//    128-byte wavefront, conflict-free under the swizzle), forms w = q*s + b in
-//    fp16 (one rounding) and stores four 16-byte chunks into the
-//    128-byte-swizzled K-major A stage.  K inside each 8-element block is in
-//    "pair order" (q_j, q_{j+4}), the order the magic-exponent unpacking
-//    produces; the token operand is stored in the same order, so the products
-//    are those of the plain order;
-//  * warps 1 and 2, one lane each (MMA): tcgen05.mma kind::f16 into one of two sets of
-//    four 64-column TMEM accumulators (tiles alternate); K slice c (16 wide) of every step goes to
-//    accumulator c, issued by MMA warp c % 2 -- four independent accumulation chains, and two issuing
-//    threads, since one thread issues an MMA only every ~175 cycles; each commit releases the step's
-//    operand stages and, after a tile, its accumulators;
-//  * 8 epilogue warps (TMEM lane quadrant = warp % 4, two warps per
-//    quadrant splitting the token columns): drain and add the finished
-//    accumulators with tcgen05.ld while the next tile's main loop runs: SwiGLU of
-//    interleaved gate/up rows (output in pair order, the next GEMM's token
-//    operand) or the down projection's LoRA delta and gating weight; staged in
-//    shared memory for coalesced fp16 stores; then the accumulator is released.
-// K must be a multiple of 128 (an even number of steps).
+// weight rows x up to 128 tokens (the MMA's N is the tile's token count rounded
+// up to 16); K advances one quantisation group (64) per step, four steps per
+// pass.  One CTA per SM walks the device-built tile list (tiles c, c + grid,
+// ...), and every role runs the same sequence of (tile, pass, step), so the
+// pipeline stays full across tiles:
+//  * warp 0, one lane (weight TMA, running ahead as far as its buffers allow):
+//    per tile the fp16 scales and biases of its 128 rows (a box of a 3-D byte
+//    map {record bytes, rows, experts} over the expert pool, two buffers when
+//    they fit); per pass the 128 code bytes of each row (a box of a second map
+//    over the same bytes, 128-byte swizzle, 16 KB, three stages);
+//  * warp 2, one lane (token TMA): per step the step's token rows (2-D map,
+//    128-byte swizzle, boxes of 32 rows, only as many as the tile has tokens;
+//    four 16 KB stages);
+//  * warp 1, one lane (MMA): per step four tcgen05.mma kind::f16 (one per 16-wide
+//    K slice) in straight-line code -- A from tensor memory, B (tokens) from
+//    shared memory -- into the tile's accumulator (two 128-column TMEM
+//    accumulators, tiles alternate); one thread issues the whole tile: a
+//    predicate, a loop or a wait around an MMA costs the issuing thread more
+//    than the MMA's own tensor-core time, so work per instruction (N up to 128)
+//    and few instructions around it are what count;
+//  * 8 warps dequantise a pass (one raw stage, four K steps) at a time straight
+//    into tensor memory (two passes in flight): a warp owns the TMEM lanes of
+//    its quadrant (warp % 4), thread = weight row, the quadrant's two warps the
+//    two halves of a step's 64 inputs; a thread reads 16 code bytes per step
+//    (conflict-free under the swizzle), forms w = q*s + b in fp16 (one rounding)
+//    and stores 16 columns with tcgen05.st; one mbarrier hand-off per pass in
+//    each direction.  K inside each 8-element block is in "pair order" (q_j,
+//    q_{j+4}), the order the magic-exponent unpacking produces; the token operand
+//    is stored in the same order, so the products are those of the plain order;
+//  * 8 epilogue warps (TMEM lane quadrant = warp % 4, two warps per quadrant,
+//    64 token columns each in two blocks of 32): drain the finished accumulator
+//    with tcgen05.ld while the next tile's main loop runs: SwiGLU of interleaved
+//    gate/up rows (output in pair order, the next GEMM's token operand) or the
+//    down projection's LoRA delta and gating weight; staged in shared memory for
+//    coalesced fp16 stores; then the accumulator is released.
 // Every wait is bounded: a role whose wait runs out stops issuing copies or
-// MMAs and records MOE_ERR_TIMEOUT; before the CTA leaves, the copies and MMAs
-// it issued are waited for (bounded).
+// MMAs and records MOE_ERR_TIMEOUT; before the CTA leaves, the copies, MMAs and
+// tensor-memory stores it issued are waited for (bounded).
 #pragma once
 
 #include "tc_primitives.cuh"
@@ -52,52 +57,46 @@ using tc::EPI_DOWN;
 using tc::EPI_SWIGLU;
 using tc::instr_desc;
 using tc::mma_commit;
-using tc::mma_f16;
+using tc::mma_f16_ts;
 using tc::sa;
 using tc::smem_desc;
 using tc::tma_load_2d;
 using tc::tmem_ld32;
+using tc::tmem_st16;
+using tc::tmem_st_wait;
 using tc::Tile;
 
 constexpr int BM = 128;
-constexpr int BN = 64;   // tokens per tile: buckets average ~50 tokens at prefill; keeps the token ring deep
+constexpr int BN = 128;     // tokens per tile
 constexpr int BK = 64;
 constexpr int BROWS = 32;   // token rows per TMA box
-constexpr int RGROUPS = 4;  // quantisation groups per raw code load: 128-byte TMA rows (narrower rows cap the
-                            // TMA request rate well below the HBM bandwidth)
+constexpr int RGROUPS = 4;  // K steps per pass = quantisation groups per raw code load: 128-byte TMA rows
+                            // (narrower rows cap the TMA request rate well below the HBM bandwidth)
 constexpr int RSTAGES = 3;  // raw code stages (16 KB each): the weight bytes in flight per SM
-// Operand stages: a dequantised weight stage (16 KB) and a token stage (8 KB) per K step, released together by
-// the MMA warps' commits.
-constexpr int STAGES = 4;
-constexpr int BSTAGES = STAGES;
-constexpr int ASTAGES = STAGES;
+constexpr int BSTAGES = 4;  // token stages (16 KB each)
+constexpr int APASS = 2;    // dequantised weight passes in tensor memory (RGROUPS stages of 32 columns each)
 constexpr int kDqWarps = 8;
 constexpr int kDq = 32 * kDqWarps;
 constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant, splitting the tile's token columns
 constexpr int kEpi = 32 * kEpiWarps;
-constexpr int kMmaWarps = 2;  // MMA-issuing warps (one thread issues an MMA only every ~175 cycles); warp 1 + w
-                              // issues the chains w, w + kMmaWarps, ...
-constexpr int kThreads = 32 * (1 + kMmaWarps) + kDq + kEpi;  // TMA warp, MMA warps, dequant warps, epilogue warps
-constexpr int kWarpDq0 = 1 + kMmaWarps;                         // first dequantising warp
-constexpr int kWarpEpi0 = kWarpDq0 + kDqWarps;                  // first epilogue warp
+constexpr int kThreads = 96 + kDq + kEpi;  // weight TMA warp, MMA warp, token TMA warp, dequant, epilogue warps
+constexpr int kWarpDq0 = 3;                // first dequantising warp
+constexpr int kWarpEpi0 = kWarpDq0 + kDqWarps;
 constexpr int RAW_STAGE = BM * 32 * RGROUPS;
-constexpr int A_STAGE = BM * BK * 2;
 constexpr int B_STAGE = BN * BK * 2;
-constexpr int SB_MAX = BM * 256;           // scales + biases of 128 rows, K <= 4096
-constexpr int STAGE_OUT = BN * BM * 2;     // epilogue staging: up to BN tokens x 128 fp16
-// MMAs that accumulate into one TMEM accumulator run one after another (each waits for the previous sum), so a
-// tile's K steps are spread over ACC_CHAINS accumulators (MMA kk of every step into accumulator kk) that the
-// tensor core works on concurrently, and the epilogue adds them.  Two tiles in flight: 2 x ACC_CHAINS x BN columns.
-constexpr int ACC_CHAINS = 4;
-constexpr uint32_t TMEM_COLS = 2 * ACC_CHAINS * BN;
-constexpr int OFF_A = 0;
-constexpr int OFF_B = OFF_A + ASTAGES * A_STAGE;
+constexpr int A_COLS = BK / 2;    // TMEM columns of one dequantised weight stage (two fp16 per column)
+constexpr int ACC_COLS = 2 * BN;  // TMEM: two tiles' accumulators, then the weight stages
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int STAGE_OUT = BN * BM * 2;  // epilogue staging: up to BN tokens x 128 fp16
+constexpr int OFF_B = 0;
 constexpr int OFF_RAW = OFF_B + BSTAGES * B_STAGE;
-constexpr int LORA_T = 2 * BN * 32 * 4;    // epilogue staging of the tile's LoRA t vectors (two sets, r <= 32) ...
+constexpr int LORA_T = 2 * BN * 32 * 4;  // epilogue staging of the tile's LoRA t vectors (two sets, r <= 32) ...
 constexpr int OFF_OUT = OFF_RAW + RSTAGES * RAW_STAGE;
 constexpr int OFF_LT = OFF_OUT + STAGE_OUT;
-constexpr int OFF_RS = OFF_LT + LORA_T;    // ... and of its gating weights
+constexpr int OFF_RS = OFF_LT + LORA_T;  // ... and of its gating weights
 constexpr int OFF_SB = OFF_RS + BN * 4;
+static_assert(ACC_COLS + APASS * RGROUPS * A_COLS <= static_cast<int>(TMEM_COLS) && BK == 64 && kDqWarps == 8,
+              "tensor memory plan");
 
 // Bytes per row of the scale/bias box: the K/64 scales and K/64 biases (4*K/64 bytes), at least one 16-byte
 // TMA unit (the row record's zero padding covers the rest).
@@ -163,8 +162,6 @@ MOE_DEV uint4 dequant_pair_order(uint32_t w, __half2 s2, __half2 b2) {
                     h2_bits(__hfma2(q3, s2, b2)));
 }
 
-static_assert(BK / 16 == ACC_CHAINS && ACC_CHAINS % kMmaWarps == 0 && TMEM_COLS <= 512, "accumulator chains");
-
 MOE_DEV uint32_t parity(int count, int stages) { return static_cast<uint32_t>(count / stages) & 1u; }
 
 // OR of v over the 256 epilogue threads (named barrier 1), so that they take the same branch.
@@ -184,7 +181,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int KT = a.K / BK;
   const int SB_ROW = sb_row_bytes(a.K);  // scales at byte 0, biases at byte 2*KT of a row
-  uint8_t* smA = sm + OFF_A;
   uint8_t* smB = sm + OFF_B;
   uint8_t* smRaw = sm + OFF_RAW;
   uint16_t* stage = reinterpret_cast<uint16_t*>(sm + OFF_OUT);
@@ -194,9 +190,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
   uint64_t* raw_full = bars;
   uint64_t* raw_empty = raw_full + RSTAGES;
   uint64_t* b_full = raw_empty + RSTAGES;
-  uint64_t* a_full = b_full + STAGES;
-  uint64_t* st_empty = a_full + STAGES;   // both operand stages of a step are free (one commit per MMA warp)
-  uint64_t* sb_full = st_empty + STAGES;  // [2]
+  uint64_t* b_empty = b_full + BSTAGES;
+  uint64_t* a_full = b_empty + BSTAGES;   // [APASS] a pass's weight stages are in tensor memory
+  uint64_t* a_empty = a_full + APASS;     // [APASS] the MMA is done with a pass's weight stages
+  uint64_t* sb_full = a_empty + APASS;    // [2]
   uint64_t* sb_empty = sb_full + 2;       // [2]
   uint64_t* acc_full = sb_empty + 2;      // [2]
   uint64_t* acc_empty = acc_full + 2;     // [2]
@@ -209,20 +206,23 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
       bar_init(raw_full + s, 1);
       bar_init(raw_empty + s, kDqWarps);  // one elected arrival per warp
     }
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < BSTAGES; ++s) {
       bar_init(b_full + s, 1);
+      bar_init(b_empty + s, 1);
+    }
+    for (int s = 0; s < APASS; ++s) {
       bar_init(a_full + s, kDqWarps);
-      bar_init(st_empty + s, kMmaWarps);
+      bar_init(a_empty + s, 1);
     }
     for (int s = 0; s < 2; ++s) {
       bar_init(sb_full + s, 1);
       bar_init(sb_empty + s, kDqWarps);
-      bar_init(acc_full + s, kMmaWarps);
+      bar_init(acc_full + s, 1);
       bar_init(acc_empty + s, kEpiWarps);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) {  // the first MMA warp owns the TMEM allocation
+  if (warp == 1) {  // the MMA warp owns the TMEM allocation
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(sa(tmem_slot)),
                  "r"(TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -234,9 +234,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
   int fail = 0;
 
   if (warp == 0) {
-    // ---------------------------------------------------------------- TMA producer
+    // ---------------------------------------------------------------- weight TMA producer: scales, raw codes
+    // (runs ahead of the token copies as far as its buffers allow)
     if (lane == 0) {
-      int n_raw = 0, n_b = 0, n_sb = 0;  // copies issued so far (stage counters)
+      int n_raw = 0, n_sb = 0;  // copies issued so far (stage counters)
 #pragma unroll 1
       for (int ti = blockIdx.x; ti < n_tiles && !fail; ti += gridDim.x) {
         const Tile tile = a.tiles[ti];
@@ -252,20 +253,38 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
         bar_expect_tx(sb_full + tb, static_cast<uint32_t>(BM * SB_ROW));
         tma_load_3d(smSB + tb * BM * SB_ROW, smap, a.K / 2, y, ez, sb_full + tb);
         ++n_sb;
+#pragma unroll 1
+        for (int kt = 0; kt < KT; kt += RGROUPS) {
+          const int rs = n_raw % RSTAGES;
+          if (!bar_wait(raw_empty + rs, parity(n_raw, RSTAGES) ^ 1u, a.timeout_ns)) {
+            fail = 1;
+            break;
+          }
+          bar_expect_tx(raw_full + rs, RAW_STAGE);
+          tma_load_3d(smRaw + rs * RAW_STAGE, cmap, kt * 32, y, ez, raw_full + rs);
+          ++n_raw;
+        }
+      }
+      if (fail) {  // let the copies already issued land before the CTA can leave
+#pragma unroll 1
+        for (int q = n_raw > RSTAGES ? n_raw - RSTAGES : 0; q < n_raw; ++q)
+          bar_wait(raw_full + q % RSTAGES, parity(q, RSTAGES), a.timeout_ns);
+#pragma unroll 1
+        for (int q = n_sb > nsb ? n_sb - nsb : 0; q < n_sb; ++q) bar_wait(sb_full + q % nsb, parity(q, nsb), a.timeout_ns);
+      }
+    }
+  } else if (warp == 2) {
+    // ---------------------------------------------------------------- token TMA producer
+    if (lane == 0) {
+      int n_b = 0;
+#pragma unroll 1
+      for (int ti = blockIdx.x; ti < n_tiles && !fail; ti += gridDim.x) {
+        const Tile tile = a.tiles[ti];
         const int nb = (tile.n + BROWS - 1) / BROWS;
 #pragma unroll 1
         for (int kt = 0; kt < KT; ++kt) {
-          const int rs = n_raw % RSTAGES, bs = n_b % BSTAGES;
-          if (kt % RGROUPS == 0) {
-            if (!bar_wait(raw_empty + rs, parity(n_raw, RSTAGES) ^ 1u, a.timeout_ns)) {
-              fail = 1;
-              break;
-            }
-            bar_expect_tx(raw_full + rs, RAW_STAGE);
-            tma_load_3d(smRaw + rs * RAW_STAGE, cmap, kt * 32, y, ez, raw_full + rs);
-            ++n_raw;
-          }
-          if (!bar_wait(st_empty + bs, parity(n_b, STAGES) ^ 1u, a.timeout_ns)) {
+          const int bs = n_b % BSTAGES;
+          if (!bar_wait(b_empty + bs, parity(n_b, BSTAGES) ^ 1u, a.timeout_ns)) {
             fail = 1;
             break;
           }
@@ -277,22 +296,16 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
           ++n_b;
         }
       }
-      if (fail) {  // let the copies already issued land before the CTA can leave
-#pragma unroll 1
-        for (int q = n_raw > RSTAGES ? n_raw - RSTAGES : 0; q < n_raw; ++q)
-          bar_wait(raw_full + q % RSTAGES, parity(q, RSTAGES), a.timeout_ns);
+      if (fail) {
 #pragma unroll 1
         for (int q = n_b > BSTAGES ? n_b - BSTAGES : 0; q < n_b; ++q)
           bar_wait(b_full + q % BSTAGES, parity(q, BSTAGES), a.timeout_ns);
-#pragma unroll 1
-        for (int q = n_sb > nsb ? n_sb - nsb : 0; q < n_sb; ++q) bar_wait(sb_full + q % nsb, parity(q, nsb), a.timeout_ns);
       }
     }
-  } else if (warp < kWarpDq0) {
+  } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issue
-    const int ch = warp - 1;
     if (lane == 0) {
-      int g = 0, it = 0, last_ab = -1;
+      int n_b = 0, np = 0, it = 0, last_ab = -1;
       uint32_t last_par = 0;
 #pragma unroll 1
       for (int ti = blockIdx.x; ti < n_tiles && !fail; ti += gridDim.x, ++it) {
@@ -303,37 +316,51 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
           break;
         }
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const uint32_t d = tmem + static_cast<uint32_t>(ab * ACC_CHAINS * BN);
+        const uint32_t d = tmem + static_cast<uint32_t>(ab * BN);
         const uint32_t idesc = instr_desc((tile.n + 15) & ~15);
 #pragma unroll 1
-        for (int kt = 0; kt < KT; ++kt, ++g) {
-          const int s = g % STAGES;
-          if (!bar_wait(a_full + s, parity(g, STAGES), a.timeout_ns) ||
-              !bar_wait(b_full + s, parity(g, STAGES), a.timeout_ns)) {
+        for (int kt = 0; kt < KT && !fail; kt += RGROUPS, ++np) {
+          const int ps = np % APASS, nst = KT - kt < RGROUPS ? KT - kt : RGROUPS;
+          if (!bar_wait(a_full + ps, parity(np, APASS), a.timeout_ns)) {
             fail = 1;
             break;
           }
-          asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-          const uint32_t a0 = sa(smA + s * A_STAGE), b0 = sa(smB + s * B_STAGE);
-#pragma unroll
-          for (int c = ch; c < ACC_CHAINS; c += kMmaWarps)  // K slice c of the step into accumulator c
-            mma_f16(d + c * BN, smem_desc(a0 + c * 32), smem_desc(b0 + c * 32), idesc, kt != 0);
-          mma_commit(st_empty + s);
+#pragma unroll 1
+          for (int st = 0; st < nst; ++st, ++n_b) {
+            const int bs = n_b % BSTAGES;
+            if (!bar_wait(b_full + bs, parity(n_b, BSTAGES), a.timeout_ns)) {
+              fail = 1;
+              break;
+            }
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            // the step's four 16-wide K slices: A 8 TMEM columns each, B 32 bytes each (the descriptor's
+            // start-address field moves by 2)
+            const uint32_t a0 = tmem + static_cast<uint32_t>(ACC_COLS + (ps * RGROUPS + st) * A_COLS);
+            const uint64_t b0 = smem_desc(sa(smB + bs * B_STAGE));
+            mma_f16_ts(d, a0, b0, idesc, (kt | st) != 0);
+            mma_f16_ts(d, a0 + 8, b0 + 2, idesc, 1u);
+            mma_f16_ts(d, a0 + 16, b0 + 4, idesc, 1u);
+            mma_f16_ts(d, a0 + 24, b0 + 6, idesc, 1u);
+            mma_commit(b_empty + bs);
+          }
+          mma_commit(a_empty + ps);
         }
         mma_commit(acc_full + ab);  // also on failure: completes once every MMA issued into this buffer has
         last_ab = ab;
         last_par = parity(it, 2);
       }
-      // never release TMEM with MMAs in flight: wait for the last commit (this chain's part of it)
+      // never release TMEM with MMAs in flight: wait for the last commit
       if (fail && last_ab >= 0) bar_wait(acc_full + last_ab, last_par, a.timeout_ns);
     }
   } else if (warp < kWarpEpi0) {
     // ---------------------------------------------------------------- dequantising warps
     const int d = tid - 32 * kWarpDq0;
-    // lanes l and l+8 take the two halves of one row; a 128-byte wavefront covers 8 consecutive rows
-    const int r = 16 * (d >> 5) + (lane & 7) + 8 * (lane >> 4), h = (lane >> 3) & 1;
+    // a warp writes the TMEM lanes of its quadrant (warp % 4): thread = weight row r, and the two warps of a
+    // quadrant take the two halves h of each step's 64 inputs
+    const int quad = warp & 3, h = (warp - kWarpDq0) >> 2, r = 32 * quad + lane;
+    const uint32_t a_lane = tmem + (static_cast<uint32_t>(32 * quad) << 16) + ACC_COLS + 16 * h;
     const bool vec8 = (KT & 7) == 0;
-    int g = 0, it = 0, nr = 0;
+    int np = 0, it = 0;
 #pragma unroll 1
     for (int ti = blockIdx.x; ti < n_tiles && !fail; ti += gridDim.x, ++it) {
       const int tb = it % nsb;
@@ -345,64 +372,67 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
       // a row's scale/bias run sits in one bank for all rows: read them 8 groups at a time
       uint4 s8 = make_uint4(0, 0, 0, 0), b8 = s8;
 #pragma unroll 1
-      for (int kt = 0; kt < KT; kt += 2, g += 2) {  // two K steps per pass (KT is even): more independent work per
-                                                   // hand-off
+      for (int kt = 0; kt < KT; kt += RGROUPS, ++np) {  // one raw stage (RGROUPS steps) per pass
+        const int nst = KT - kt < RGROUPS ? KT - kt : RGROUPS;
         if (vec8 && (kt & 7) == 0) {
           s8 = reinterpret_cast<const uint4*>(sbr)[kt >> 3];
           b8 = reinterpret_cast<const uint4*>(sbr + KT)[kt >> 3];
         }
-        uint32_t sw, bw;  // low half: step kt, high half: step kt + 1
+        uint32_t sw[2], bw[2];  // fp16 pairs: steps (kt, kt + 1), (kt + 2, kt + 3)
         if (vec8) {
-          const int j = (kt & 7) >> 1;
-          sw = j == 0 ? s8.x : j == 1 ? s8.y : j == 2 ? s8.z : s8.w;
-          bw = j == 0 ? b8.x : j == 1 ? b8.y : j == 2 ? b8.z : b8.w;
+          const bool hi = (kt & 7) != 0;
+          sw[0] = hi ? s8.z : s8.x;
+          sw[1] = hi ? s8.w : s8.y;
+          bw[0] = hi ? b8.z : b8.x;
+          bw[1] = hi ? b8.w : b8.y;
         } else {
-          sw = sbr[kt] | (static_cast<uint32_t>(sbr[kt + 1]) << 16);
-          bw = sbr[KT + kt] | (static_cast<uint32_t>(sbr[KT + kt + 1]) << 16);
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int k0 = kt + 2 * j < KT ? kt + 2 * j : KT - 1, k1 = kt + 2 * j + 1 < KT ? kt + 2 * j + 1 : KT - 1;
+            sw[j] = sbr[k0] | (static_cast<uint32_t>(sbr[k1]) << 16);
+            bw[j] = sbr[KT + k0] | (static_cast<uint32_t>(sbr[KT + k1]) << 16);
+          }
         }
-        const int rs = nr % RSTAGES, grp = kt % RGROUPS;  // grp is even: groups grp and grp + 1 of the raw stage
-        if (__any_sync(0xffffffffu, grp == 0 && !bar_wait(raw_full + rs, parity(nr, RSTAGES), a.timeout_ns))) {
+        const int rs = np % RSTAGES;  // raw stages go round once per pass, as the passes do
+        if (__any_sync(0xffffffffu, !bar_wait(raw_full + rs, parity(np, RSTAGES), a.timeout_ns))) {
           fail = 1;
           break;
         }
-        // chunk (2 grp + h) of row r, 128-byte swizzle: 16-byte chunk c of a row sits at c ^ (r % 8)
+        // chunk (2 st + h) of row r, 128-byte swizzle: 16-byte chunk c of a row sits at c ^ (r % 8)
         const uint8_t* rrow = smRaw + rs * RAW_STAGE + r * 128;
-        const uint4 q0 = *reinterpret_cast<const uint4*>(rrow + (((2 * grp + h) ^ (r & 7)) << 4));
-        const uint4 q1 = *reinterpret_cast<const uint4*>(rrow + (((2 * grp + 2 + h) ^ (r & 7)) << 4));
-        if (grp + 1 == RGROUPS - 1 || kt + 1 == KT - 1) {
-          __syncwarp();
-          if (lane == 0) bar_arrive(raw_empty + rs);
-          ++nr;
-        }
-        const __half2 s0 = __half2half2(__ushort_as_half(static_cast<uint16_t>(sw))),
-                      b0 = __half2half2(__ushort_as_half(static_cast<uint16_t>(bw)));
-        const __half2 s1 = __half2half2(__ushort_as_half(static_cast<uint16_t>(sw >> 16))),
-                      b1 = __half2half2(__ushort_as_half(static_cast<uint16_t>(bw >> 16)));
-        uint4 w[8];
-        w[0] = dequant_pair_order(q0.x, s0, b0);
-        w[1] = dequant_pair_order(q0.y, s0, b0);
-        w[2] = dequant_pair_order(q0.z, s0, b0);
-        w[3] = dequant_pair_order(q0.w, s0, b0);
-        w[4] = dequant_pair_order(q1.x, s1, b1);
-        w[5] = dequant_pair_order(q1.y, s1, b1);
-        w[6] = dequant_pair_order(q1.z, s1, b1);
-        w[7] = dequant_pair_order(q1.w, s1, b1);
-        const int c0 = 4 * h, x = r & 7;
+        uint4 q[RGROUPS];
 #pragma unroll
-        for (int st = 0; st < 2; ++st) {
-          const int as = (g + st) % STAGES;
-          if (__any_sync(0xffffffffu, !bar_wait(st_empty + as, parity(g + st, STAGES) ^ 1u, a.timeout_ns))) {
-            fail = 1;  // the MMA may still read this stage
-            break;
+        for (int st = 0; st < RGROUPS; ++st)
+          q[st] = st < nst ? *reinterpret_cast<const uint4*>(rrow + (((2 * st + h) ^ (r & 7)) << 4))
+                           : make_uint4(0, 0, 0, 0);
+        __syncwarp();
+        if (lane == 0) bar_arrive(raw_empty + rs);
+        const int ps = np % APASS;
+        if (__any_sync(0xffffffffu, !bar_wait(a_empty + ps, parity(np, APASS) ^ 1u, a.timeout_ns))) {
+          fail = 1;  // the MMA may still read this pass's stages
+          break;
+        }
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+#pragma unroll
+        for (int st = 0; st < RGROUPS; ++st) {
+          if (st < nst) {
+            const uint32_t sp = (st & 1) ? sw[st >> 1] >> 16 : sw[st >> 1] & 0xFFFFu;
+            const uint32_t bp = (st & 1) ? bw[st >> 1] >> 16 : bw[st >> 1] & 0xFFFFu;
+            const __half2 s2 = __half2half2(__ushort_as_half(static_cast<uint16_t>(sp)));
+            const __half2 b2 = __half2half2(__ushort_as_half(static_cast<uint16_t>(bp)));
+            const uint4 w0 = dequant_pair_order(q[st].x, s2, b2), w1 = dequant_pair_order(q[st].y, s2, b2);
+            const uint4 w2 = dequant_pair_order(q[st].z, s2, b2), w3 = dequant_pair_order(q[st].w, s2, b2);
+            const uint32_t v[16] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w,
+                                    w2.x, w2.y, w2.z, w2.w, w3.x, w3.y, w3.z, w3.w};
+            // inputs 32 h .. 32 h + 31 of the step: columns 16 h .. 16 h + 15 of its stage
+            tmem_st16(a_lane + (ps * RGROUPS + st) * A_COLS, v);
           }
-          uint8_t* dd = smA + as * A_STAGE + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(dd + (((c0 + j) ^ x) << 4)) = w[4 * st + j];
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          __syncwarp();
-          if (lane == 0 && !(g + st == 0 && d == 0 && ti == a.drop_tile)) bar_arrive(a_full + as);
         }
-        if (fail) break;
+        tmem_st_wait();
+        // the pass's stages are in tensor memory: hand them to the MMA
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        __syncwarp();
+        if (lane == 0 && !(kt == 0 && d == 0 && ti == a.drop_tile)) bar_arrive(a_full + ps);
       }
       if (fail) break;
       __syncwarp();
@@ -412,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
     // ---------------------------------------------------------------- epilogue (TMEM lane quadrant = warp % 4)
     const int ew = warp - kWarpEpi0;  // 0..7
     const int quad = warp & 3;
-    const int chalf = ew >> 2;             // token columns [32 chalf, 32 chalf + 32)
+    const int chalf = ew >> 2;             // token columns [64 chalf, 64 chalf + 64), two blocks of 32
     const int L = quad * 32 + lane;        // TMEM lane = tile row
     const int et = tid - 32 * kWarpEpi0;  // 0..255 among the epilogue threads
     const int r = a.lora_r;
@@ -424,7 +454,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
       const Tile tile = a.tiles[ti];
       const int ab = it & 1;
       const int o = tile.mt * BM + L;
-      const int c0 = 32 * chalf;
       // per-tile inputs of the epilogue, staged once while the accumulator is still being written
       const bool swiglu = a.epi == EPI_SWIGLU;
       const bool up = swiglu && (L & 1) != 0;
@@ -452,50 +481,58 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
         break;
       }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t taddr =
-          tmem + static_cast<uint32_t>(ab * ACC_CHAINS * BN) + ((static_cast<uint32_t>(quad) * 32u) << 16);
+      const uint32_t taddr = tmem + static_cast<uint32_t>(ab * BN) + ((static_cast<uint32_t>(quad) * 32u) << 16);
       const float* ltr = lt + (up ? BN * 32 : 0);
-      float v[32];
-      const bool live = c0 < tile.n;
-      if (live) {  // the sum of the accumulator chains
-        tmem_ld32(taddr + c0, v);
+      bool range_bad = false;  // a SwiGLU output fp16 cannot hold: MOE_ERR_RANGE
 #pragma unroll 1
-        for (int ch = 1; ch < ACC_CHAINS; ++ch) {
-          float w[32];
-          tmem_ld32(taddr + ch * BN + c0, w);
-#pragma unroll
-          for (int t = 0; t < 32; ++t) v[t] += w[t];
+      for (int blk = 0; blk < 2; ++blk) {
+        const int c0 = 64 * chalf + 32 * blk;
+        float v[32];
+        const bool live = c0 < tile.n;
+        if (live) tmem_ld32(taddr + c0, v);
+        if (blk == 1) {  // the accumulator is read: release it for the tile after next
+          asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) bar_arrive(acc_empty + ab);
         }
-      }
-      // the accumulator is read: release it for the tile after next
-      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-      __syncwarp();
-      if (lane == 0) bar_arrive(acc_empty + ab);
-      if (live && Bsrc) {  // unmerged LoRA: + scale * B[row] . t[token]
+        if (live && Bsrc) {  // unmerged LoRA: + scale * B[row] . t[token]
 #pragma unroll 1
-        for (int i = 0; i < r; ++i) {
-          const float bi = a.lora_scale * half_bits_to_float(Bsrc[static_cast<size_t>(brow) * r + i]);
+          for (int i = 0; i < r; ++i) {
+            const float bi = a.lora_scale * half_bits_to_float(Bsrc[static_cast<size_t>(brow) * r + i]);
 #pragma unroll
-          for (int t = 0; t < 32; ++t) {
-            const int tt = c0 + t < tile.n ? c0 + t : tile.n - 1;
-            v[t] = fmaf(bi, ltr[tt * r + i], v[t]);
+            for (int t = 0; t < 32; ++t) {
+              const int tt = c0 + t < tile.n ? c0 + t : tile.n - 1;
+              v[t] = fmaf(bi, ltr[tt * r + i], v[t]);
+            }
+          }
+        }
+        if (swiglu) {
+          const int col = pair_pos(L >> 1);  // SwiGLU outputs in pair order (the down GEMM's token operand)
+          if (live) {
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+              const float partner = __shfl_xor_sync(0xffffffffu, v[t], 1);
+              if (!up && c0 + t < tile.n) {
+                const float hv = __fdividef(v[t], 1.0f + __expf(-v[t])) * partner;  // fp16 result: fast SiLU
+                range_bad |= !(fabsf(hv) <= kF16Max);
+                stage[(c0 + t) * 64 + col] = __half_as_ushort(__float2half_rn(hv));
+              }
+            }
+          }
+        } else {
+          const bool scaled = tile.e < a.E && a.row_scale;
+          if (live) {
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+              if (c0 + t < tile.n) {
+                const float xv = scaled ? v[t] * rsc[c0 + t] : v[t];
+                stage[(c0 + t) * 128 + L] = __half_as_ushort(__float2half_rn(xv));
+              }
+            }
           }
         }
       }
       if (swiglu) {
-        bool range_bad = false;  // a SwiGLU output fp16 cannot hold: MOE_ERR_RANGE
-        const int col = pair_pos(L >> 1);  // SwiGLU outputs in pair order (the down GEMM's token operand)
-        if (live) {
-#pragma unroll
-          for (int t = 0; t < 32; ++t) {
-            const float partner = __shfl_xor_sync(0xffffffffu, v[t], 1);
-            if (!up && c0 + t < tile.n) {
-              const float hv = __fdividef(v[t], 1.0f + __expf(-v[t])) * partner;  // fp16 result: fast SiLU suffices
-              range_bad |= !(fabsf(hv) <= kF16Max);
-              stage[(c0 + t) * 64 + col] = __half_as_ushort(__float2half_rn(hv));
-            }
-          }
-        }
         if (range_bad) report(a.err, 6);
         asm volatile("bar.sync 1, 256;" ::: "memory");
         for (int i = et; i < tile.n * 8; i += kEpi) {
@@ -504,16 +541,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
               reinterpret_cast<const uint4*>(stage + t * 64)[ch];
         }
       } else {
-        const bool scaled = tile.e < a.E && a.row_scale;
-        if (live) {
-#pragma unroll
-          for (int t = 0; t < 32; ++t) {
-            if (c0 + t < tile.n) {
-              const float xv = scaled ? v[t] * rsc[c0 + t] : v[t];
-              stage[(c0 + t) * 128 + L] = __half_as_ushort(__float2half_rn(xv));
-            }
-          }
-        }
         asm volatile("bar.sync 1, 256;" ::: "memory");
         for (int i = et; i < tile.n * 16; i += kEpi) {
           const int t = i >> 4, ch = i & 15;

@@ -300,7 +300,7 @@ GWs carve_gemm(void* base, int T, int K, int E, int H, int I, int r) {
 
 bool gemm_path(const moe_layer* L, int T, int K) {
   return static_cast<long long>(T) * K >= kGemmMinSlots && L->H % gg3::BM == 0 && (2 * L->I) % gg3::BM == 0 &&
-         L->I % (2 * gg3::BK) == 0;  // the dequantising warps take two K steps per pass
+         L->I % gg3::BK == 0;
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
