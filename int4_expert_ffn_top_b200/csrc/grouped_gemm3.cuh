@@ -93,8 +93,10 @@ constexpr int OFF_RAW = OFF_B + BSTAGES * B_STAGE;
 constexpr int LORA_T = 2 * BN * 32 * 4;  // epilogue staging of the tile's LoRA t vectors (two sets, r <= 32) ...
 constexpr int OFF_OUT = OFF_RAW + RSTAGES * RAW_STAGE;
 constexpr int OFF_LT = OFF_OUT + STAGE_OUT;
-constexpr int OFF_RS = OFF_LT + LORA_T;  // ... and of its gating weights
-constexpr int OFF_SB = OFF_RS + BN * 4;
+constexpr int OFF_RS = OFF_LT + LORA_T;  // ... of its gating weights ...
+constexpr int LORA_B = BM * 32 * 4;
+constexpr int OFF_BL = OFF_RS + BN * 4;  // ... and of its rows' LoRA B values times the LoRA scale, [i][row]
+constexpr int OFF_SB = OFF_BL + LORA_B;
 static_assert(ACC_COLS + APASS * RGROUPS * A_COLS <= static_cast<int>(TMEM_COLS) && BK == 64 && kDqWarps == 8,
               "tensor memory plan");
 
@@ -448,12 +450,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
     const int r = a.lora_r;
     float* lt = reinterpret_cast<float*>(sm + OFF_LT);   // [token][r] LoRA t vectors of the tile (two sets)
     float* rsc = reinterpret_cast<float*>(sm + OFF_RS);  // [token] gating weights of the tile
+    float* bls = reinterpret_cast<float*>(sm + OFF_BL);  // [i][row] LoRA B of the tile's rows, times the scale
     int it = 0;
 #pragma unroll 1
     for (int ti = blockIdx.x; ti < n_tiles && !fail; ti += gridDim.x, ++it) {
       const Tile tile = a.tiles[ti];
       const int ab = it & 1;
-      const int o = tile.mt * BM + L;
       // per-tile inputs of the epilogue, staged once while the accumulator is still being written
       const bool swiglu = a.epi == EPI_SWIGLU;
       const bool up = swiglu && (L & 1) != 0;
@@ -463,7 +465,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
       else
         Bsrc = tile.e < a.E ? (a.lora_Bex ? a.lora_Bex + static_cast<size_t>(tile.e) * a.out_ld * r : nullptr)
                             : a.lora_B1;
-      const int brow = swiglu ? (o >> 1) : o;
       const bool any_lora = swiglu ? tile.e == a.E && (a.lora_B1 || a.lora_B2)
                                    : (tile.e < a.E ? a.lora_Bex != nullptr : a.lora_B1 != nullptr);
       if (any_lora) {  // gate and up rows read different t arrays on SwiGLU tiles: even rows t1, odd rows t2
@@ -475,6 +476,16 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
       }
       if (!swiglu && tile.e < a.E && a.row_scale)
         for (int i = et; i < tile.n; i += kEpi) rsc[i] = a.row_scale[tile.row0 + i];
+      if (any_lora) {  // the rows' LoRA B values, read once per tile (consecutive threads: consecutive i of a row)
+        const uint16_t* Bdn = tile.e < a.E ? (a.lora_Bex ? a.lora_Bex + static_cast<size_t>(tile.e) * a.out_ld * r : nullptr)
+                                           : a.lora_B1;
+        for (int i = et; i < BM * r; i += kEpi) {
+          const int row = i / r, j = i - row * r, oo = tile.mt * BM + row;
+          const uint16_t* src = swiglu ? ((row & 1) ? a.lora_B2 : a.lora_B1) : Bdn;
+          bls[j * BM + row] =
+              src ? a.lora_scale * half_bits_to_float(src[static_cast<size_t>(swiglu ? oo >> 1 : oo) * r + j]) : 0.f;
+        }
+      }
       // the epilogue warps leave together (they meet at named barriers below)
       if (epi_any(!bar_wait(acc_full + ab, parity(it, 2), a.timeout_ns))) {
         fail = 1;
@@ -498,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
         if (live && Bsrc) {  // unmerged LoRA: + scale * B[row] . t[token]
 #pragma unroll 1
           for (int i = 0; i < r; ++i) {
-            const float bi = a.lora_scale * half_bits_to_float(Bsrc[static_cast<size_t>(brow) * r + i]);
+            const float bi = bls[i * BM + L];
 #pragma unroll
             for (int t = 0; t < 32; ++t) {
               const int tt = c0 + t < tile.n ? c0 + t : tile.n - 1;
