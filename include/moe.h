@@ -181,9 +181,9 @@ moe_status moe_route_topk(const moe_layer* L, const uint16_t* u, int32_t T, int3
  *   (slot t*K+k; stable, ascending slot id within an expert).
  * workspace: device scratch of at least moe_workspace_size(L, T, K) bytes,
  *   256-byte aligned; its contents on entry do not matter.
- * Paths (chosen by shape only): T*K < 128 slots run dequant-fused GEMVs on the
+ * Paths (chosen by shape only): T*K < 48 slots run dequant-fused GEMVs on the
  *   CUDA cores (fp32 accumulation of exact fp16 x int4-code products); T*K >=
- *   128 slots (with H and 2I multiples of 128) run grouped GEMMs on the tcgen05
+ *   48 slots (with H and 2I multiples of 128) run grouped GEMMs on the tcgen05
  *   tensor cores over per-expert token buckets, where the dequantised weights
  *   and the SwiGLU output are rounded to fp16 and products accumulate in fp32.
  * Bounded waits: every device-side wait of the tensor-core path gives up after

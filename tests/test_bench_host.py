@@ -111,7 +111,48 @@ def test_clock_sampler_names_the_visible_gpu(monkeypatch):
     assert bench.smi_gpu_id(0) == "4" and bench.smi_gpu_id(1) == "6"
     monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "GPU-0a1b, GPU-2c3d")
     assert bench.smi_gpu_id(1) == "GPU-2c3d"
-    assert bench.Clocks(0).gpu == "GPU-0a1b"
+
+
+def test_clock_sampler_reads_nvml_in_a_thread(monkeypatch):
+    """Read-only NVML queries (a fake here) every few ms plus one at each window edge: a window as short as
+    a 20-step run still has samples, and the throttle-reason bits map to their names."""
+    import sys
+    import time
+    import types
+
+    import torch
+
+    class FakeNvml(types.ModuleType):
+        NVML_CLOCK_SM = 1
+
+        def nvmlInit(self):
+            pass
+
+        def nvmlDeviceGetHandleByUUID(self, u):
+            assert u == "GPU-1234"
+            return "handle"
+
+        def nvmlDeviceGetMaxClockInfo(self, h, c):
+            return 1965
+
+        def nvmlDeviceGetClockInfo(self, h, c):
+            return 1800
+
+        def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+            return 0x4 | 0x1  # sw power cap, and an idle bit that is not a slowdown
+
+    monkeypatch.setitem(sys.modules, "pynvml", FakeNvml("pynvml"))
+    monkeypatch.setattr(torch.cuda, "get_device_properties", lambda d: types.SimpleNamespace(uuid="1234"))
+    clk = bench.Clocks(torch.device("cpu")).start()
+    t0 = time.time()
+    clk.edge()
+    time.sleep(0.002)
+    clk.edge()
+    t1 = time.time()
+    clk.stop()
+    s = clk.summary((t0, t1))
+    assert s["samples"] >= 2 and s["sm_mhz"] == 1800 and s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["sw_power_cap"] and s["source"] == "nvml"
 
 
 def test_headline_line_carries_every_contract_key():

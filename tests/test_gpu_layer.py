@@ -430,8 +430,14 @@ def test_expert_forward_max_shapes(cuda_ok, T):
 @pytest.mark.parametrize("T", [64, 200])
 @pytest.mark.parametrize("routed_lora", [False, True])
 def test_expert_forward_grouped_gemm_small(cuda_ok, T, routed_lora):
-    """T*K >= 128 slots take the tcgen05 grouped-GEMM path; same definition as the decode path."""
+    """T*K >= 48 slots take the tcgen05 grouped-GEMM path; same definition as the decode path."""
     _grouped_gemm_case(dataclasses.replace(CONFIGS[0], lora_routed_down=routed_lora), T)
+
+
+@pytest.mark.parametrize("T", [23, 24])  # 46 slots (GEMVs) and 48 slots (grouped GEMMs) at top-2
+def test_expert_forward_at_the_path_switch(cuda_ok, T):
+    """Both sides of the GEMV / grouped-GEMM switch give the oracle's output, bucket permutation included."""
+    _grouped_gemm_case(dataclasses.replace(CONFIGS[0], lora_routed_down=True), T)
 
 
 # (H, I): gate/up and down with different m-tile counts; K/64 above the pipeline depth of 4
