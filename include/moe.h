@@ -220,6 +220,59 @@ moe_status prerouter_predict(const moe_prerouter* head, const uint16_t* u, const
  * T < 0 or T > MOE_MAX_TOKENS. */
 size_t prerouter_workspace_size(const moe_prerouter* head, int32_t T);
 
+/*
+ * Tiered expert pool (p1 flow and p3 offload: experts sharded on SSD, only the
+ * active ones brought into RAM; p2 Prerouter and p3 Prerouter: the head's
+ * prediction lets the loads start early).  Here pinned host memory plays the
+ * SSD and HBM the RAM: a layer's routed expert blocks live in a host pool,
+ * and an HBM cache of n_slots blocks holds the ones in use.  A moe_tier is a
+ * host object (least-recently-used replacement; host-to-device copies with
+ * cudaMemcpyAsync).  One call of the expert forward over the cache:
+ *   moe_tier_acquire   makes the call's experts resident (copies of the missing
+ *                      ones on `stream`) and writes the call's expert ids
+ *                      remapped to slot ids (idx_slot, device);
+ *   moe_expert_forward with a layer view whose pool is the slot array
+ *                      (expert_stride = slot_stride, E = n_slots, no routed
+ *                      LoRA) and idx = idx_slot, on the same stream;
+ *   moe_tier_release   records that the slots' readers so far are enqueued.
+ * moe_tier_prefetch starts copies of predicted experts on a second stream (one
+ * copy stream per tier); they wait for the last release, never evict the last
+ * acquire's experts, and the next acquire waits for them.
+ * host_pool: pinned (page-locked or registered) host memory, n_experts blocks
+ *   host_stride bytes apart; block_bytes per expert; hbm_slots: device memory
+ *   of n_slots blocks, slot_stride bytes apart (>= block_bytes, a multiple of
+ *   256, 256-byte aligned); n_experts <= 256.  The caller owns both buffers
+ *   and keeps them alive until moe_tier_destroy.  Calls on one tier are
+ *   serialised by a lock.  Errors: MOE_ERR_INVALID_ARG for bad pointers or
+ *   sizes, MOE_ERR_WORKSPACE when one acquire asks for more distinct experts
+ *   than there are slots, MOE_ERR_CUDA when a copy or launch fails; an id in
+ *   idx whose expert was not acquired stores MOE_ERR_INVALID_ARG in err_word.
+ */
+typedef struct moe_tier moe_tier;
+
+typedef struct {
+  int64_t acquires;          /* moe_tier_acquire calls */
+  int64_t requested;         /* distinct experts asked for, summed over acquires */
+  int64_t hits;              /* ... already resident */
+  int64_t prefetch_hits;     /* ... of which a prefetch brought in */
+  int64_t misses;            /* ... copied by the acquire */
+  int64_t prefetched;        /* experts a prefetch copied */
+  int64_t bytes_acquired;    /* bytes copied by acquires */
+  int64_t bytes_prefetched;  /* bytes copied by prefetches */
+} moe_tier_stats;
+
+moe_status moe_tier_create(const void* host_pool, int64_t host_stride, int32_t n_experts, int64_t block_bytes,
+                           void* hbm_slots, int64_t slot_stride, int32_t n_slots, moe_tier** out);
+void moe_tier_destroy(moe_tier* tier);
+/* experts: host array of n_list expert ids (repeats allowed; the call's distinct experts); idx: device
+ * [n_idx] expert ids of the call; idx_slot: device [n_idx] output. */
+moe_status moe_tier_acquire(moe_tier* tier, const int32_t* experts, int32_t n_list, const int32_t* idx,
+                            int32_t n_idx, int32_t* idx_slot, int32_t* err_word, void* stream);
+moe_status moe_tier_release(moe_tier* tier, void* stream);
+/* experts: host array of n predicted expert ids; at most n_slots distinct ones are copied. */
+moe_status moe_tier_prefetch(moe_tier* tier, const int32_t* experts, int32_t n, void* copy_stream);
+moe_status moe_tier_get_stats(const moe_tier* tier, moe_tier_stats* out);
+
 /* Options of moe_stack_decode (NULL = all defaults). */
 typedef struct {
   int64_t timeout_ns;  /* bound on every device-side wait (single-launch kernel; per-layer grouped GEMMs);

@@ -9,10 +9,11 @@ from __future__ import annotations
 
 import ctypes
 
+import numpy as np
 import torch
 
 from . import _lib
-from .weights import DeviceHead, DeviceLayer, DeviceStack, block_bytes, block_stride, qrow_bytes  # noqa: F401
+from .weights import DeviceHead, DeviceLayer, DeviceStack, block_bytes, block_stride, host_pool, qrow_bytes  # noqa: F401
 
 OUT_F32, OUT_BF16, OUT_ADD_F32 = 0, 1, 2
 
@@ -175,6 +176,96 @@ def prerouter_predict(head: DeviceHead, u: torch.Tensor, sel: torch.Tensor, K_ne
     err = _arg(fn, "err_word", err_word, I32, 1, optional=True)
     _check(fn, lib().prerouter_predict(ctypes.byref(P), _p(u), args[0], T, K, *args[1:], *_ws(fn, workspace), err,
                                        _stream(stream)))
+
+
+class TieredPool:
+    """A layer's routed experts in pinned host memory behind an HBM cache of ``n_slots`` expert blocks
+    (``moe_tier_*``).  Its ``struct`` is the layer view that ``moe_expert_forward`` takes with slot ids (pass the
+    TieredPool as the layer): pool = the slot array, E = n_slots, no routed LoRA; ``moe_expert_forward`` reads
+    neither the router nor any expert outside the pool."""
+
+    def __init__(self, layer: DeviceLayer, host_blocks: torch.Tensor, n_slots: int, device=None):
+        fn = "moe_tier_create"
+        c = layer.cfg
+        if not isinstance(host_blocks, torch.Tensor) or host_blocks.dtype != torch.uint8 or \
+                host_blocks.dim() != 2 or host_blocks.shape[0] != c.E or not host_blocks.is_pinned():
+            raise ValueError(f"{fn}: host_blocks must be a pinned uint8 [E, stride] tensor")
+        if layer.struct.ex_lora_A:
+            raise ValueError(f"{fn}: routed LoRA is not served from a tiered pool")
+        self.layer, self.host = layer, host_blocks
+        self.stride = block_stride(c.H, c.I)
+        self.n_slots = n_slots
+        self.slots = torch.zeros(n_slots * self.stride, dtype=torch.uint8,
+                                 device=device if device is not None else layer.pool.device)
+        h = ctypes.c_void_p()
+        _check(fn, lib().moe_tier_create(host_blocks.data_ptr(), host_blocks.stride(0), c.E, block_bytes(c.H, c.I),
+                                         self.slots.data_ptr(), self.stride, n_slots, ctypes.byref(h)))
+        self.handle = h
+        v = _lib.moe_layer()
+        ctypes.memmove(ctypes.byref(v), ctypes.byref(layer.struct), ctypes.sizeof(v))
+        v.E = n_slots
+        v.router = _lib.moe_qrows(layer.struct.router.rows, n_slots, c.H, 8)
+        v.pool, v.expert_stride = self.slots.data_ptr(), self.stride
+        v.ex_lora_A = v.ex_lora_B = None
+        self.struct = v  # a TieredPool stands in for the layer in moe_expert_forward / moe_workspace_size
+
+    def acquire(self, experts, idx: torch.Tensor, idx_slot: torch.Tensor, err_word: torch.Tensor | None = None,
+                stream=None):
+        fn = "moe_tier_acquire"
+        ex = np.ascontiguousarray(np.asarray(experts, dtype=np.int32).reshape(-1))
+        n = idx.numel()
+        a = _arg(fn, "idx", idx, I32, n)
+        b = _arg(fn, "idx_slot", idx_slot, I32, n)
+        err = _arg(fn, "err_word", err_word, I32, 1, optional=True)
+        _check(fn, lib().moe_tier_acquire(self.handle, ex.ctypes.data, ex.size, a, n, b, err, _stream(stream)))
+
+    def release(self, stream=None):
+        _check("moe_tier_release", lib().moe_tier_release(self.handle, _stream(stream)))
+
+    def prefetch(self, experts, stream=None):
+        ex = np.ascontiguousarray(np.asarray(experts, dtype=np.int32).reshape(-1))
+        _check("moe_tier_prefetch", lib().moe_tier_prefetch(self.handle, ex.ctypes.data, ex.size, _stream(stream)))
+
+    def stats(self) -> dict:
+        st = _lib.moe_tier_stats()
+        _check("moe_tier_get_stats", lib().moe_tier_get_stats(self.handle, ctypes.byref(st)))
+        return {n: getattr(st, n) for n, _ in st._fields_}
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lib().moe_tier_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def moe_tier_create(layer: DeviceLayer, host_blocks: torch.Tensor, n_slots: int, device=None) -> TieredPool:
+    return TieredPool(layer, host_blocks, n_slots, device)
+
+
+def moe_tier_destroy(tier: TieredPool):
+    tier.close()
+
+
+def moe_tier_acquire(tier: TieredPool, experts, idx: torch.Tensor, idx_slot: torch.Tensor,
+                     err_word: torch.Tensor | None = None, stream=None):
+    tier.acquire(experts, idx, idx_slot, err_word, stream)
+
+
+def moe_tier_release(tier: TieredPool, stream=None):
+    tier.release(stream)
+
+
+def moe_tier_prefetch(tier: TieredPool, experts, stream=None):
+    tier.prefetch(experts, stream)
+
+
+def moe_tier_get_stats(tier: TieredPool) -> dict:
+    return tier.stats()
 
 
 class StackStructs:

@@ -34,6 +34,11 @@ class moe_prerouter(ctypes.Structure):
                 ("H", c_int32), ("E", c_int32), ("P", c_int32), ("E_next", c_int32)]
 
 
+class moe_tier_stats(ctypes.Structure):
+    _fields_ = [(n, c_int64) for n in ("acquires", "requested", "hits", "prefetch_hits", "misses", "prefetched",
+                                       "bytes_acquired", "bytes_prefetched")]
+
+
 # name -> (restype, argtypes); mirrors include/moe.h
 SIGNATURES = {
     "moe_status_string": (c_char_p, [c_int32]),
@@ -55,6 +60,12 @@ SIGNATURES = {
     "moe_expert_forward_noalloc": (c_int32, [POINTER(moe_layer), c_void_p, c_int32, c_int32, c_void_p, c_void_p,
                                              c_void_p, c_int32, c_void_p, c_void_p, c_void_p]),
     "moe_noalloc_scratch_bytes": (c_size_t, []),
+    "moe_tier_create": (c_int32, [c_void_p, c_int64, c_int32, c_int64, c_void_p, c_int64, c_int32, POINTER(c_void_p)]),
+    "moe_tier_destroy": (None, [c_void_p]),
+    "moe_tier_acquire": (c_int32, [c_void_p, c_void_p, c_int32, c_void_p, c_int32, c_void_p, c_void_p, c_void_p]),
+    "moe_tier_release": (c_int32, [c_void_p, c_void_p]),
+    "moe_tier_prefetch": (c_int32, [c_void_p, c_void_p, c_int32, c_void_p]),
+    "moe_tier_get_stats": (c_int32, [c_void_p, POINTER(moe_tier_stats)]),
     "moe_stack_grid": (c_int32, []),
     "moe_stack_workspace_size": (c_size_t, [POINTER(moe_layer), POINTER(moe_prerouter), c_int32, c_int32, c_int32,
                                             c_int32]),

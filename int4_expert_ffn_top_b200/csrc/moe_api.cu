@@ -12,6 +12,7 @@
 #include "prefill_kernels.cuh"
 #include "stack_kernel.cuh"
 #include "stack2_kernel.cuh"
+#include "tier.cuh"
 
 namespace {
 
@@ -1321,3 +1322,144 @@ moe_status moe_expert_forward_noalloc(const moe_layer* L, const uint16_t* u, int
 
 }  // extern "C"
 
+
+// ----------------------------------------------------------------------------- tiered expert pool
+struct moe_tier : moe::tier::Tier {};
+
+extern "C" {
+
+moe_status moe_tier_create(const void* host_pool, int64_t host_stride, int32_t n_experts, int64_t block_bytes,
+                           void* hbm_slots, int64_t slot_stride, int32_t n_slots, moe_tier** out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!host_pool || !hbm_slots || n_experts < 1 || n_experts > moe::tier::kMaxExperts || n_slots < 1 ||
+      block_bytes < 1 || host_stride < block_bytes || slot_stride < block_bytes || slot_stride % 256 != 0 ||
+      !aligned(hbm_slots, 256))
+    return MOE_ERR_INVALID_ARG;
+  cudaPointerAttributes ah{}, ad{};
+  if (cudaPointerGetAttributes(&ah, host_pool) != cudaSuccess || ah.type != cudaMemoryTypeHost ||
+      cudaPointerGetAttributes(&ad, hbm_slots) != cudaSuccess || ad.type != cudaMemoryTypeDevice) {
+    cudaGetLastError();
+    return MOE_ERR_INVALID_ARG;
+  }
+  moe_tier* t = new moe_tier();
+  t->host = static_cast<const uint8_t*>(host_pool);
+  t->host_stride = host_stride;
+  t->E = n_experts;
+  t->bytes = block_bytes;
+  t->slots = static_cast<uint8_t*>(hbm_slots);
+  t->slot_stride = slot_stride;
+  t->S = n_slots;
+  t->slot_of.assign(n_experts, -1);
+  t->expert_in.assign(n_slots, -1);
+  t->last_use.assign(n_slots, 0);
+  t->prefetched.assign(n_slots, 0);
+  if (cudaEventCreateWithFlags(&t->use_ev, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&t->pf_ev, cudaEventDisableTiming) != cudaSuccess) {
+    if (t->use_ev) cudaEventDestroy(t->use_ev);
+    delete t;
+    return MOE_ERR_CUDA;
+  }
+  *out = t;
+  return MOE_OK;
+}
+
+void moe_tier_destroy(moe_tier* t) {
+  if (!t) return;
+  cudaEventDestroy(t->use_ev);
+  cudaEventDestroy(t->pf_ev);
+  delete t;
+}
+
+moe_status moe_tier_acquire(moe_tier* t, const int32_t* experts, int32_t n_list, const int32_t* idx,
+                            int32_t n_idx, int32_t* idx_slot, int32_t* err_word, void* stream) {
+  if (!t || (n_list > 0 && !experts) || n_list < 0 || n_idx < 0 || (n_idx > 0 && (!idx || !idx_slot)))
+    return MOE_ERR_INVALID_ARG;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(t->mu);
+  const std::vector<int32_t> want = t->distinct(experts, n_list);
+  if (static_cast<int>(want.size()) > t->S) return MOE_ERR_WORKSPACE;
+  if (t->pf_pending) {  // the prefetched blocks are complete before anything later on this stream
+    if (cudaStreamWaitEvent(st, t->pf_ev, 0) != cudaSuccess) return MOE_ERR_CUDA;
+    t->pf_pending = false;
+  }
+  ++t->tick;
+  std::vector<int32_t> missing;
+  for (int e : want) {
+    const int s = t->slot_of[e];
+    if (s >= 0) {
+      ++t->st.hits;
+      if (t->prefetched[s]) ++t->st.prefetch_hits;
+      t->prefetched[s] = 0;
+      t->last_use[s] = t->tick;
+    } else {
+      missing.push_back(e);
+    }
+  }
+  t->acq_tick = t->tick;
+  for (int e : missing) {  // no slot wanted at this tick is reused: the call's experts stay resident
+    const int v = t->victim(t->tick);
+    if (v < 0) return MOE_ERR_WORKSPACE;
+    if (!t->place(e, v, st)) return MOE_ERR_CUDA;
+    t->prefetched[v] = 0;
+    ++t->st.misses;
+    t->st.bytes_acquired += t->bytes;
+  }
+  ++t->st.acquires;
+  t->st.requested += static_cast<int64_t>(want.size());
+  if (n_idx > 0) {
+    moe::tier::Table tab;
+    for (int e = 0; e < moe::tier::kMaxExperts; ++e) tab.slot[e] = e < t->E ? t->slot_of[e] : -1;
+    const int threads = 256, blocks = (n_idx + threads - 1) / threads;
+    moe::tier::remap_kernel<<<blocks < 1024 ? blocks : 1024, threads, 0, st>>>(idx, n_idx, tab, t->E, idx_slot,
+                                                                                 err_word);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+moe_status moe_tier_release(moe_tier* t, void* stream) {
+  if (!t) return MOE_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(t->mu);
+  if (cudaEventRecord(t->use_ev, static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  t->use_recorded = true;
+  return MOE_OK;
+}
+
+moe_status moe_tier_prefetch(moe_tier* t, const int32_t* experts, int32_t n, void* copy_stream) {
+  if (!t || n < 0 || (n > 0 && !experts)) return MOE_ERR_INVALID_ARG;
+  const cudaStream_t cs = static_cast<cudaStream_t>(copy_stream);
+  std::lock_guard<std::mutex> lock(t->mu);
+  std::vector<int32_t> want = t->distinct(experts, n);
+  if (static_cast<int>(want.size()) > t->S) want.resize(t->S);
+  // no copy may overwrite a slot before the kernels enqueued up to the last release have read it
+  if (t->use_recorded && cudaStreamWaitEvent(cs, t->use_ev, 0) != cudaSuccess) return MOE_ERR_CUDA;
+  ++t->tick;
+  for (int e : want)
+    if (t->slot_of[e] >= 0) t->last_use[t->slot_of[e]] = t->tick;
+  bool any = false;
+  for (int e : want) {
+    if (t->slot_of[e] >= 0) continue;
+    const int v = t->victim(t->acq_tick);  // the last acquire's experts are never evicted by a prefetch
+    if (v < 0) break;
+    if (!t->place(e, v, cs)) return MOE_ERR_CUDA;
+    t->prefetched[v] = 1;
+    ++t->st.prefetched;
+    t->st.bytes_prefetched += t->bytes;
+    any = true;
+  }
+  if (any || t->pf_pending) {
+    if (cudaEventRecord(t->pf_ev, cs) != cudaSuccess) return MOE_ERR_CUDA;
+    t->pf_pending = true;
+  }
+  return MOE_OK;
+}
+
+moe_status moe_tier_get_stats(const moe_tier* t, moe_tier_stats* out) {
+  if (!t || !out) return MOE_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(const_cast<moe_tier*>(t)->mu);
+  *out = t->st;
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -61,6 +61,18 @@ def _ptr(t: torch.Tensor | None) -> int | None:
     return None if t is None else t.data_ptr()
 
 
+def host_pool(cfg, experts: dict) -> torch.Tensor:
+    """The routed expert blocks of a layer in pinned host memory: uint8 ``[E, block_stride]``, expert ``e`` at
+    row ``e`` (experts missing from ``experts`` stay zero)."""
+    stride = block_stride(cfg.H, cfg.I)
+    pool = torch.zeros((cfg.E, stride), dtype=torch.uint8).pin_memory()
+    arr = pool.numpy()
+    for e, ex in experts.items():
+        b = expert_block(ex)
+        arr[e, :b.size] = b
+    return pool
+
+
 class DeviceLayer:
     """One layer's tensors on the device and its ``moe_layer`` struct.
 

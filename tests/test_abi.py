@@ -43,6 +43,25 @@ def test_python_binding_mirrors_the_header():
         assert hasattr(M, n), n
 
 
+def test_tier_host_side_rejections(lib):
+    """The tiered pool's entry points refuse null handles, pointers and bad sizes before any CUDA call."""
+    from int4_expert_ffn_top_b200 import _lib
+    h = ctypes.c_void_p()
+    bad = _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_tier_create(None, 4096, 16, 4096, None, 4096, 4, ctypes.byref(h)) == bad and not h.value
+    assert lib.moe_tier_create(1 << 20, 4096, 0, 4096, 1 << 21, 4096, 4, ctypes.byref(h)) == bad  # no experts
+    assert lib.moe_tier_create(1 << 20, 4096, 300, 4096, 1 << 21, 4096, 4, ctypes.byref(h)) == bad  # > 256
+    assert lib.moe_tier_create(1 << 20, 4096, 16, 4096, 1 << 21, 4000, 4, ctypes.byref(h)) == bad  # stride < block
+    assert lib.moe_tier_create(1 << 20, 4096, 16, 4096, (1 << 21) + 16, 4096, 4, ctypes.byref(h)) == bad  # align
+    assert lib.moe_tier_create(1 << 20, 4096, 16, 4096, 1 << 21, 4096, 4, None) == bad
+    assert lib.moe_tier_acquire(None, None, 0, None, 0, None, None, None) == bad
+    assert lib.moe_tier_release(None, None) == bad
+    assert lib.moe_tier_prefetch(None, None, 0, None) == bad
+    st = _lib.moe_tier_stats()
+    assert lib.moe_tier_get_stats(None, ctypes.byref(st)) == bad
+    lib.moe_tier_destroy(None)  # a null handle is ignored
+
+
 def test_status_strings(lib):
     from int4_expert_ffn_top_b200 import moe_status_string
     assert moe_status_string(0) == "ok"
