@@ -297,6 +297,103 @@ def batched_decode_leg(dev, M, steps: int = 20):
                          "scope": "whole step; bytes = experts touched (with their down LoRA) + per-layer fixed weights"}}
 
 
+def tiered_leg(dev, M, n_layers: int = 8, n_slots: int = 32, warm_tokens: int = 16, tokens: int = 48):
+    """35B-shaped batch-1 decode over the first n_layers layers (Zipf-offset router), each layer's routed experts
+    in pinned host memory behind an HBM cache of n_slots expert blocks (moe_tier_*): per-layer launches and one
+    host read of the routing per layer.  Four modes on the same tokens, each with fresh caches warmed by
+    warm_tokens tokens: every expert resident in HBM; tiered (copies on demand); tiered with Prerouter prefetch
+    (layer l's head predicts layer l+1's experts, copied on a side stream as soon as the prediction is read);
+    tiered with ideal prefetch (the next layer's true experts, recorded in the resident pass, issued when a
+    layer starts) -- the bound for a perfect predictor."""
+    import dataclasses
+    import torch
+    cfg = dataclasses.replace(CONFIGS[PREFILL_CFG_ID], T=1)
+    K, H = cfg.K, cfg.H
+    hosts = [inputs.layer(cfg, l) for l in range(n_layers)]
+    full = [M.DeviceLayer(cfg, h, device=dev) for h in hosts]
+    heads = [M.DeviceHead(cfg, h["prerouter"], device=dev) for h in hosts]
+    stride = M.block_stride(cfg.H, cfg.I)
+    lean = [M.DeviceLayer(cfg, dict(h, experts={}), device=dev, pool=torch.zeros(stride, dtype=torch.uint8, device=dev))
+            for h in hosts]
+    pools = [M.host_pool(cfg, h["experts"]) for h in hosts]
+    del hosts
+    n_tok = warm_tokens + tokens
+    xs = torch.from_numpy(np.stack([inputs.bf16_bits_to_f32(inputs.activations(cfg, step=5000 + i, T=1))
+                                    for i in range(n_tok)])).to(dev)
+    x = torch.empty((1, H), device=dev)
+    u = torch.empty((1, H), dtype=torch.int16, device=dev)
+    logits = torch.empty((1, cfg.E), device=dev)
+    idx = torch.empty((1, K), dtype=torch.int32, device=dev)
+    idx_slot = torch.empty_like(idx)
+    w = torch.empty((1, K), device=dev)
+    pred = torch.empty((1, K), dtype=torch.int32, device=dev)
+    scores = torch.empty((1, cfg.E_next), device=dev)
+    pws = M.workspace(M.prerouter_workspace_size(heads[0], 1), device=dev)
+    ws = M.workspace(M.moe_workspace_size(full[0], 1, K), device=dev)
+    side = torch.cuda.Stream(device=dev)
+    stream = torch.cuda.current_stream(dev)
+    recorded = np.zeros((n_tok, n_layers, K), np.int32)
+
+    def token(i, mode, tiers):
+        x.copy_(xs[i])
+        for l in range(n_layers):
+            if mode == "ideal" and l + 1 < n_layers:
+                tiers[l + 1].prefetch(recorded[i, l + 1], stream=side)
+            M.moe_rmsnorm_bf16(x, EPS, u)
+            M.moe_route_topk(full[l], u, K, logits, idx, w)
+            idx_h = idx.cpu().numpy()  # the host reads the routing (one sync per layer)
+            if mode == "resident":
+                recorded[i, l] = idx_h[0]
+                M.moe_expert_forward(full[l], u, K, idx, w, x, 2, ws)
+            else:
+                tiers[l].acquire(idx_h, idx, idx_slot)
+                M.moe_expert_forward(tiers[l], u, K, idx_slot, w, x, 2, tws)
+                tiers[l].release()
+            M.prerouter_predict(heads[l], u, idx, K, pred, scores, pws)
+            if mode == "prerouter" and l + 1 < n_layers:
+                tiers[l + 1].prefetch(pred.cpu().numpy(), stream=side)
+
+    out = {"workload": f"{cfg.name} shapes, batch-1 decode over the first {n_layers} layers (Zipf-offset router), "
+                       f"routed experts in pinned host memory behind {n_slots} HBM slots per layer "
+                       f"({n_slots / cfg.E:.0%} of the experts); per-layer launches, one host read of the routing "
+                       "per layer",
+           "n_slots": n_slots, "tokens": tokens, "warm_tokens": warm_tokens, "modes": {}}
+    tws = None
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    bb = M.block_bytes(cfg.H, cfg.I)
+    for mode in ("resident", "tiered", "prerouter", "ideal"):
+        tiers = None
+        if mode != "resident":
+            tiers = [M.TieredPool(lean[l], pools[l], n_slots) for l in range(n_layers)]
+            tws = M.workspace(M.moe_workspace_size(tiers[0], 1, K), device=dev)
+        for i in range(warm_tokens):
+            token(i, mode, tiers)
+        torch.cuda.synchronize(dev)
+        before = [t.stats() for t in tiers] if tiers else None
+
+        def timed():
+            e0.record(stream)
+            for i in range(warm_tokens, n_tok):
+                token(i, mode, tiers)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+
+        _, win = timed_window(timed)
+        ms = e0.elapsed_time(e1) / tokens
+        r = {"ms_per_token": ms, "value": 1000.0 / ms, "unit": "tok/s", "clocks": clock_summary(win)}
+        if tiers:
+            d = {k: sum(t.stats()[k] - b[k] for t, b in zip(tiers, before)) for k in before[0]}
+            r.update({"hit_rate": d["hits"] / max(d["requested"], 1),
+                      "prefetch_hit_rate": d["prefetch_hits"] / max(d["requested"], 1),
+                      "mb_copied_per_token": (d["bytes_acquired"] + d["bytes_prefetched"]) / tokens / 1e6,
+                      "mb_on_demand_per_token": d["bytes_acquired"] / tokens / 1e6,
+                      "experts_per_layer_call": d["requested"] / (tokens * n_layers), "block_bytes": bb})
+            for t in tiers:
+                t.close()
+        out["modes"][mode] = r
+    return out
+
+
 def launches_per_step(cfg, single: bool, predicted=False) -> int:
     if single:
         return 1  # the whole stack is one cooperative launch (plus two cudaMemsetAsync, not kernels)
@@ -896,10 +993,13 @@ def main():
         out["prefill"] = pre
     if not args.no_extra:
         for key, fn in (("decode_8b", lambda: decode_leg(dev, M, DECODE_8B_CFG_ID, steps=500)),
-                        ("batched_decode", lambda: batched_decode_leg(dev, M))):
+                        ("batched_decode", lambda: batched_decode_leg(dev, M)),
+                        ("tiered_pool", lambda: tiered_leg(dev, M))):
             try:
                 leg = fn()
                 ms_leg = leg.get("ms_per_token", leg.get("ms_per_step"))
+                if ms_leg is None:  # the tiered-pool leg: its on-demand mode's time
+                    ms_leg = leg["modes"]["tiered"]["ms_per_token"]
             except Exception as exc:  # a failing extra leg must not lose the headline line
                 leg, ms_leg = {"error": f"{type(exc).__name__}: {exc}"}, -1.0
             # every rank takes this collective, on the error path too
