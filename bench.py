@@ -304,7 +304,8 @@ def tiered_leg(dev, M, n_layers: int = 8, n_slots: int = 32, warm_tokens: int = 
     warm_tokens tokens: every expert resident in HBM; tiered (copies on demand); tiered with Prerouter prefetch
     (layer l's head predicts layer l+1's experts, copied on a side stream as soon as the prediction is read);
     tiered with ideal prefetch (the next layer's true experts, recorded in the resident pass, issued when a
-    layer starts) -- the bound for a perfect predictor."""
+    layer starts) -- the bound for a perfect predictor.  ``cold_ms_per_token`` times the warm-up tokens, the
+    first through empty caches."""
     import dataclasses
     import torch
     cfg = dataclasses.replace(CONFIGS[PREFILL_CFG_ID], T=1)
@@ -366,9 +367,13 @@ def tiered_leg(dev, M, n_layers: int = 8, n_slots: int = 32, warm_tokens: int = 
         if mode != "resident":
             tiers = [M.TieredPool(lean[l], pools[l], n_slots) for l in range(n_layers)]
             tws = M.workspace(M.moe_workspace_size(tiers[0], 1, K), device=dev)
-        for i in range(warm_tokens):
-            token(i, mode, tiers)
         torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for i in range(warm_tokens):  # cold: the first tokens through empty caches
+            token(i, mode, tiers)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_cold = e0.elapsed_time(e1) / warm_tokens
         before = [t.stats() for t in tiers] if tiers else None
 
         def timed():
@@ -380,7 +385,8 @@ def tiered_leg(dev, M, n_layers: int = 8, n_slots: int = 32, warm_tokens: int = 
 
         _, win = timed_window(timed)
         ms = e0.elapsed_time(e1) / tokens
-        r = {"ms_per_token": ms, "value": 1000.0 / ms, "unit": "tok/s", "clocks": clock_summary(win)}
+        r = {"ms_per_token": ms, "value": 1000.0 / ms, "unit": "tok/s", "clocks": clock_summary(win),
+             "cold_ms_per_token": ms_cold}
         if tiers:
             d = {k: sum(t.stats()[k] - b[k] for t, b in zip(tiers, before)) for k in before[0]}
             r.update({"hit_rate": d["hits"] / max(d["requested"], 1),
