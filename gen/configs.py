@@ -29,6 +29,7 @@ class MoEConfig:
     P: int            # Prerouter hidden width
     lora_shared: bool = True        # LoRA on every shared-expert projection
     lora_routed_down: bool = False  # LoRA on every routed expert's down projection
+    lora_routed_gate_up: bool = False  # LoRA on every routed expert's gate and up projections
     zipf_s: float = 0.0             # per-expert router logit offset exponent (0 = none)
     predicted_routing: bool = False  # layers >= 1 route by the previous head's prediction
 

@@ -43,6 +43,7 @@ TID = dict(
     sh_gu_q=5, sh_gu_s=6, sh_dn_q=7, sh_dn_s=8,
     sh_A_gate=9, sh_B_gate=10, sh_A_up=11, sh_B_up=12, sh_A_down=13, sh_B_down=14,
     ex_gu_q=20, ex_gu_s=21, ex_dn_q=22, ex_dn_s=23, ex_A_down=24, ex_B_down=25,
+    ex_A_gate=26, ex_B_gate=27, ex_A_up=28, ex_B_up=29,
     pre_W1=30, pre_b1=31, pre_W2=32, pre_b2=33,
     act=40,
 )
@@ -110,6 +111,9 @@ def expert(cfg: MoEConfig, layer: int, e: int, seed: int = 0) -> dict:
     )
     if cfg.lora_routed_down:
         d["down_lora"] = lora(cfg, layer, e, TID["ex_A_down"], TID["ex_B_down"], cfg.H, cfg.I, seed)
+    if cfg.lora_routed_gate_up:
+        d["gate_lora"] = lora(cfg, layer, e, TID["ex_A_gate"], TID["ex_B_gate"], cfg.I, cfg.H, seed)
+        d["up_lora"] = lora(cfg, layer, e, TID["ex_A_up"], TID["ex_B_up"], cfg.I, cfg.H, seed)
     return d
 
 

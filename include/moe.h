@@ -98,8 +98,14 @@ typedef struct {
  * LoRA (unmerged, 2kiu.com "Recover-LoRA" bullet): the delta on a projection
  * with input x is lora_scale * B (A x), added before the activation; A is
  * [r][in] fp16, B is [out][r] fp16.  Shared expert: index 0 gate, 1 up, 2 down;
- * a NULL A disables that projection's delta.  Routed experts (optional, down
- * projection only): ex_lora_A [E][r][I], ex_lora_B [E][H][r], or NULL.
+ * a NULL A disables that projection's delta.  Routed experts (optional):
+ * down projection ex_lora_A [E][r][I], ex_lora_B [E][H][r], or NULL; gate and
+ * up projections ex_lora_A_gu [E][2][r][H] (gate's A, then up's A) and
+ * ex_lora_B_gu [E][2I][r] in the expert block's interleaved row order (row 2j:
+ * gate row j, row 2j+1: up row j), or NULL.  With routed gate/up adapters
+ * moe_expert_forward takes its tensor-core path at every T (H and 2I
+ * multiples of 128, I of 64; else MOE_ERR_UNSUPPORTED), and moe_stack_decode
+ * its per-layer path.
  */
 typedef struct {
   int32_t H, E, I, I_s, r;
@@ -114,6 +120,8 @@ typedef struct {
   int64_t expert_stride;
   const uint16_t* ex_lora_A;
   const uint16_t* ex_lora_B;
+  const uint16_t* ex_lora_A_gu;
+  const uint16_t* ex_lora_B_gu;
 } moe_layer;
 
 /*

@@ -21,7 +21,8 @@ class moe_layer(ctypes.Structure):
                 ("router", moe_qrows), ("router_bias", c_void_p), ("shared_gate", moe_qrows),
                 ("shared_block", c_void_p),
                 ("sh_lora_A", c_void_p * 3), ("sh_lora_B", c_void_p * 3), ("lora_scale", c_float),
-                ("pool", c_void_p), ("expert_stride", c_int64), ("ex_lora_A", c_void_p), ("ex_lora_B", c_void_p)]
+                ("pool", c_void_p), ("expert_stride", c_int64), ("ex_lora_A", c_void_p), ("ex_lora_B", c_void_p),
+                ("ex_lora_A_gu", c_void_p), ("ex_lora_B_gu", c_void_p)]
 
 
 class moe_stack_opts(ctypes.Structure):

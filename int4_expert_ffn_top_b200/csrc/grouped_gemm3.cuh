@@ -122,6 +122,7 @@ struct Args {
   const uint16_t* lora_B2;
   const float* lora_t2;
   const uint16_t* lora_Bex;
+  const uint16_t* lora_Bgu_ex;  // SwiGLU, routed: per-expert B [E][2I][r] in the block's interleaved row order
   int lora_r;
   float lora_scale;
   int* err;
@@ -460,12 +461,14 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
       const bool swiglu = a.epi == EPI_SWIGLU;
       const bool up = swiglu && (L & 1) != 0;
       const uint16_t* Bsrc;
-      if (swiglu)
-        Bsrc = tile.e == a.E ? (up ? a.lora_B2 : a.lora_B1) : nullptr;  // LoRA on the shared expert's gate/up
+      const uint16_t* Bgu = tile.e < a.E && a.lora_Bgu_ex ? a.lora_Bgu_ex + static_cast<size_t>(tile.e) * 2 * a.out_ld * r
+                                                          : nullptr;  // SwiGLU: out_ld = I
+      if (swiglu)  // LoRA on the shared expert's gate/up, or on a routed expert's
+        Bsrc = tile.e == a.E ? (up ? a.lora_B2 : a.lora_B1) : Bgu;
       else
         Bsrc = tile.e < a.E ? (a.lora_Bex ? a.lora_Bex + static_cast<size_t>(tile.e) * a.out_ld * r : nullptr)
                             : a.lora_B1;
-      const bool any_lora = swiglu ? tile.e == a.E && (a.lora_B1 || a.lora_B2)
+      const bool any_lora = swiglu ? (tile.e == a.E ? (a.lora_B1 || a.lora_B2) : Bgu != nullptr)
                                    : (tile.e < a.E ? a.lora_Bex != nullptr : a.lora_B1 != nullptr);
       if (any_lora) {  // gate and up rows read different t arrays on SwiGLU tiles: even rows t1, odd rows t2
         const int tn = tile.n * r;
@@ -481,9 +484,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
                                            : a.lora_B1;
         for (int i = et; i < BM * r; i += kEpi) {
           const int row = i / r, j = i - row * r, oo = tile.mt * BM + row;
-          const uint16_t* src = swiglu ? ((row & 1) ? a.lora_B2 : a.lora_B1) : Bdn;
+          // shared gate/up: B per projection ([I][r], row oo / 2); routed gate/up: interleaved rows ([2I][r], row oo)
+          const bool per_proj = swiglu && tile.e == a.E;
+          const uint16_t* src = swiglu ? (per_proj ? ((row & 1) ? a.lora_B2 : a.lora_B1) : Bgu) : Bdn;
           bls[j * BM + row] =
-              src ? a.lora_scale * half_bits_to_float(src[static_cast<size_t>(swiglu ? oo >> 1 : oo) * r + j]) : 0.f;
+              src ? a.lora_scale * half_bits_to_float(src[static_cast<size_t>(per_proj ? oo >> 1 : oo) * r + j]) : 0.f;
         }
       }
       // the epilogue warps leave together (they meet at named barriers below)

@@ -59,8 +59,9 @@ moe_status check_expert_weights(const moe_layer* L) {
     for (int p = 0; p < 3; ++p)
       if ((L->sh_lora_A[p] != nullptr) != (L->sh_lora_B[p] != nullptr)) return MOE_ERR_INVALID_ARG;
     if ((L->ex_lora_A != nullptr) != (L->ex_lora_B != nullptr)) return MOE_ERR_INVALID_ARG;
-    const void* lp[8] = {L->sh_lora_A[0], L->sh_lora_A[1], L->sh_lora_A[2], L->ex_lora_A,
-                         L->sh_lora_B[0], L->sh_lora_B[1], L->sh_lora_B[2], L->ex_lora_B};
+    if ((L->ex_lora_A_gu != nullptr) != (L->ex_lora_B_gu != nullptr)) return MOE_ERR_INVALID_ARG;
+    const void* lp[10] = {L->sh_lora_A[0], L->sh_lora_A[1], L->sh_lora_A[2], L->ex_lora_A, L->ex_lora_A_gu,
+                          L->sh_lora_B[0], L->sh_lora_B[1], L->sh_lora_B[2], L->ex_lora_B, L->ex_lora_B_gu};
     for (const void* p : lp)
       if (p && !aligned(p, 16)) return MOE_ERR_INVALID_ARG;
   }
@@ -303,9 +304,13 @@ GWs carve_gemm(void* base, int T, int K, int E, int H, int I, int r) {
   return w;
 }
 
+bool gemm_shapes(const moe_layer* L) {
+  return L->H % gg3::BM == 0 && (2 * L->I) % gg3::BM == 0 && L->I % gg3::BK == 0;
+}
+
+// Routed gate/up adapters exist only on the tensor-core path, which serves any number of tokens.
 bool gemm_path(const moe_layer* L, int T, int K) {
-  return static_cast<long long>(T) * K >= kGemmMinSlots && L->H % gg3::BM == 0 && (2 * L->I) % gg3::BM == 0 &&
-         L->I % gg3::BK == 0;
+  return (static_cast<long long>(T) * K >= kGemmMinSlots || (L->r > 0 && L->ex_lora_A_gu)) && gemm_shapes(L);
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -492,6 +497,12 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
         u, T, TK, r, static_cast<const uint8_t*>(L->shared_gate.rows), lora ? L->sh_lora_A[0] : nullptr,
         lora ? L->sh_lora_A[1] : nullptr, ws.g, ws.t1, ws.t2);
   }
+  const bool ex_gu = r > 0 && L->ex_lora_A_gu;
+  if (ex_gu) {  // the routed gate/up adapters' A products on the permuted token rows
+    const long long warps = static_cast<long long>(TK) * 2 * r;
+    pf::lora_a_gu_rows_kernel<<<static_cast<unsigned>((warps + kWarps - 1) / kWarps), kThreads, 0, st>>>(
+        ws.X, H, TK, r, L->ex_lora_A_gu, ws.idx, ws.perm, ws.t1, ws.t2);
+  }
   const int RGU = qrow_bytes(H, 4), RDN = qrow_bytes(I, 4);
   const int64_t dn_off = static_cast<int64_t>(2 * I) * RGU;
   gg3::Maps m_gu, m_dn;
@@ -529,10 +540,13 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
     a.out_ld = I;
     if (lora) {
       a.lora_B1 = L->sh_lora_B[0];
-      a.lora_t1 = ws.t1;
       a.lora_B2 = L->sh_lora_B[1];
+    }
+    if (lora || ex_gu) {
+      a.lora_t1 = ws.t1;
       a.lora_t2 = ws.t2;
     }
+    a.lora_Bgu_ex = ex_gu ? L->ex_lora_B_gu : nullptr;
     gg3::grouped_gemm3_kernel<<<grid_gu, gg3::kThreads, smem_gu, st>>>(m_gu, a);
   }
   const bool ex = r > 0 && L->ex_lora_A;
@@ -567,6 +581,7 @@ moe_status expert_forward_h(const moe_layer* L, const uint16_t* u, int T, int K,
                             int drop_tile, cudaStream_t st) {
   if (gemm_path(L, T, K))
     return expert_forward_gemm<H>(L, u, T, K, idx, w, out, out_mode, perm_out, ws.base, err, timeout_ns, drop_tile, st);
+  if (L->r > 0 && L->ex_lora_A_gu) return MOE_ERR_UNSUPPORTED;
   switch (L->I) {
     case 128: return expert_forward_hi<H, 128>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, err, st);
     case 256: return expert_forward_hi<H, 256>(L, u, T, K, idx, w, out, out_mode, perm_out, ws, err, st);
@@ -784,7 +799,7 @@ Persist plan_persistent(const moe_layer* Ls, const moe_prerouter* Ps, int n, int
   if (lora && (r % 8 || r > 32)) return pl;
   for (int l = 0; l < n; ++l) {
     const moe_layer& L = Ls[l];
-    if (L.ex_lora_A) return pl;
+    if (L.ex_lora_A || L.ex_lora_A_gu) return pl;
     for (int q = 0; q < 3; ++q)
       if ((L.sh_lora_A[q] != nullptr) != lora || (L.sh_lora_B[q] != nullptr) != lora) return pl;
     if (!L.shared_block || !aligned(L.shared_block, 16) || !qrows_ok(L.shared_gate, 1, H, 8)) return pl;
@@ -950,7 +965,7 @@ Persist2 plan_persistent2(const moe_layer* Ls, const moe_prerouter* Ps, int n, i
   if (lora && (r % 8 || r > 32)) return pl;
   for (int l = 0; l < n; ++l) {
     const moe_layer& L = Ls[l];
-    if (L.ex_lora_A) return pl;
+    if (L.ex_lora_A || L.ex_lora_A_gu) return pl;
     for (int q = 0; q < 3; ++q)
       if ((L.sh_lora_A[q] != nullptr) != lora || (L.sh_lora_B[q] != nullptr) != lora) return pl;
     if (!L.shared_block || !aligned(L.shared_block, 16) || !qrows_ok(L.shared_gate, 1, H, 8)) return pl;

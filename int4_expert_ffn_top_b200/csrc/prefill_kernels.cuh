@@ -238,6 +238,33 @@ __global__ void __launch_bounds__(kThreads) lora_a_rows_kernel(const uint16_t* _
   if (lane == 0) t[static_cast<size_t>(row) * r + i] = acc;
 }
 
+// LoRA-A products of the routed experts' gate and up adapters on the permuted token rows (rows < TK):
+// t1[row][i] = A_gate[e][i] . x[row] and t2[row][i] = A_up[e][i] . x[row], e the row's expert.  One warp per
+// (row, j < 2r); x rows are fp16 in pair order, A rows in natural order ([E][2][r][H]: gate's, then up's).
+__global__ void __launch_bounds__(kThreads) lora_a_gu_rows_kernel(const uint16_t* __restrict__ X, int H, int TK, int r,
+                                                                  const uint16_t* __restrict__ A_gu,
+                                                                  const int32_t* __restrict__ idx,
+                                                                  const int32_t* __restrict__ perm,
+                                                                  float* __restrict__ t1, float* __restrict__ t2) {
+  const long long gw = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (gw >= static_cast<long long>(TK) * 2 * r) return;
+  const int row = static_cast<int>(gw / (2 * r)), j = static_cast<int>(gw % (2 * r));
+  const uint16_t* A = A_gu + (static_cast<size_t>(idx[perm[row]]) * 2 * r + j) * H;
+  const uint16_t* xr = X + static_cast<size_t>(row) * H;
+  float acc = 0.f;
+  for (int c = lane; c < H / 8; c += 32) {
+    const uint4 w = reinterpret_cast<const uint4*>(A)[c];
+    const uint4 xv = reinterpret_cast<const uint4*>(xr)[c];
+    acc = dot2_mix(prmt(w.x, w.z, 0x5410u), xv.x, acc);  // A chunk to pair order
+    acc = dot2_mix(prmt(w.x, w.z, 0x7632u), xv.y, acc);
+    acc = dot2_mix(prmt(w.y, w.w, 0x5410u), xv.z, acc);
+    acc = dot2_mix(prmt(w.y, w.w, 0x7632u), xv.w, acc);
+  }
+  acc = warp_reduce(acc);
+  if (lane == 0) (j < r ? t1 : t2)[static_cast<size_t>(row) * r + (j < r ? j : j - r)] = acc;
+}
+
 // out[t] (=, bf16, or +=) sum_k y[inv[t*K+k]] + g[t] * y[TK+t]; the routed rows of
 // y already carry their gating weight; k order fixed.
 __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ y, int T, int K, int H,

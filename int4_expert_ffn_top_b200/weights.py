@@ -111,6 +111,15 @@ class DeviceLayer:
         else:
             assert not ex_lora
             t["exA"] = t["exB"] = None
+        if getattr(cfg, "lora_routed_gate_up", False):
+            A = np.zeros((E, 2, r, H), np.float16)
+            B = np.zeros((E, 2 * I, r), np.float16)
+            for e, ex in host["experts"].items():
+                A[e, 0], A[e, 1] = ex["gate_lora"]["A"], ex["up_lora"]["A"]
+                B[e, 0::2], B[e, 1::2] = ex["gate_lora"]["B"], ex["up_lora"]["B"]  # the block's interleaved rows
+            t["exAgu"], t["exBgu"] = _dev(A, device), _dev(B, device)
+        else:
+            t["exAgu"] = t["exBgu"] = None
         self.struct = self._make_struct()
 
     def fill_experts(self, experts: dict):
@@ -146,6 +155,7 @@ class DeviceLayer:
         L.pool = self.pool.data_ptr()
         L.expert_stride = self.stride
         L.ex_lora_A, L.ex_lora_B = _ptr(t["exA"]), _ptr(t["exB"])
+        L.ex_lora_A_gu, L.ex_lora_B_gu = _ptr(t["exAgu"]), _ptr(t["exBgu"])
         return L
 
 

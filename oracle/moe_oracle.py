@@ -155,7 +155,7 @@ def routed_outputs(u: np.ndarray, experts: dict, idx: np.ndarray) -> np.ndarray:
     for e in np.unique(idx):
         ts, ks = np.nonzero(idx == e)
         ex = experts[int(e)]
-        y[ts, ks] = expert_ffn(u[ts], ex, lora_down=ex.get("down_lora"))
+        y[ts, ks] = expert_ffn(u[ts], ex, ex.get("gate_lora"), ex.get("up_lora"), ex.get("down_lora"))
     return y
 
 

@@ -100,3 +100,33 @@ def test_8b_shape_prefill_layer(cuda_ok):
     tau_p = prerouter_tau(u[toks], idx[toks], head, cfg.E, tc=True)
     assert np.all(np.abs(scores[toks] - ref_p) <= tau_p)
     check_topk(pred[toks], ref_p, tau_p, cfg.K)
+
+
+@pytest.mark.parametrize("T", [1, 4, 64])  # one token, below the 48-slot switch, above it: tensor cores throughout
+def test_lora_on_every_routed_projection(cuda_ok, T):
+    """LoRA on the gate, up and down projections of every routed expert (and of the shared expert)."""
+    cfg = dataclasses.replace(CONFIGS[0], lora_routed_down=True, lora_routed_gate_up=True)
+    lay = Layer(cfg, 0)
+    ub = inputs.activations(cfg, step=70 + T, T=T)
+    u = u_vals(ub)
+    _, idx, w = route(lay, ub, cfg.K)
+    out, _ = expert_forward(lay, ub, cfg.K, idx, w)
+    ref = oracle_out(lay, u, idx, w)
+    assert_close_inf(out, ref)
+    # the gate/up adapters matter: without them the oracle's output moves by several times the tolerance
+    bare = {e: {k: v for k, v in ex.items() if k not in ("gate_lora", "up_lora")} for e, ex in lay.host["experts"].items()}
+    ref_bare = O.combine(w, O.routed_outputs(u, bare, idx), O.shared_gate(u, lay.host["shared"]),
+                         O.shared_expert(u, lay.host["shared"]))
+    assert np.max(np.abs(ref - ref_bare)) > 3 * 2e-3 * np.max(np.abs(ref))
+
+
+def test_stack_with_lora_on_every_routed_projection(cuda_ok):
+    """moe_stack_decode over layers whose routed experts carry gate/up/down adapters (the per-layer path)."""
+    from test_gpu_layer import _check_stack, run_stack
+    cfg = dataclasses.replace(CONFIGS[0], layers=3, lora_routed_down=True, lora_routed_gate_up=True)
+    layer_fn = lambda l: inputs.layer(cfg, l)  # noqa: E731
+    stack = M().DeviceStack(cfg, layer_fn)
+    T = 1
+    x0 = inputs.bf16_bits_to_f32(inputs.activations(cfg, step=19, T=T)) * 3.0
+    res = run_stack(stack, cfg, T, x0, False)
+    _check_stack(cfg, layer_fn, T, res, x0, range(cfg.layers))

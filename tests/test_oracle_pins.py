@@ -357,6 +357,36 @@ def test_routed_down_lora_reaches_the_layer_output():
     assert np.count_nonzero(np.delete(dout, od, axis=1)) == 0
 
 
+def test_routed_gate_up_lora_reaches_the_slot_outputs():
+    """One-hot gate and up adapters on every routed expert: the gate adapter adds ``cg * u[ig]`` to gate output
+    ``jg`` and the up adapter ``cu * u[iu]`` to up output ``ju`` of every slot, before the SiLU, so each slot's
+    hidden values change at ``jg`` and ``ju`` only, by the closed form through ``silu(a) * b``."""
+    cfg = CONFIGS[0]
+    L = _tiny_layer(cfg)
+    u = O.round_bf16(inputs.bf16_bits_to_f32(inputs.activations(cfg)).astype(np.float64))
+    ig, jg, cg, iu, ju, cu = 5, 7, 0.75, 11, 19, -0.5
+    base = O.layer_forward(u, L, cfg.K)
+    for e in L["experts"]:
+        L["experts"][e]["gate_lora"] = _one_hot_lora(cfg.I, cfg.H, ig, jg, cg)
+        L["experts"][e]["up_lora"] = _one_hot_lora(cfg.I, cfg.H, iu, ju, cu)
+    r = O.layer_forward(u, L, cfg.K)
+    assert np.array_equal(r["idx"], base["idx"])
+    for t in range(cfg.T):
+        for k, e in enumerate(base["idx"][t]):
+            ex = L["experts"][int(e)]
+            Wgu = O.dequant(ex["gate_up"])
+            I = Wgu.shape[0] // 2
+            a = u[t] @ Wgu[:I].T
+            b = u[t] @ Wgu[I:].T
+            a2, b2 = a.copy(), b.copy()
+            a2[jg] += cg * u[t, ig]
+            b2[ju] += cu * u[t, iu]
+            h2 = O.silu(a2) * b2
+            assert np.allclose(r["y"][t, k], h2 @ O.dequant(ex["down"]).T, rtol=1e-11, atol=1e-12)
+            dh = h2 - O.silu(a) * b
+            assert np.count_nonzero(np.delete(dh, [jg, ju])) == 0 and dh[jg] != 0 and dh[ju] != 0
+
+
 def test_shared_gate_half_on_zero_weights():
     H = 128
     sh = dict(gate=zero_qmat(1, H, s=0.01 / 16, bits=8))
@@ -558,6 +588,14 @@ def test_planted_mistakes_are_caught(monkeypatch):
         "routed down LoRA dropped": lambda: monkeypatch.setattr(
             O, "routed_outputs", lambda u, experts, idx, _r=O.routed_outputs: _r(
                 u, {e: {k: v for k, v in ex.items() if k != "down_lora"} for e, ex in experts.items()}, idx)),
+        "routed gate/up adapters dropped": lambda: monkeypatch.setattr(
+            O, "routed_outputs", lambda u, experts, idx, _r=O.routed_outputs: _r(
+                u, {e: {k: v for k, v in ex.items() if k not in ("gate_lora", "up_lora")} for e, ex in experts.items()},
+                idx)),
+        "routed gate/up adapters swapped": lambda: monkeypatch.setattr(
+            O, "routed_outputs", lambda u, experts, idx, _r=O.routed_outputs: _r(
+                u, {e: dict(ex, **({"gate_lora": ex["up_lora"], "up_lora": ex["gate_lora"]} if "up_lora" in ex else {}))
+                    for e, ex in experts.items()}, idx)),
         "shared gate/up adapters swapped": lambda: monkeypatch.setattr(
             O, "shared_expert", lambda u, sh, _f=O.expert_ffn: _f(u, sh, sh.get("lora_up"), sh.get("lora_gate"),
                                                                   sh.get("lora_down"))),
@@ -571,7 +609,8 @@ def test_planted_mistakes_are_caught(monkeypatch):
             test_layer_with_zero_routed_experts_is_half_shared, test_layer_sparse_equals_dense_masked_mixture,
             test_prerouter_closed_forms, test_prerouter_reads_the_executed_experts_under_predicted_routing,
             test_buckets_brute_force_and_invariants, test_lora_on_every_projection_closed_form,
-            test_lora_unmerged_equals_merged_on_up_and_down, test_routed_down_lora_reaches_the_layer_output]
+            test_lora_unmerged_equals_merged_on_up_and_down, test_routed_down_lora_reaches_the_layer_output,
+            test_routed_gate_up_lora_reaches_the_slot_outputs]
     for name, plant in planted.items():
         plant()
         failed = False
