@@ -475,7 +475,9 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
                                void* out, int out_mode, int32_t* perm_out, void* workspace, int* err,
                                long long timeout_ns, int drop_tile, cudaStream_t st) {
   const int E = L->E, I = L->I, TK = T * K, R = TK + T;
-  const bool lora = L->r > 0 && L->sh_lora_A[0];
+  // the shared expert's adapters, each projection on its own
+  const bool lora_g = L->r > 0 && L->sh_lora_A[0], lora_u = L->r > 0 && L->sh_lora_A[1];
+  const bool lora_d = L->r > 0 && L->sh_lora_A[2], lora_gu = lora_g || lora_u;
   const int r = L->r > 0 ? L->r : 0;
   const GWs ws = carve_gemm(workspace, T, K, E, H, I, L->r);
   int* err_dev = err ? err : ws.err;  // without a caller's word, reports go to the workspace's own (unread) word
@@ -488,14 +490,16 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
                                               ws.tiles_dn, ws.n_tiles);
   // The GEMMs trust the device-built tile list: stop here if any launch so far failed.
   if (launch_status() != MOE_OK) return MOE_ERR_CUDA;
-  {
-    const int nrows = 1 + (lora ? 2 * r : 0);
-    const size_t smem = gemv_smem(H, false, true);
-    allow_smem(pf::lora_a_tokens_kernel<H / 8>, smem);
-    dim3 grid((T + TB - 1) / TB, (nrows + kWarps - 1) / kWarps);
-    pf::lora_a_tokens_kernel<H / 8><<<grid, kThreads, smem, st>>>(
-        u, T, TK, r, static_cast<const uint8_t*>(L->shared_gate.rows), lora ? L->sh_lora_A[0] : nullptr,
-        lora ? L->sh_lora_A[1] : nullptr, ws.g, ws.t1, ws.t2);
+  {  // the shared expert's gate and gate/up LoRA-A products, one pass over u
+    const int nt = lora_gu ? pf::shared_tokens_nt(r) : 0, smem = pf::shared_tokens_smem(H, nt);
+    auto kern = nt == 0 ? pf::shared_tokens_kernel<0>
+                        : (nt == 2 ? pf::shared_tokens_kernel<2> : (nt == 4 ? pf::shared_tokens_kernel<4>
+                                                                            : pf::shared_tokens_kernel<8>));
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    kern<<<(T + pf::kStTok - 1) / pf::kStTok, 32 * pf::kStWarps, smem, st>>>(
+        u, T, H, static_cast<const uint8_t*>(L->shared_gate.rows), ws.g, TK, r, lora_g ? L->sh_lora_A[0] : nullptr,
+        lora_u ? L->sh_lora_A[1] : nullptr, ws.t1, ws.t2);
   }
   const bool ex_gu = r > 0 && L->ex_lora_A_gu;
   if (ex_gu) {  // the routed gate/up adapters' A products on the permuted token rows
@@ -538,11 +542,9 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
     a.drop_tile = drop_tile;
     a.out = ws.Hh;
     a.out_ld = I;
-    if (lora) {
-      a.lora_B1 = L->sh_lora_B[0];
-      a.lora_B2 = L->sh_lora_B[1];
-    }
-    if (lora || ex_gu) {
+    a.lora_B1 = lora_g ? L->sh_lora_B[0] : nullptr;
+    a.lora_B2 = lora_u ? L->sh_lora_B[1] : nullptr;
+    if (lora_gu || ex_gu) {
       a.lora_t1 = ws.t1;
       a.lora_t2 = ws.t2;
     }
@@ -550,10 +552,10 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
     gg3::grouped_gemm3_kernel<<<grid_gu, gg3::kThreads, smem_gu, st>>>(m_gu, a);
   }
   const bool ex = r > 0 && L->ex_lora_A;
-  if (lora || ex) {  // LoRA A products on the SwiGLU output (shared down, routed down)
-    const int row_begin = ex ? 0 : TK, nrows = ex ? (lora ? R : TK) : T;
+  if (lora_d || ex) {  // LoRA A products on the SwiGLU output (shared down, routed down)
+    const int row_begin = ex ? 0 : TK, nrows = ex ? (lora_d ? R : TK) : T;
     pf::lora_a_rows_kernel<<<(nrows * r + kWarps - 1) / kWarps, kThreads, 0, st>>>(
-        ws.Hh, I, TK, nrows, row_begin, r, lora ? L->sh_lora_A[2] : nullptr, ex ? L->ex_lora_A : nullptr, ws.idx,
+        ws.Hh, I, TK, nrows, row_begin, r, lora_d ? L->sh_lora_A[2] : nullptr, ex ? L->ex_lora_A : nullptr, ws.idx,
         ws.perm, ws.t1);
   }
   {  // down (+ LoRA), routed rows scaled by their gating weight
@@ -566,7 +568,7 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
     a.out = ws.Y;
     a.out_ld = H;
     a.row_scale = ws.w_pos;
-    a.lora_B1 = lora ? L->sh_lora_B[2] : nullptr;
+    a.lora_B1 = lora_d ? L->sh_lora_B[2] : nullptr;
     a.lora_t1 = ws.t1;
     a.lora_Bex = ex ? L->ex_lora_B : nullptr;
     gg3::grouped_gemm3_kernel<<<grid_dn, gg3::kThreads, smem_dn, st>>>(m_dn, a);

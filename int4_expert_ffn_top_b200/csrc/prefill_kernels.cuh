@@ -29,39 +29,48 @@ __global__ void __launch_bounds__(kChunk) bucket_count_kernel(const int32_t* __r
 }
 
 // One block: expert offsets (exclusive scan of the totals) and, per block and
-// expert, the first sorted position of that block's slots (in place).
+// expert, the first sorted position of that block's slots (in place).  Thread e
+// owns expert e; the scan over experts is a warp-shuffle scan plus the warps'
+// totals, and each thread reads its column of the block histograms 8 blocks at
+// a time before writing them back.
 __global__ void __launch_bounds__(256) bucket_scan_kernel(int nblk, int E, int32_t* __restrict__ blockhist,
                                                           int32_t* __restrict__ count, int32_t* __restrict__ offset) {
-  __shared__ int tot[256];
-  __shared__ int off[257];
-  const int e = threadIdx.x;
+  __shared__ int wsum[8];
+  const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
+  int t = 0;
   if (e < E) {
-    int t = 0;
 #pragma unroll 8
     for (int b = 0; b < nblk; ++b) t += blockhist[static_cast<size_t>(b) * E + e];
-    tot[e] = t;
   }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int run = 0;
-    for (int i = 0; i < E; ++i) {
-      off[i] = run;
-      run += tot[i];
-    }
-    off[E] = run;
+  int incl = t;  // inclusive scan within the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
   }
+  if (lane == 31) wsum[warp] = incl;
   __syncthreads();
+  int excl = incl - t;
+  for (int w = 0; w < warp; ++w) excl += wsum[w];
   if (e < E) {
-    count[e] = tot[e];
-    offset[e] = off[e];
-    int run = off[e];
-    for (int b = 0; b < nblk; ++b) {
-      const int c = blockhist[static_cast<size_t>(b) * E + e];
-      blockhist[static_cast<size_t>(b) * E + e] = run;
-      run += c;
+    count[e] = t;
+    offset[e] = excl;
+    if (e == E - 1) offset[E] = excl + t;
+    int run = excl;
+#pragma unroll 1
+    for (int b0 = 0; b0 < nblk; b0 += 8) {
+      int c[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) c[i] = b0 + i < nblk ? blockhist[static_cast<size_t>(b0 + i) * E + e] : 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (b0 + i < nblk) {
+          blockhist[static_cast<size_t>(b0 + i) * E + e] = run;
+          run += c[i];
+        }
+      }
     }
   }
-  if (threadIdx.x == 0) offset[E] = off[E];
 }
 
 // Stable placement: the rank of a slot among equal experts of its block
@@ -160,52 +169,166 @@ __global__ void __launch_bounds__(128) tile_list_kernel(const int32_t* __restric
   }
 }
 
-// Shared-expert gate and LoRA-A products for many tokens: g[t], t1[TK+t][i] =
-// A_gate[i] . u_t, t2[TK+t][i] = A_up[i] . u_t.  grid (ceil(T / TB), row blocks).
-template <int NCH8>  // H / 8
-__global__ void __launch_bounds__(kThreads) lora_a_tokens_kernel(const uint16_t* __restrict__ u, int T, int TK, int r,
-                                                                 const uint8_t* __restrict__ sg_rec,
-                                                                 const uint16_t* __restrict__ A_gate,
-                                                                 const uint16_t* __restrict__ A_up, float* __restrict__ g,
-                                                                 float* __restrict__ t1, float* __restrict__ t2) {
-  // (the activation range is checked by permute_kernel, which reads every token)
-  constexpr int H = NCH8 * 8;
-  constexpr int SEG8 = (H / 16) < 32 ? (H / 16) : 32;
-  extern __shared__ uint4 smem[];
-  uint4* us = smem;
-  float* sum16 = reinterpret_cast<float*>(us + TB * (H / 8));
-  __shared__ int tok[TB];
-  const int t0 = blockIdx.x * TB, nt = min(TB, T - t0);
-  if (threadIdx.x < TB) tok[threadIdx.x] = t0 + min(static_cast<int>(threadIdx.x), nt - 1);
+// Shared expert's gate and LoRA-A products for many tokens, in one pass over u:
+//   g[t] = sigmoid(w . u_t), w the 8-bit gate row (affine groups of 64): per group s * sum (q - 128) u + (b + 128 s) * sum u;
+//   t1[TK + t][i] = A_gate[i] . u_t and t2[TK + t][i] = A_up[i] . u_t (a projection without adapter gets zeros).
+// A CTA takes 16 tokens and copies their rows of u into shared memory (16-byte asynchronous copies, all in flight
+// at once; rows padded by 64 bytes so that a warp's reads hit distinct banks).  Its 8 warps split the input
+// dimension into 32-wide chunks (warp w: chunks w, w + 8, ...), and the warps' partial sums are added in warp
+// order at the end.  The LoRA-A products run on tensor cores as tf32 m16n8k8 MMAs: bf16 u and fp16 A are exact in
+// tf32, so the products are exact and only the fp32 accumulation rounds.  Within a chunk, lane (g, q) supplies
+// inputs 8q + 2s and 8q + 2s + 1 as the MMA's k = q and k = q + 4 of step s, for both operands alike.
+constexpr int kStTok = 16, kStWarps = 8;
+inline int shared_tokens_nt(int r) { return r <= 0 ? 0 : (2 * r <= 16 ? 2 : (2 * r <= 32 ? 4 : 8)); }
+inline int shared_tokens_smem(int H, int nt) {
+  const int stage = kStTok * (2 * H + 64), red = kStWarps * kStTok * 8 * nt * 4;
+  return stage > red ? stage : red;
+}
+
+MOE_DEV void mma_tf32(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <int NT>  // 8-row tiles of the 2r LoRA rows (gate rows, then up rows); 0: the gate only
+__global__ void __launch_bounds__(256) shared_tokens_kernel(const uint16_t* __restrict__ u, int T, int H,
+                                                            const uint8_t* __restrict__ rec, float* __restrict__ g,
+                                                            int TK, int r, const uint16_t* __restrict__ A_gate,
+                                                            const uint16_t* __restrict__ A_up, float* __restrict__ t1,
+                                                            float* __restrict__ t2) {
+  constexpr int NTa = NT > 0 ? NT : 1, NC = 8 * NTa;
+  extern __shared__ __align__(16) uint8_t st_smem[];
+  __shared__ float gred[kStWarps][kStTok];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gi = lane >> 2, q = lane & 3;
+  const int t0 = blockIdx.x * kStTok, ld = 2 * H + 64;  // staged row stride in bytes
+  // stage the 16 token rows (rows past T are zeros)
+  const int n16 = H / 8;  // 16-byte pieces per row
+  for (int i = threadIdx.x; i < kStTok * n16; i += blockDim.x) {
+    const int row = i / n16, piece = i - row * n16;
+    uint8_t* dst = st_smem + row * ld + piece * 16;
+    if (t0 + row < T)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                   "l"(u + static_cast<size_t>(t0 + row) * H + piece * 8)
+                   : "memory");
+    else
+      *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  const uint16_t* sc = reinterpret_cast<const uint16_t*>(rec + H);
+  const uint16_t* arow[NTa];
+#pragma unroll
+  for (int n = 0; n < NTa; ++n) {
+    const int j = 8 * n + gi;
+    arow[n] = NT == 0 ? nullptr
+                      : (j < r ? (A_gate ? A_gate + static_cast<size_t>(j) * H : nullptr)
+                               : (j < 2 * r && A_up ? A_up + static_cast<size_t>(j - r) * H : nullptr));
+  }
+  // per-chunk global inputs: the gate codes and scales, the A fragments; fetched one chunk ahead
+  struct Pre {
+    uint2 qc;
+    uint16_t s, b;
+    uint4 a[NTa];
+  };
+  auto fetch = [&](int c, Pre& p) {
+    const int k = c * 32 + 8 * q;
+    p.qc = *reinterpret_cast<const uint2*>(rec + k);
+    p.s = sc[k >> 6];
+    p.b = sc[H / 64 + (k >> 6)];
+#pragma unroll
+    for (int n = 0; n < NTa; ++n)
+      p.a[n] = (NT > 0 && arow[n]) ? *reinterpret_cast<const uint4*>(arow[n] + k) : make_uint4(0, 0, 0, 0);
+  };
+  float acc[NTa][4];
+#pragma unroll
+  for (int n = 0; n < NTa; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+  float ga = 0.f, gb = 0.f;  // gate partials of tokens gi and gi + 8
+  const int nch = H / 32;
+  Pre cur, nxt;
+  if (warp < nch) fetch(warp, cur);
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
-  stage_tokens(u, H, tok, nt, us, nullptr, sum16, false, nullptr);
+#pragma unroll 1
+  for (int c = warp; c < nch; c += kStWarps) {
+    if (c + kStWarps < nch) fetch(c + kStWarps, nxt);
+    const int k = c * 32 + 8 * q;
+    const uint4 xa = *reinterpret_cast<const uint4*>(st_smem + gi * ld + 2 * k);
+    const uint4 xb = *reinterpret_cast<const uint4*>(st_smem + (gi + 8) * ld + 2 * k);
+    // u as fp32 bit patterns (bf16 << 16): element 2e is the low half of word e
+    const uint32_t wa[4] = {xa.x, xa.y, xa.z, xa.w}, wb[4] = {xb.x, xb.y, xb.z, xb.w};
+    uint32_t ua[8], ub[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      ua[2 * e] = wa[e] << 16;
+      ua[2 * e + 1] = wa[e] & 0xFFFF0000u;
+      ub[2 * e] = wb[e] << 16;
+      ub[2 * e + 1] = wb[e] & 0xFFFF0000u;
+    }
+    {  // gate
+      float da = 0.f, sa = 0.f, db = 0.f, sb = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t w = i < 4 ? cur.qc.x : cur.qc.y;
+        const float qv = static_cast<float>(static_cast<int>((w >> (8 * (i & 3))) & 0xFFu) - 128);
+        const float x = __uint_as_float(ua[i]), y = __uint_as_float(ub[i]);
+        da = fmaf(qv, x, da);
+        sa += x;
+        db = fmaf(qv, y, db);
+        sb += y;
+      }
+      const float s = half_bits_to_float(cur.s), bb = fmaf(128.f, s, half_bits_to_float(cur.b));
+      ga += fmaf(s, da, bb * sa);
+      gb += fmaf(s, db, bb * sb);
+    }
+    if (NT > 0) {
+#pragma unroll
+      for (int n = 0; n < NTa; ++n) {
+        const uint32_t aw[4] = {cur.a[n].x, cur.a[n].y, cur.a[n].z, cur.a[n].w};
+#pragma unroll
+        for (int st = 0; st < 4; ++st) {
+          const float2 f = __half22float2(as_h2(aw[st]));
+          mma_tf32(acc[n], ua[2 * st], ub[2 * st], ua[2 * st + 1], ub[2 * st + 1], __float_as_uint(f.x),
+                   __float_as_uint(f.y));
+        }
+      }
+    }
+    cur = nxt;
+  }
+  ga += __shfl_xor_sync(0xFFFFFFFFu, ga, 1);
+  ga += __shfl_xor_sync(0xFFFFFFFFu, ga, 2);
+  gb += __shfl_xor_sync(0xFFFFFFFFu, gb, 1);
+  gb += __shfl_xor_sync(0xFFFFFFFFu, gb, 2);
+  __syncthreads();  // the staged rows are read: the area now holds the warps' partial products
+  float* red = reinterpret_cast<float*>(st_smem);  // [warp][token][NC]
+  if (q == 0) {
+    gred[warp][gi] = ga;
+    gred[warp][gi + 8] = gb;
+  }
+  if (NT > 0) {
+#pragma unroll
+    for (int n = 0; n < NTa; ++n) {
+      float* p = red + (warp * kStTok + gi) * NC + 8 * n + 2 * q;
+      p[0] = acc[n][0];
+      p[1] = acc[n][1];
+      p[8 * NC] = acc[n][2];
+      p[8 * NC + 1] = acc[n][3];
+    }
+  }
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.y * kWarps + warp;  // 0: shared gate; 1..r: A_gate; r+1..2r: A_up
-  const int nrows = 1 + (A_gate ? r : 0) + (A_up ? r : 0);
-  if (row >= nrows) return;
-  float acc[TB];
+  if (threadIdx.x < kStTok && t0 + threadIdx.x < T) {
+    float z = 0.f;
 #pragma unroll
-  for (int t = 0; t < TB; ++t) acc[t] = 0.f;
-  if (row == 0) {
-    const uint16_t* sc = reinterpret_cast<const uint16_t*>(sg_rec + H);
-    row_int8<H / 16, SEG8>(reinterpret_cast<const uint32_t*>(sg_rec), sc, sc + H / 64, us, sum16, nt, lane % SEG8, acc);
+    for (int w = 0; w < kStWarps; ++w) z += gred[w][threadIdx.x];
+    g[t0 + threadIdx.x] = sigmoid(z);
+  }
+  if (NT > 0) {
+    for (int i = threadIdx.x; i < kStTok * NC; i += blockDim.x) {
+      const int tok = i / NC, j = i - tok * NC, t = t0 + tok;
+      if (t >= T || j >= 2 * r) continue;
+      float z = 0.f;
 #pragma unroll
-    for (int t = 0; t < TB; ++t) acc[t] = seg_reduce<SEG8>(acc[t]);
-    if (lane == 0)
-      for (int t = 0; t < nt; ++t) g[t0 + t] = sigmoid(acc[t]);
-  } else {
-    constexpr int SEG = NCH8 < 32 ? NCH8 : 32;
-    const int i = row - 1;
-    const bool is_gate = A_gate && i < r;
-    const int ri = is_gate ? i : (A_gate ? i - r : i);
-    const uint16_t* A = is_gate ? A_gate : A_up;
-    if (lane < SEG) row_f16<NCH8, SEG>(A + static_cast<size_t>(ri) * H, us, H / 8, nt, lane, acc);
-#pragma unroll
-    for (int t = 0; t < TB; ++t) acc[t] = seg_reduce<32>(acc[t]);
-    if (lane == 0) {
-      float* dst = is_gate ? t1 : t2;
-      for (int t = 0; t < nt; ++t) dst[static_cast<size_t>(TK + t0 + t) * r + ri] = acc[t];
+      for (int w = 0; w < kStWarps; ++w) z += red[(w * kStTok + tok) * NC + j];
+      (j < r ? t1 : t2)[static_cast<size_t>(TK + t) * r + (j < r ? j : j - r)] = z;
     }
   }
 }

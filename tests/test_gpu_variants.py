@@ -130,3 +130,34 @@ def test_stack_with_lora_on_every_routed_projection(cuda_ok):
     x0 = inputs.bf16_bits_to_f32(inputs.activations(cfg, step=19, T=T)) * 3.0
     res = run_stack(stack, cfg, T, x0, False)
     _check_stack(cfg, layer_fn, T, res, x0, range(cfg.layers))
+
+
+@pytest.mark.parametrize("T", [4, 64])  # GEMV path and grouped-GEMM path
+def test_shared_adapter_on_some_projections_only(cuda_ok, T):
+    """A shared-expert adapter on the up and down projections but not the gate: each projection is taken on its
+    own, and the gate's zero LoRA-A rows leave its products untouched."""
+    cfg = CONFIGS[0]
+    lay = Layer(cfg, 0)
+    from int4_expert_ffn_top_b200 import _lib
+    s = _lib.moe_layer()
+    ctypes.memmove(ctypes.byref(s), ctypes.byref(lay.dev.struct), ctypes.sizeof(s))
+    s.sh_lora_A[0] = s.sh_lora_B[0] = None
+
+    class View:
+        struct = s
+
+    sh = {k: v for k, v in lay.host["shared"].items() if k != "lora_gate"}
+    assert "lora_up" in sh and "lora_down" in sh
+    ub = inputs.activations(cfg, step=80 + T, T=T)
+    u = u_vals(ub)
+    _, idx, w = route(lay, ub, cfg.K)
+    m = M()
+    out = torch.full((T, cfg.H), float("nan"), device=DEV)
+    m.moe_expert_forward(View, torch.from_numpy(ub.view(np.int16)).to(DEV), cfg.K,
+                         torch.from_numpy(idx.astype(np.int32)).to(DEV), torch.from_numpy(w.astype(np.float32)).to(DEV),
+                         out, 0, m.workspace(m.moe_workspace_size(View, T, cfg.K)))
+    torch.cuda.synchronize()
+    ref = O.combine(w, O.routed_outputs(u, lay.host["experts"], idx), O.shared_gate(u, sh), O.shared_expert(u, sh))
+    assert_close_inf(out.cpu().numpy().astype(np.float64), ref)
+    full = oracle_out(lay, u, idx, w)  # the gate's adapter matters here
+    assert np.max(np.abs(full - ref)) > 3 * 2e-3 * np.max(np.abs(ref))
