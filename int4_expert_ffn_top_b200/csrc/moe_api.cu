@@ -485,7 +485,7 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
   pf::bucket_count_kernel<<<ws.nblk, pf::kChunk, 0, st>>>(idx, TK, E, ws.idx, ws.blockhist);
   pf::bucket_scan_kernel<<<1, 256, 0, st>>>(ws.nblk, E, ws.blockhist, ws.count, ws.offset);
   pf::bucket_place_kernel<<<ws.nblk, pf::kChunk, 0, st>>>(ws.idx, TK, E, ws.blockhist, ws.perm, ws.inv, perm_out);
-  pf::permute_kernel<<<R, 256, 0, st>>>(u, T, K, H, ws.perm, w, ws.X, ws.w_pos, err_dev);
+  pf::permute_kernel<H><<<(R + 7) / 8, 256, 0, st>>>(u, T, K, ws.perm, w, ws.X, ws.w_pos, err_dev);
   pf::tile_list_kernel<<<E + 1, 128, 0, st>>>(ws.count, ws.offset, E, T, K, 2 * I / gg3::BM, H / gg3::BM, ws.tiles_gu,
                                               ws.tiles_dn, ws.n_tiles);
   // The GEMMs trust the device-built tile list: stop here if any launch so far failed.
@@ -573,7 +573,7 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
     a.lora_Bex = ex ? L->ex_lora_B : nullptr;
     gg3::grouped_gemm3_kernel<<<grid_dn, gg3::kThreads, smem_dn, st>>>(m_dn, a);
   }
-  pf::combine_kernel<<<T, 256, 0, st>>>(ws.Y, T, K, H, ws.inv, ws.g, out, out_mode);
+  pf::combine_kernel<H><<<T, 256, 0, st>>>(ws.Y, T, K, ws.inv, ws.g, out, out_mode);
   return launch_status();
 }
 

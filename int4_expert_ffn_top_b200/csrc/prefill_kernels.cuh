@@ -104,37 +104,45 @@ __global__ void __launch_bounds__(kChunk) bucket_place_kernel(const int32_t* __r
 // order (u_j, u_{j+4}), j = 0..3, the K order of the dequantised weight tiles.
 // Activations fp16 cannot hold (|u| > 65504 or not finite) report MOE_ERR_RANGE
 // into err (checked on the shared-expert rows, which hold every token once).
-__global__ void __launch_bounds__(256) permute_kernel(const uint16_t* __restrict__ u, int T, int K, int H,
+// One warp per row, 8 rows per CTA; a lane's H / 256 16-byte loads are all issued before its stores.
+template <int H>
+__global__ void __launch_bounds__(256) permute_kernel(const uint16_t* __restrict__ u, int T, int K,
                                                       const int32_t* __restrict__ perm, const float* __restrict__ w,
                                                       uint16_t* __restrict__ X, float* __restrict__ w_pos, int* err) {
-  const int row = blockIdx.x;
+  constexpr int NV = H / 256;
+  const int lane = threadIdx.x & 31, row = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int TK = T * K;
+  if (row >= TK + T) return;  // whole warps
   int tok;
   if (row < TK) {
     const int slot = perm[row];
     tok = slot / K;
-    if (threadIdx.x == 0) w_pos[row] = w[slot];
+    if (lane == 0) w_pos[row] = w[slot];
   } else {
     tok = row - TK;
   }
   const uint4* src = reinterpret_cast<const uint4*>(u + static_cast<size_t>(tok) * H);
   uint4* dst = reinterpret_cast<uint4*>(X + static_cast<size_t>(row) * H);
+  uint4 v[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) v[i] = src[lane + 32 * i];
   bool bad = false;
-  for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
-    const uint4 v = src[c];
-    const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const uint32_t vw[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
     uint16_t e[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint16_t lo = static_cast<uint16_t>(vw[i] & 0xffffu), hi = static_cast<uint16_t>(vw[i] >> 16);
+    for (int j = 0; j < 4; ++j) {
+      const uint16_t lo = static_cast<uint16_t>(vw[j] & 0xffffu), hi = static_cast<uint16_t>(vw[j] >> 16);
       bad |= !(fabsf(bf16_bits_to_float(lo)) <= kF16Max) || !(fabsf(bf16_bits_to_float(hi)) <= kF16Max);
-      e[2 * i] = bf16_to_f16_bits(lo);
-      e[2 * i + 1] = bf16_to_f16_bits(hi);
+      e[2 * j] = bf16_to_f16_bits(lo);
+      e[2 * j + 1] = bf16_to_f16_bits(hi);
     }
-    dst[c] = make_uint4(e[0] | (static_cast<uint32_t>(e[4]) << 16), e[1] | (static_cast<uint32_t>(e[5]) << 16),
-                        e[2] | (static_cast<uint32_t>(e[6]) << 16), e[3] | (static_cast<uint32_t>(e[7]) << 16));
+    dst[lane + 32 * i] =
+        make_uint4(e[0] | (static_cast<uint32_t>(e[4]) << 16), e[1] | (static_cast<uint32_t>(e[5]) << 16),
+                   e[2] | (static_cast<uint32_t>(e[6]) << 16), e[3] | (static_cast<uint32_t>(e[7]) << 16));
   }
-  if (bad && row >= TK) report(err, 6);
+  if (row >= TK && __any_sync(0xFFFFFFFFu, bad) && lane == 0) report(err, 6);
 }
 
 // Tile lists of both GEMMs: per expert (then the shared expert) its token
@@ -390,18 +398,33 @@ __global__ void __launch_bounds__(kThreads) lora_a_gu_rows_kernel(const uint16_t
 
 // out[t] (=, bf16, or +=) sum_k y[inv[t*K+k]] + g[t] * y[TK+t]; the routed rows of
 // y already carry their gating weight; k order fixed.
-__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ y, int T, int K, int H,
+// A thread's K + 1 row loads are all issued before the sum (row ids read once per token); the stores are
+// 16-byte vectors when out is 16-byte aligned.
+template <int H>
+__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ y, int T, int K,
                                                       const int32_t* __restrict__ inv, const float* __restrict__ g,
                                                       void* __restrict__ out, int out_mode) {
+  constexpr int kMaxK = 8;
   const int t = blockIdx.x;
   const int TK = T * K;
+  int rows[kMaxK];
+#pragma unroll
+  for (int k = 0; k < kMaxK; ++k) rows[k] = k < K ? inv[t * K + k] : 0;
+  const float gt = g[t];
+  const bool vec = (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
   for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
+    uint4 v[kMaxK + 1];
+#pragma unroll
+    for (int k = 0; k < kMaxK; ++k)
+      if (k < K) v[k] = reinterpret_cast<const uint4*>(y + static_cast<size_t>(rows[k]) * H)[c];
+    v[kMaxK] = reinterpret_cast<const uint4*>(y + static_cast<size_t>(TK + t) * H)[c];
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    for (int k = 0; k < K; ++k) {
-      const uint4 v = reinterpret_cast<const uint4*>(y + static_cast<size_t>(inv[t * K + k]) * H)[c];
-      const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < kMaxK; ++k) {
+      if (k >= K) break;
+      const uint32_t vw[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float2 f = __half22float2(as_h2(vw[i]));
@@ -409,24 +432,45 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
         acc[2 * i + 1] += f.y;
       }
     }
-    const float gt = g[t];
-    const uint4 v = reinterpret_cast<const uint4*>(y + static_cast<size_t>(TK + t) * H)[c];
-    const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+    {
+      const uint32_t vw[4] = {v[kMaxK].x, v[kMaxK].y, v[kMaxK].z, v[kMaxK].w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __half22float2(as_h2(vw[i]));
-      acc[2 * i] = fmaf(gt, f.x, acc[2 * i]);
-      acc[2 * i + 1] = fmaf(gt, f.y, acc[2 * i + 1]);
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(as_h2(vw[i]));
+        acc[2 * i] = fmaf(gt, f.x, acc[2 * i]);
+        acc[2 * i + 1] = fmaf(gt, f.y, acc[2 * i + 1]);
+      }
     }
     const size_t o = static_cast<size_t>(t) * H + c * 8;
     if (out_mode == 1) {
       uint16_t* ob = reinterpret_cast<uint16_t*>(out) + o;
+      uint16_t b[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) ob[i] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[i]));
+      for (int i = 0; i < 8; ++i) b[i] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[i]));
+      if (vec) {
+        *reinterpret_cast<uint4*>(ob) =
+            make_uint4(b[0] | (static_cast<uint32_t>(b[1]) << 16), b[2] | (static_cast<uint32_t>(b[3]) << 16),
+                       b[4] | (static_cast<uint32_t>(b[5]) << 16), b[6] | (static_cast<uint32_t>(b[7]) << 16));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ob[i] = b[i];
+      }
     } else {
       float* of = reinterpret_cast<float*>(out) + o;
+      if (vec) {
+        float4* o4 = reinterpret_cast<float4*>(of);
+        float4 x0 = make_float4(acc[0], acc[1], acc[2], acc[3]), x1 = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        if (out_mode == 2) {
+          const float4 p0 = o4[0], p1 = o4[1];
+          x0 = make_float4(p0.x + x0.x, p0.y + x0.y, p0.z + x0.z, p0.w + x0.w);
+          x1 = make_float4(p1.x + x1.x, p1.y + x1.y, p1.z + x1.z, p1.w + x1.w);
+        }
+        o4[0] = x0;
+        o4[1] = x1;
+      } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) of[i] = out_mode == 2 ? of[i] + acc[i] : acc[i];
+        for (int i = 0; i < 8; ++i) of[i] = out_mode == 2 ? of[i] + acc[i] : acc[i];
+      }
     }
   }
 }

@@ -50,15 +50,17 @@ def route(layer: Layer, u_bits: np.ndarray, K: int):
     return logits.cpu().numpy().astype(np.float64), idx.cpu().numpy(), w.cpu().numpy().astype(np.float64)
 
 
-def expert_forward(layer: Layer, u_bits, K, idx, w, mode=0, x0=None, perm=False):
+def expert_forward(layer: Layer, u_bits, K, idx, w, mode=0, x0=None, perm=False, offset=0):
+    """offset > 0 places out that many elements into a larger buffer (an output not 16-byte aligned)."""
     m = M()
     T, H = u_bits.shape[0], layer.cfg.H
     if mode == 1:
-        out = torch.zeros((T, H), dtype=torch.int16, device=DEV)
+        out = torch.zeros(T * H + offset, dtype=torch.int16, device=DEV)[offset:].view(T, H)
     elif mode == 2:
-        out = torch.from_numpy(x0.astype(np.float32)).to(DEV)
+        out = torch.empty(T * H + offset, device=DEV)[offset:].view(T, H)
+        out.copy_(torch.from_numpy(x0.astype(np.float32)))
     else:
-        out = torch.full((T, H), float("nan"), device=DEV)
+        out = torch.full((T * H + offset,), float("nan"), device=DEV)[offset:].view(T, H)
     ws = m.workspace(m.moe_workspace_size(layer.dev, T, K))
     ws.fill_(0xA5)  # contents on entry must not matter
     perm_out = torch.full((T * K,), -1, dtype=torch.int32, device=DEV) if perm else None
@@ -161,6 +163,29 @@ def test_expert_forward_c0(c0, T, mode):
     w = O.gating(ref_logits, idx)
     x0 = np.random.default_rng(T).standard_normal((T, cfg.H)) * 4 if mode == 2 else None
     out, _ = expert_forward(c0, ub, cfg.K, idx, w, mode=mode, x0=x0)
+    ref = oracle_out(c0, u, idx, w)
+    if mode == 2:
+        out = out - x0.astype(np.float32)
+    if mode == 1:
+        half_ulp = np.abs(O.round_bf16(ref) - ref)
+        assert np.all(np.abs(out - ref) <= 2e-3 * np.abs(ref).max() + half_ulp + 1e-30)
+    else:
+        assert_close_inf(out, ref)
+
+
+@pytest.mark.parametrize("offset", [0, 1])
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_expert_forward_gemm_output_modes(c0, mode, offset):
+    """The three output modes on the grouped-GEMM path (80 slots), with out aligned and not 16-byte aligned."""
+    cfg = c0.cfg
+    T = 40
+    ub = inputs.activations(cfg, step=90 + mode, T=T)
+    u = u_vals(ub)
+    ref_logits = O.router_logits(u, c0.host["router"])
+    idx = O.topk(ref_logits, cfg.K)
+    w = O.gating(ref_logits, idx)
+    x0 = np.random.default_rng(mode).standard_normal((T, cfg.H)) * 4 if mode == 2 else None
+    out, _ = expert_forward(c0, ub, cfg.K, idx, w, mode=mode, x0=x0, offset=offset)
     ref = oracle_out(c0, u, idx, w)
     if mode == 2:
         out = out - x0.astype(np.float32)
