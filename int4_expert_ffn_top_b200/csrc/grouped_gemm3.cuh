@@ -61,6 +61,7 @@ using tc::mma_f16_ts;
 using tc::sa;
 using tc::smem_desc;
 using tc::tma_load_2d;
+using tc::tmem_ld16;
 using tc::tmem_ld32;
 using tc::tmem_st16;
 using tc::tmem_st_wait;
@@ -94,6 +95,7 @@ constexpr int LORA_T = 2 * BN * 32 * 4;  // epilogue staging of the tile's LoRA 
 constexpr int OFF_OUT = OFF_RAW + RSTAGES * RAW_STAGE;
 constexpr int OFF_LT = OFF_OUT + STAGE_OUT;
 constexpr int OFF_RS = OFF_LT + LORA_T;  // ... of its gating weights ...
+static_assert(BN * BM * 2 <= LORA_T, "a tile of precomputed fp16 deltas fits the LoRA staging area");
 constexpr int LORA_B = BM * 32 * 4;
 constexpr int OFF_BL = OFF_RS + BN * 4;  // ... and of its rows' LoRA B values times the LoRA scale, [i][row]
 constexpr int OFF_SB = OFF_BL + LORA_B;
@@ -123,6 +125,11 @@ struct Args {
   const float* lora_t2;
   const uint16_t* lora_Bex;
   const uint16_t* lora_Bgu_ex;  // SwiGLU, routed: per-expert B [E][2I][r] in the block's interleaved row order
+  // the shared expert's unmerged LoRA deltas, computed per token beforehand: fp16 [token][lora_D_ld] (output
+  // rows in the weight matrix's order); shared rows start at tile row lora_D_row0 (null: none)
+  const uint16_t* lora_D;
+  int lora_D_ld;
+  int lora_D_row0;
   int lora_r;
   float lora_scale;
   int* err;
@@ -166,6 +173,14 @@ MOE_DEV uint4 dequant_pair_order(uint32_t w, __half2 s2, __half2 b2) {
 }
 
 MOE_DEV uint32_t parity(int count, int stages) { return static_cast<uint32_t>(count / stages) & 1u; }
+
+// Barrier of the 256 epilogue threads (named barrier 1).  The warp is reconverged first and the barrier is the
+// non-aligned form: the lanes of a warp may come from loops of different trip counts, and the aligned form
+// would let a warp that arrives diverged release the others early.
+MOE_DEV void epi_sync() {
+  __syncwarp();
+  asm volatile("barrier.sync 1, 256;" ::: "memory");
+}
 
 // OR of v over the 256 epilogue threads (named barrier 1), so that they take the same branch.
 MOE_DEV bool epi_any(bool v) {
@@ -468,13 +483,51 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
       else
         Bsrc = tile.e < a.E ? (a.lora_Bex ? a.lora_Bex + static_cast<size_t>(tile.e) * a.out_ld * r : nullptr)
                             : a.lora_B1;
-      const bool any_lora = swiglu ? (tile.e == a.E ? (a.lora_B1 || a.lora_B2) : Bgu != nullptr)
-                                   : (tile.e < a.E ? a.lora_Bex != nullptr : a.lora_B1 != nullptr);
+      const bool dtile = tile.e == a.E && a.lora_D;  // the shared expert's precomputed deltas (they take the
+                                                     // LoRA staging area: no B.t term on such a tile)
+      if (dtile) Bsrc = nullptr;
+      const bool any_lora = !dtile && (swiglu ? (tile.e == a.E ? (a.lora_B1 || a.lora_B2) : Bgu != nullptr)
+                                              : (tile.e < a.E ? a.lora_Bex != nullptr : a.lora_B1 != nullptr));
+      if (dtile) {  // [token][128 rows] fp16 into the LoRA staging area, every load in flight at once
+        const uint16_t* src = a.lora_D + static_cast<size_t>(tile.row0 - a.lora_D_row0) * a.lora_D_ld + tile.mt * BM;
+#pragma unroll 1
+        for (int i0 = et; i0 < BN * 16; i0 += 4 * kEpi) {  // four 16-byte loads in flight per thread
+          uint4 x[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int i = i0 + q * kEpi, t = i >> 4, ch = i & 15;
+            if (t < tile.n) x[q] = *reinterpret_cast<const uint4*>(src + static_cast<size_t>(t) * a.lora_D_ld + ch * 8);
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int i = i0 + q * kEpi;
+            if ((i >> 4) < tile.n) reinterpret_cast<uint4*>(lt)[i] = x[q];
+          }
+        }
+      }
+      const int rs = (r + 3) & ~3;  // staged t rows are padded with zeros to whole float4s
       if (any_lora) {  // gate and up rows read different t arrays on SwiGLU tiles: even rows t1, odd rows t2
-        const int tn = tile.n * r;
-        for (int i = et; i < tn; i += kEpi) {
-          lt[i] = a.lora_t1[static_cast<size_t>(tile.row0) * r + i];
-          if (swiglu) lt[BN * 32 + i] = a.lora_t2 ? a.lora_t2[static_cast<size_t>(tile.row0) * r + i] : 0.f;
+        const int tn = tile.n * rs;
+        const float* g1 = a.lora_t1 + static_cast<size_t>(tile.row0) * r;
+        const float* g2 = swiglu && a.lora_t2 ? a.lora_t2 + static_cast<size_t>(tile.row0) * r : nullptr;
+#pragma unroll 1
+        for (int i0 = et; i0 < tn; i0 += 4 * kEpi) {  // four loads of each set in flight per thread
+          float x1[4], x2[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int i = i0 + q * kEpi, t = i / rs, j = i - t * rs;
+            const bool in = i < tn && j < r;
+            x1[q] = in ? g1[t * r + j] : 0.f;
+            x2[q] = in && g2 ? g2[t * r + j] : 0.f;
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int i = i0 + q * kEpi;
+            if (i < tn) {
+              lt[i] = x1[q];
+              if (swiglu) lt[BN * 32 + i] = x2[q];
+            }
+          }
         }
       }
       if (!swiglu && tile.e < a.E && a.row_scale)
@@ -484,7 +537,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
                                            : a.lora_B1;
         for (int i = et; i < BM * r; i += kEpi) {
           const int row = i / r, j = i - row * r, oo = tile.mt * BM + row;
-          // shared gate/up: B per projection ([I][r], row oo / 2); routed gate/up: interleaved rows ([2I][r], row oo)
           const bool per_proj = swiglu && tile.e == a.E;
           const uint16_t* src = swiglu ? (per_proj ? ((row & 1) ? a.lora_B2 : a.lora_B1) : Bgu) : Bdn;
           bls[j * BM + row] =
@@ -501,24 +553,30 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
       const float* ltr = lt + (up ? BN * 32 : 0);
       bool range_bad = false;  // a SwiGLU output fp16 cannot hold: MOE_ERR_RANGE
 #pragma unroll 1
-      for (int blk = 0; blk < 2; ++blk) {
-        const int c0 = 64 * chalf + 32 * blk;
-        float v[32];
+      for (int blk = 0; blk < 4; ++blk) {  // 16 columns at a time: fewer live registers
+        const int c0 = 64 * chalf + 16 * blk;
+        float v[16];
         const bool live = c0 < tile.n;
-        if (live) tmem_ld32(taddr + c0, v);
-        if (blk == 1) {  // the accumulator is read: release it for the tile after next
+        if (live) tmem_ld16(taddr + c0, v);
+        if (blk == 3) {  // the accumulator is read: release it for the tile after next
           asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
           __syncwarp();
           if (lane == 0) bar_arrive(acc_empty + ab);
+        }
+        if (live && dtile) {  // + the shared expert's delta of this row and token
+          const uint16_t* ds = reinterpret_cast<const uint16_t*>(lt);
+#pragma unroll
+          for (int t = 0; t < 16; ++t)
+            if (c0 + t < tile.n) v[t] += half_bits_to_float(ds[(c0 + t) * BM + L]);
         }
         if (live && Bsrc) {  // unmerged LoRA: + scale * B[row] . t[token]
 #pragma unroll 1
           for (int i = 0; i < r; ++i) {
             const float bi = bls[i * BM + L];
 #pragma unroll
-            for (int t = 0; t < 32; ++t) {
+            for (int t = 0; t < 16; ++t) {
               const int tt = c0 + t < tile.n ? c0 + t : tile.n - 1;
-              v[t] = fmaf(bi, ltr[tt * r + i], v[t]);
+              v[t] = fmaf(bi, ltr[tt * rs + i], v[t]);
             }
           }
         }
@@ -526,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
           const int col = pair_pos(L >> 1);  // SwiGLU outputs in pair order (the down GEMM's token operand)
           if (live) {
 #pragma unroll
-            for (int t = 0; t < 32; ++t) {
+            for (int t = 0; t < 16; ++t) {
               const float partner = __shfl_xor_sync(0xffffffffu, v[t], 1);
               if (!up && c0 + t < tile.n) {
                 const float hv = __fdividef(v[t], 1.0f + __expf(-v[t])) * partner;  // fp16 result: fast SiLU
@@ -539,7 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
           const bool scaled = tile.e < a.E && a.row_scale;
           if (live) {
 #pragma unroll
-            for (int t = 0; t < 32; ++t) {
+            for (int t = 0; t < 16; ++t) {
               if (c0 + t < tile.n) {
                 const float xv = scaled ? v[t] * rsc[c0 + t] : v[t];
                 stage[(c0 + t) * 128 + L] = __half_as_ushort(__float2half_rn(xv));
@@ -550,21 +608,21 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
       }
       if (swiglu) {
         if (range_bad) report(a.err, 6);
-        asm volatile("bar.sync 1, 256;" ::: "memory");
+        epi_sync();
         for (int i = et; i < tile.n * 8; i += kEpi) {
           const int t = i >> 3, ch = i & 7;
           *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(tile.row0 + t) * a.out_ld + tile.mt * 64 + ch * 8) =
               reinterpret_cast<const uint4*>(stage + t * 64)[ch];
         }
       } else {
-        asm volatile("bar.sync 1, 256;" ::: "memory");
+        epi_sync();
         for (int i = et; i < tile.n * 16; i += kEpi) {
           const int t = i >> 4, ch = i & 15;
           *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(tile.row0 + t) * a.out_ld + tile.mt * BM + ch * 8) =
               reinterpret_cast<const uint4*>(stage + t * 128)[ch];
         }
       }
-      asm volatile("bar.sync 1, 256;" ::: "memory");  // staging buffers are free for the next tile
+      epi_sync();  // staging buffers are free for the next tile
     }
   }
   if (fail) report(a.err, 5);

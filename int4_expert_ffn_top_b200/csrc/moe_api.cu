@@ -262,6 +262,7 @@ struct GWs {
   int32_t *idx, *count, *offset, *perm, *inv, *blockhist;
   float *w_pos, *t1, *t2, *g;
   uint16_t *X, *Hh, *Y;
+  uint16_t* D;  // the shared expert's per-token LoRA deltas: gate/up [T][2I], then (reused) down [T][H]
   tc::Tile *tiles_gu, *tiles_dn;
   int* n_tiles;
   int* err;
@@ -296,6 +297,7 @@ GWs carve_gemm(void* base, int T, int K, int E, int H, int I, int r) {
   w.X = reinterpret_cast<uint16_t*>(take(R * H * 2));
   w.Hh = reinterpret_cast<uint16_t*>(take(R * I * 2));
   w.Y = reinterpret_cast<uint16_t*>(take(R * H * 2));
+  w.D = reinterpret_cast<uint16_t*>(take(r > 0 ? static_cast<size_t>(T) * (2 * I > H ? 2 * I : H) * 2 : 16));
   w.tiles_gu = reinterpret_cast<tc::Tile*>(take(static_cast<size_t>(w.max_gu) * sizeof(tc::Tile)));
   w.tiles_dn = reinterpret_cast<tc::Tile*>(take(static_cast<size_t>(w.max_dn) * sizeof(tc::Tile)));
   w.n_tiles = reinterpret_cast<int*>(take(2 * 4));
@@ -490,7 +492,7 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
                                               ws.tiles_dn, ws.n_tiles);
   // The GEMMs trust the device-built tile list: stop here if any launch so far failed.
   if (launch_status() != MOE_OK) return MOE_ERR_CUDA;
-  {  // the shared expert's gate and gate/up LoRA-A products, one pass over u
+  {  // the shared expert's gate and gate/up LoRA deltas, one pass over u
     const int nt = lora_gu ? pf::shared_tokens_nt(r) : 0, smem = pf::shared_tokens_smem(H, nt);
     auto kern = nt == 0 ? pf::shared_tokens_kernel<0>
                         : (nt == 2 ? pf::shared_tokens_kernel<2> : (nt == 4 ? pf::shared_tokens_kernel<4>
@@ -498,8 +500,9 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return MOE_ERR_CUDA;
     kern<<<(T + pf::kStTok - 1) / pf::kStTok, 32 * pf::kStWarps, smem, st>>>(
-        u, T, H, static_cast<const uint8_t*>(L->shared_gate.rows), ws.g, TK, r, lora_g ? L->sh_lora_A[0] : nullptr,
-        lora_u ? L->sh_lora_A[1] : nullptr, ws.t1, ws.t2);
+        u, T, H, static_cast<const uint8_t*>(L->shared_gate.rows), ws.g, r, lora_g ? L->sh_lora_A[0] : nullptr,
+        lora_u ? L->sh_lora_A[1] : nullptr, I, lora_g ? L->sh_lora_B[0] : nullptr, lora_u ? L->sh_lora_B[1] : nullptr,
+        L->lora_scale, ws.D);
   }
   const bool ex_gu = r > 0 && L->ex_lora_A_gu;
   if (ex_gu) {  // the routed gate/up adapters' A products on the permuted token rows
@@ -542,9 +545,12 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
     a.drop_tile = drop_tile;
     a.out = ws.Hh;
     a.out_ld = I;
-    a.lora_B1 = lora_g ? L->sh_lora_B[0] : nullptr;
-    a.lora_B2 = lora_u ? L->sh_lora_B[1] : nullptr;
-    if (lora_gu || ex_gu) {
+    if (lora_gu) {  // the shared expert's rows add their precomputed deltas
+      a.lora_D = ws.D;
+      a.lora_D_ld = 2 * I;
+      a.lora_D_row0 = TK;
+    }
+    if (ex_gu) {
       a.lora_t1 = ws.t1;
       a.lora_t2 = ws.t2;
     }
@@ -552,12 +558,12 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
     gg3::grouped_gemm3_kernel<<<grid_gu, gg3::kThreads, smem_gu, st>>>(m_gu, a);
   }
   const bool ex = r > 0 && L->ex_lora_A;
-  if (lora_d || ex) {  // LoRA A products on the SwiGLU output (shared down, routed down)
-    const int row_begin = ex ? 0 : TK, nrows = ex ? (lora_d ? R : TK) : T;
-    pf::lora_a_rows_kernel<<<(nrows * r + kWarps - 1) / kWarps, kThreads, 0, st>>>(
-        ws.Hh, I, TK, nrows, row_begin, r, lora_d ? L->sh_lora_A[2] : nullptr, ex ? L->ex_lora_A : nullptr, ws.idx,
-        ws.perm, ws.t1);
-  }
+  if (lora_d)  // the shared expert's down-projection LoRA deltas (the gate/up deltas are consumed)
+    pf::shared_down_lora_kernel<<<(T + pf::kStTok - 1) / pf::kStTok, 256, 0, st>>>(
+        ws.Hh + static_cast<size_t>(TK) * I, T, I, H, r, L->sh_lora_A[2], L->sh_lora_B[2], L->lora_scale, ws.D);
+  if (ex)  // the routed down adapters' A products on the SwiGLU output rows
+    pf::lora_a_rows_kernel<<<(TK * r + kWarps - 1) / kWarps, kThreads, 0, st>>>(
+        ws.Hh, I, TK, TK, 0, r, nullptr, L->ex_lora_A, ws.idx, ws.perm, ws.t1);
   {  // down (+ LoRA), routed rows scaled by their gating weight
     gg3::Args a = base_args();
     a.tiles = ws.tiles_dn;
@@ -568,7 +574,11 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
     a.out = ws.Y;
     a.out_ld = H;
     a.row_scale = ws.w_pos;
-    a.lora_B1 = lora_d ? L->sh_lora_B[2] : nullptr;
+    if (lora_d) {
+      a.lora_D = ws.D;
+      a.lora_D_ld = H;
+      a.lora_D_row0 = TK;
+    }
     a.lora_t1 = ws.t1;
     a.lora_Bex = ex ? L->ex_lora_B : nullptr;
     gg3::grouped_gemm3_kernel<<<grid_dn, gg3::kThreads, smem_dn, st>>>(m_dn, a);

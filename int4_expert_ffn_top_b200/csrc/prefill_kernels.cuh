@@ -177,9 +177,11 @@ __global__ void __launch_bounds__(128) tile_list_kernel(const int32_t* __restric
   }
 }
 
-// Shared expert's gate and LoRA-A products for many tokens, in one pass over u:
+// Shared expert's gate and gate/up LoRA deltas for many tokens, in one pass over u:
 //   g[t] = sigmoid(w . u_t), w the 8-bit gate row (affine groups of 64): per group s * sum (q - 128) u + (b + 128 s) * sum u;
-//   t1[TK + t][i] = A_gate[i] . u_t and t2[TK + t][i] = A_up[i] . u_t (a projection without adapter gets zeros).
+//   the LoRA-A products t1 = A_gate u_t and t2 = A_up u_t (r values each; a projection without adapter gets
+//   zeros), then D[t][o] = fp16(scale * B[o] . t) for the 2I interleaved gate/up rows o (even: gate row o / 2
+//   with t1, odd: up row o / 2 with t2): the unmerged LoRA deltas the gate/up GEMM adds to its accumulators.
 // A CTA takes 16 tokens and copies their rows of u into shared memory (16-byte asynchronous copies, all in flight
 // at once; rows padded by 64 bytes so that a warp's reads hit distinct banks).  Its 8 warps split the input
 // dimension into 32-wide chunks (warp w: chunks w, w + 8, ...), and the warps' partial sums are added in warp
@@ -199,15 +201,70 @@ MOE_DEV void mma_tf32(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint
                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// D[t0 + tok][o] = fp16(scale * B_o . t[tok]) for the tokens of a 16-token block and the outputs o < n_out,
+// t[tok] = tS[j][tok] (j < r).  pairs = false: B_o is row o of B_even ([n_out][r]).  pairs = true (the
+// interleaved gate/up rows): B_o is row o / 2 of B_even for even o and of B_odd for odd o (each [n_out / 2][r]),
+// and the odd rows read t from tS[r + j].  A null B gives zeros.  Each thread takes four outputs blockDim.x
+// apart per pass, for all 16 tokens.
+MOE_DEV void lora_delta_rows(const float (*tS)[kStTok], bool pairs, int r, int t0, int T, int n_out,
+                             const uint16_t* __restrict__ B_even, const uint16_t* __restrict__ B_odd, float scale,
+                             uint16_t* __restrict__ D) {
+  for (int o0 = threadIdx.x; o0 < n_out; o0 += 4 * blockDim.x) {
+    const bool odd = pairs && (o0 & 1);  // the four outputs share o0's parity (blockDim.x is even)
+    const uint16_t* src[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int o = o0 + m * blockDim.x;
+      const uint16_t* B = odd ? B_odd : B_even;
+      src[m] = (o < n_out && B) ? B + static_cast<size_t>(pairs ? o >> 1 : o) * r : nullptr;
+    }
+    const int js = odd ? r : 0;
+    float acc[4][kStTok];
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+#pragma unroll
+      for (int k = 0; k < kStTok; ++k) acc[m][k] = 0.f;
+#pragma unroll 1
+    for (int j = 0; j < r; ++j) {
+      float b[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) b[m] = src[m] ? half_bits_to_float(src[m][j]) : 0.f;
+      const float4* tr = reinterpret_cast<const float4*>(tS[js + j]);
+#pragma unroll
+      for (int q = 0; q < kStTok / 4; ++q) {
+        const float4 x = tr[q];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          acc[m][4 * q] = fmaf(b[m], x.x, acc[m][4 * q]);
+          acc[m][4 * q + 1] = fmaf(b[m], x.y, acc[m][4 * q + 1]);
+          acc[m][4 * q + 2] = fmaf(b[m], x.z, acc[m][4 * q + 2]);
+          acc[m][4 * q + 3] = fmaf(b[m], x.w, acc[m][4 * q + 3]);
+        }
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int o = o0 + m * blockDim.x;
+      if (o >= n_out) continue;
+#pragma unroll
+      for (int k = 0; k < kStTok; ++k)
+        if (t0 + k < T) D[static_cast<size_t>(t0 + k) * n_out + o] = __half_as_ushort(__float2half_rn(scale * acc[m][k]));
+    }
+  }
+}
+
 template <int NT>  // 8-row tiles of the 2r LoRA rows (gate rows, then up rows); 0: the gate only
 __global__ void __launch_bounds__(256) shared_tokens_kernel(const uint16_t* __restrict__ u, int T, int H,
                                                             const uint8_t* __restrict__ rec, float* __restrict__ g,
-                                                            int TK, int r, const uint16_t* __restrict__ A_gate,
-                                                            const uint16_t* __restrict__ A_up, float* __restrict__ t1,
-                                                            float* __restrict__ t2) {
+                                                            int r, const uint16_t* __restrict__ A_gate,
+                                                            const uint16_t* __restrict__ A_up, int I,
+                                                            const uint16_t* __restrict__ B_gate,
+                                                            const uint16_t* __restrict__ B_up, float scale,
+                                                            uint16_t* __restrict__ D) {
   constexpr int NTa = NT > 0 ? NT : 1, NC = 8 * NTa;
   extern __shared__ __align__(16) uint8_t st_smem[];
   __shared__ float gred[kStWarps][kStTok];
+  __shared__ __align__(16) float tS[64][kStTok];  // [j][token]: the 2r LoRA-A products (gate's, then up's)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gi = lane >> 2, q = lane & 3;
   const int t0 = blockIdx.x * kStTok, ld = 2 * H + 64;  // staged row stride in bytes
   // stage the 16 token rows (rows past T are zeros)
@@ -331,14 +388,47 @@ __global__ void __launch_bounds__(256) shared_tokens_kernel(const uint16_t* __re
   }
   if (NT > 0) {
     for (int i = threadIdx.x; i < kStTok * NC; i += blockDim.x) {
-      const int tok = i / NC, j = i - tok * NC, t = t0 + tok;
-      if (t >= T || j >= 2 * r) continue;
+      const int tok = i / NC, j = i - tok * NC;
+      if (j >= 2 * r) continue;
       float z = 0.f;
 #pragma unroll
       for (int w = 0; w < kStWarps; ++w) z += red[(w * kStTok + tok) * NC + j];
-      (j < r ? t1 : t2)[static_cast<size_t>(TK + t) * r + (j < r ? j : j - r)] = z;
+      tS[j][tok] = z;  // rows past T hold zeros, like their staged u
     }
+    __syncthreads();
+    lora_delta_rows(tS, true, r, t0, T, 2 * I, B_gate, B_up, scale, D);
   }
+}
+
+// Shared expert's down-projection LoRA delta for many tokens: t_t = A_down h_t (r values) and
+// D[t][o] = fp16(scale * B_down[o] . t_t), h_t the token's SwiGLU output (fp16, pair order within 8-element
+// blocks; A_down [r][I] in natural order).  A CTA takes 16 tokens; a thread first forms one or two of the
+// 16 x r products, then four outputs per pass of the delta.
+__global__ void __launch_bounds__(256) shared_down_lora_kernel(const uint16_t* __restrict__ h, int T, int I, int H,
+                                                               int r, const uint16_t* __restrict__ A_d,
+                                                               const uint16_t* __restrict__ B_d, float scale,
+                                                               uint16_t* __restrict__ D) {
+  __shared__ __align__(16) float tS[32][kStTok];
+  const int t0 = blockIdx.x * kStTok;
+  for (int p = threadIdx.x; p < kStTok * r; p += blockDim.x) {
+    const int tok = p & (kStTok - 1), j = p / kStTok;
+    float acc = 0.f;
+    if (t0 + tok < T) {
+      const uint4* hr = reinterpret_cast<const uint4*>(h + static_cast<size_t>(t0 + tok) * I);
+      const uint4* ar = reinterpret_cast<const uint4*>(A_d + static_cast<size_t>(j) * I);
+#pragma unroll 4
+      for (int c = 0; c < I / 8; ++c) {
+        const uint4 w = ar[c], hv = hr[c];
+        acc = dot2_mix(prmt(w.x, w.z, 0x5410u), hv.x, acc);  // A chunk to pair order
+        acc = dot2_mix(prmt(w.x, w.z, 0x7632u), hv.y, acc);
+        acc = dot2_mix(prmt(w.y, w.w, 0x5410u), hv.z, acc);
+        acc = dot2_mix(prmt(w.y, w.w, 0x7632u), hv.w, acc);
+      }
+    }
+    tS[j][tok] = acc;
+  }
+  __syncthreads();
+  lora_delta_rows(tS, false, r, t0, T, H, B_d, nullptr, scale, D);
 }
 
 // LoRA-A products on the SwiGLU output rows: t[row][i] = A_row[i] . h[row] with
