@@ -558,9 +558,14 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
     gg3::grouped_gemm3_kernel<<<grid_gu, gg3::kThreads, smem_gu, st>>>(m_gu, a);
   }
   const bool ex = r > 0 && L->ex_lora_A;
-  if (lora_d)  // the shared expert's down-projection LoRA deltas (the gate/up deltas are consumed)
-    pf::shared_down_lora_kernel<<<(T + pf::kStTok - 1) / pf::kStTok, 256, 0, st>>>(
+  if (lora_d) {  // the shared expert's down-projection LoRA deltas (the gate/up deltas are consumed)
+    const int smem = pf::shared_down_lora_smem(I, r);
+    if (cudaFuncSetAttribute(pf::shared_down_lora_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+    pf::shared_down_lora_kernel<<<(T + pf::kStTok - 1) / pf::kStTok, 256, smem, st>>>(
         ws.Hh + static_cast<size_t>(TK) * I, T, I, H, r, L->sh_lora_A[2], L->sh_lora_B[2], L->lora_scale, ws.D);
+  }
   if (ex)  // the routed down adapters' A products on the SwiGLU output rows
     pf::lora_a_rows_kernel<<<(TK * r + kWarps - 1) / kWarps, kThreads, 0, st>>>(
         ws.Hh, I, TK, TK, 0, r, nullptr, L->ex_lora_A, ws.idx, ws.perm, ws.t1);

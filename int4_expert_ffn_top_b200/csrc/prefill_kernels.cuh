@@ -204,52 +204,54 @@ MOE_DEV void mma_tf32(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint
 // D[t0 + tok][o] = fp16(scale * B_o . t[tok]) for the tokens of a 16-token block and the outputs o < n_out,
 // t[tok] = tS[j][tok] (j < r).  pairs = false: B_o is row o of B_even ([n_out][r]).  pairs = true (the
 // interleaved gate/up rows): B_o is row o / 2 of B_even for even o and of B_odd for odd o (each [n_out / 2][r]),
-// and the odd rows read t from tS[r + j].  A null B gives zeros.  Each thread takes four outputs blockDim.x
-// apart per pass, for all 16 tokens.
+// and the odd rows read t from tS[r + j].  A null B gives zeros.  One output per thread and pass, all 16
+// tokens; a B row is read 8 ranks per 16-byte load when r is a multiple of 8.
 MOE_DEV void lora_delta_rows(const float (*tS)[kStTok], bool pairs, int r, int t0, int T, int n_out,
                              const uint16_t* __restrict__ B_even, const uint16_t* __restrict__ B_odd, float scale,
                              uint16_t* __restrict__ D) {
-  for (int o0 = threadIdx.x; o0 < n_out; o0 += 4 * blockDim.x) {
-    const bool odd = pairs && (o0 & 1);  // the four outputs share o0's parity (blockDim.x is even)
-    const uint16_t* src[4];
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int o = o0 + m * blockDim.x;
-      const uint16_t* B = odd ? B_odd : B_even;
-      src[m] = (o < n_out && B) ? B + static_cast<size_t>(pairs ? o >> 1 : o) * r : nullptr;
-    }
-    const int js = odd ? r : 0;
-    float acc[4][kStTok];
-#pragma unroll
-    for (int m = 0; m < 4; ++m)
-#pragma unroll
-      for (int k = 0; k < kStTok; ++k) acc[m][k] = 0.f;
+  const bool vec = (r & 7) == 0;
 #pragma unroll 1
-    for (int j = 0; j < r; ++j) {
-      float b[4];
+  for (int o = threadIdx.x; o < n_out; o += blockDim.x) {
+    const bool odd = pairs && (o & 1);
+    const uint16_t* B = odd ? B_odd : B_even;
+    const uint16_t* src = B ? B + static_cast<size_t>(pairs ? o >> 1 : o) * r : nullptr;
+    const int js = odd ? r : 0;
+    float acc[kStTok];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) b[m] = src[m] ? half_bits_to_float(src[m][j]) : 0.f;
-      const float4* tr = reinterpret_cast<const float4*>(tS[js + j]);
+    for (int k = 0; k < kStTok; ++k) acc[k] = 0.f;
+#pragma unroll 1
+    for (int j0 = 0; src && j0 < r; j0 += 8) {
+      float b[8];
+      if (vec) {
+        const uint4 w = *reinterpret_cast<const uint4*>(src + j0);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-      for (int q = 0; q < kStTok / 4; ++q) {
-        const float4 x = tr[q];
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(as_h2(ww[e]));
+          b[2 * e] = f.x;
+          b[2 * e + 1] = f.y;
+        }
+      } else {
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          acc[m][4 * q] = fmaf(b[m], x.x, acc[m][4 * q]);
-          acc[m][4 * q + 1] = fmaf(b[m], x.y, acc[m][4 * q + 1]);
-          acc[m][4 * q + 2] = fmaf(b[m], x.z, acc[m][4 * q + 2]);
-          acc[m][4 * q + 3] = fmaf(b[m], x.w, acc[m][4 * q + 3]);
+        for (int e = 0; e < 8; ++e) b[e] = j0 + e < r ? half_bits_to_float(src[j0 + e]) : 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if (j0 + e >= r) break;
+        const float4* tr = reinterpret_cast<const float4*>(tS[js + j0 + e]);
+#pragma unroll
+        for (int q = 0; q < kStTok / 4; ++q) {
+          const float4 x = tr[q];
+          acc[4 * q] = fmaf(b[e], x.x, acc[4 * q]);
+          acc[4 * q + 1] = fmaf(b[e], x.y, acc[4 * q + 1]);
+          acc[4 * q + 2] = fmaf(b[e], x.z, acc[4 * q + 2]);
+          acc[4 * q + 3] = fmaf(b[e], x.w, acc[4 * q + 3]);
         }
       }
     }
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int o = o0 + m * blockDim.x;
-      if (o >= n_out) continue;
-#pragma unroll
-      for (int k = 0; k < kStTok; ++k)
-        if (t0 + k < T) D[static_cast<size_t>(t0 + k) * n_out + o] = __half_as_ushort(__float2half_rn(scale * acc[m][k]));
-    }
+    for (int k = 0; k < kStTok; ++k)
+      if (t0 + k < T) D[static_cast<size_t>(t0 + k) * n_out + o] = __half_as_ushort(__float2half_rn(scale * acc[k]));
   }
 }
 
@@ -402,28 +404,45 @@ __global__ void __launch_bounds__(256) shared_tokens_kernel(const uint16_t* __re
 
 // Shared expert's down-projection LoRA delta for many tokens: t_t = A_down h_t (r values) and
 // D[t][o] = fp16(scale * B_down[o] . t_t), h_t the token's SwiGLU output (fp16, pair order within 8-element
-// blocks; A_down [r][I] in natural order).  A CTA takes 16 tokens; a thread first forms one or two of the
-// 16 x r products, then four outputs per pass of the delta.
+// blocks; A_down [r][I] in natural order).  A CTA takes 16 tokens: their h rows and the r rows of A_down go to
+// shared memory first (16-byte asynchronous copies, all in flight; rows padded by 16 bytes so that the eight
+// lanes of a 16-byte load phase, eight tokens, hit distinct banks); a thread then forms one or two of the
+// 16 x r products, and one output per pass of the delta.
+inline int shared_down_lora_smem(int I, int r) { return (kStTok + r) * (2 * I + 16); }
 __global__ void __launch_bounds__(256) shared_down_lora_kernel(const uint16_t* __restrict__ h, int T, int I, int H,
                                                                int r, const uint16_t* __restrict__ A_d,
                                                                const uint16_t* __restrict__ B_d, float scale,
                                                                uint16_t* __restrict__ D) {
+  extern __shared__ __align__(16) uint8_t sd_smem[];
   __shared__ __align__(16) float tS[32][kStTok];
-  const int t0 = blockIdx.x * kStTok;
+  const int t0 = blockIdx.x * kStTok, ld = 2 * I + 16, n16 = I / 8;  // staged row stride in bytes
+  for (int i = threadIdx.x; i < (kStTok + r) * n16; i += blockDim.x) {
+    const int row = i / n16, piece = i - row * n16;
+    uint8_t* dst = sd_smem + row * ld + piece * 16;
+    const uint16_t* src = row < kStTok ? (t0 + row < T ? h + static_cast<size_t>(t0 + row) * I : nullptr)
+                                       : A_d + static_cast<size_t>(row - kStTok) * I;
+    if (src)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                   "l"(src + piece * 8)
+                   : "memory");
+    else
+      *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
   for (int p = threadIdx.x; p < kStTok * r; p += blockDim.x) {
     const int tok = p & (kStTok - 1), j = p / kStTok;
+    const uint4* hr = reinterpret_cast<const uint4*>(sd_smem + tok * ld);
+    const uint4* ar = reinterpret_cast<const uint4*>(sd_smem + (kStTok + j) * ld);
     float acc = 0.f;
-    if (t0 + tok < T) {
-      const uint4* hr = reinterpret_cast<const uint4*>(h + static_cast<size_t>(t0 + tok) * I);
-      const uint4* ar = reinterpret_cast<const uint4*>(A_d + static_cast<size_t>(j) * I);
 #pragma unroll 4
-      for (int c = 0; c < I / 8; ++c) {
-        const uint4 w = ar[c], hv = hr[c];
-        acc = dot2_mix(prmt(w.x, w.z, 0x5410u), hv.x, acc);  // A chunk to pair order
-        acc = dot2_mix(prmt(w.x, w.z, 0x7632u), hv.y, acc);
-        acc = dot2_mix(prmt(w.y, w.w, 0x5410u), hv.z, acc);
-        acc = dot2_mix(prmt(w.y, w.w, 0x7632u), hv.w, acc);
-      }
+    for (int c = 0; c < n16; ++c) {
+      const uint4 w = ar[c], hv = hr[c];
+      acc = dot2_mix(prmt(w.x, w.z, 0x5410u), hv.x, acc);  // A chunk to pair order
+      acc = dot2_mix(prmt(w.x, w.z, 0x7632u), hv.y, acc);
+      acc = dot2_mix(prmt(w.y, w.w, 0x5410u), hv.z, acc);
+      acc = dot2_mix(prmt(w.y, w.w, 0x7632u), hv.w, acc);
     }
     tS[j][tok] = acc;
   }
