@@ -204,36 +204,47 @@ MOE_DEV void mma_tf32(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint
 // D[t0 + tok][o] = fp16(scale * B_o . t[tok]) for the tokens of a 16-token block and the outputs o < n_out,
 // t[tok] = tS[j][tok] (j < r).  pairs = false: B_o is row o of B_even ([n_out][r]).  pairs = true (the
 // interleaved gate/up rows): B_o is row o / 2 of B_even for even o and of B_odd for odd o (each [n_out / 2][r]),
-// and the odd rows read t from tS[r + j].  A null B gives zeros.  One output per thread and pass, all 16
+// and the odd rows read t from tS[r + j].  A null B gives zeros.  Two outputs per thread and pass, all 16
 // tokens; a B row is read 8 ranks per 16-byte load when r is a multiple of 8.
 MOE_DEV void lora_delta_rows(const float (*tS)[kStTok], bool pairs, int r, int t0, int T, int n_out,
                              const uint16_t* __restrict__ B_even, const uint16_t* __restrict__ B_odd, float scale,
                              uint16_t* __restrict__ D) {
   const bool vec = (r & 7) == 0;
+  // two outputs blockDim.x apart per pass (same parity: blockDim.x is even), their B loads issued together
 #pragma unroll 1
-  for (int o = threadIdx.x; o < n_out; o += blockDim.x) {
-    const bool odd = pairs && (o & 1);
+  for (int o0 = threadIdx.x; o0 < n_out; o0 += 2 * blockDim.x) {
+    const bool odd = pairs && (o0 & 1);
     const uint16_t* B = odd ? B_odd : B_even;
-    const uint16_t* src = B ? B + static_cast<size_t>(pairs ? o >> 1 : o) * r : nullptr;
+    const uint16_t* src[2];
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const int o = o0 + m * blockDim.x;
+      src[m] = (B && o < n_out) ? B + static_cast<size_t>(pairs ? o >> 1 : o) * r : nullptr;
+    }
     const int js = odd ? r : 0;
-    float acc[kStTok];
+    float acc[2][kStTok];
 #pragma unroll
-    for (int k = 0; k < kStTok; ++k) acc[k] = 0.f;
+    for (int m = 0; m < 2; ++m)
+#pragma unroll
+      for (int k = 0; k < kStTok; ++k) acc[m][k] = 0.f;
 #pragma unroll 1
-    for (int j0 = 0; src && j0 < r; j0 += 8) {
-      float b[8];
-      if (vec) {
-        const uint4 w = *reinterpret_cast<const uint4*>(src + j0);
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    for (int j0 = 0; (src[0] || src[1]) && j0 < r; j0 += 8) {
+      float b[2][8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __half22float2(as_h2(ww[e]));
-          b[2 * e] = f.x;
-          b[2 * e + 1] = f.y;
+      for (int m = 0; m < 2; ++m) {
+        if (vec) {
+          const uint4 w = src[m] ? *reinterpret_cast<const uint4*>(src[m] + j0) : make_uint4(0, 0, 0, 0);
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(as_h2(ww[e]));
+            b[m][2 * e] = f.x;
+            b[m][2 * e + 1] = f.y;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) b[m][e] = (src[m] && j0 + e < r) ? half_bits_to_float(src[m][j0 + e]) : 0.f;
         }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) b[e] = j0 + e < r ? half_bits_to_float(src[j0 + e]) : 0.f;
       }
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -242,16 +253,25 @@ MOE_DEV void lora_delta_rows(const float (*tS)[kStTok], bool pairs, int r, int t
 #pragma unroll
         for (int q = 0; q < kStTok / 4; ++q) {
           const float4 x = tr[q];
-          acc[4 * q] = fmaf(b[e], x.x, acc[4 * q]);
-          acc[4 * q + 1] = fmaf(b[e], x.y, acc[4 * q + 1]);
-          acc[4 * q + 2] = fmaf(b[e], x.z, acc[4 * q + 2]);
-          acc[4 * q + 3] = fmaf(b[e], x.w, acc[4 * q + 3]);
+#pragma unroll
+          for (int m = 0; m < 2; ++m) {
+            acc[m][4 * q] = fmaf(b[m][e], x.x, acc[m][4 * q]);
+            acc[m][4 * q + 1] = fmaf(b[m][e], x.y, acc[m][4 * q + 1]);
+            acc[m][4 * q + 2] = fmaf(b[m][e], x.z, acc[m][4 * q + 2]);
+            acc[m][4 * q + 3] = fmaf(b[m][e], x.w, acc[m][4 * q + 3]);
+          }
         }
       }
     }
 #pragma unroll
-    for (int k = 0; k < kStTok; ++k)
-      if (t0 + k < T) D[static_cast<size_t>(t0 + k) * n_out + o] = __half_as_ushort(__float2half_rn(scale * acc[k]));
+    for (int m = 0; m < 2; ++m) {
+      const int o = o0 + m * blockDim.x;
+      if (o >= n_out) continue;
+#pragma unroll
+      for (int k = 0; k < kStTok; ++k)
+        if (t0 + k < T)
+          D[static_cast<size_t>(t0 + k) * n_out + o] = __half_as_ushort(__float2half_rn(scale * acc[m][k]));
+    }
   }
 }
 
@@ -409,7 +429,7 @@ __global__ void __launch_bounds__(256) shared_tokens_kernel(const uint16_t* __re
 // lanes of a 16-byte load phase, eight tokens, hit distinct banks); a thread then forms one or two of the
 // 16 x r products, and one output per pass of the delta.
 inline int shared_down_lora_smem(int I, int r) { return (kStTok + r) * (2 * I + 16); }
-__global__ void __launch_bounds__(256) shared_down_lora_kernel(const uint16_t* __restrict__ h, int T, int I, int H,
+__global__ void __launch_bounds__(256, 2) shared_down_lora_kernel(const uint16_t* __restrict__ h, int T, int I, int H,
                                                                int r, const uint16_t* __restrict__ A_d,
                                                                const uint16_t* __restrict__ B_d, float scale,
                                                                uint16_t* __restrict__ D) {
