@@ -263,6 +263,7 @@ struct GWs {
   float *w_pos, *t1, *t2, *g;
   uint16_t *X, *Hh, *Y;
   uint16_t* D;  // the shared expert's per-token LoRA deltas: gate/up [T][2I], then (reused) down [T][H]
+  float* tv;    // their per-token LoRA-A products: gate/up [T][2r], then (reused) down [T][r]
   tc::Tile *tiles_gu, *tiles_dn;
   int* n_tiles;
   int* err;
@@ -298,6 +299,7 @@ GWs carve_gemm(void* base, int T, int K, int E, int H, int I, int r) {
   w.Hh = reinterpret_cast<uint16_t*>(take(R * I * 2));
   w.Y = reinterpret_cast<uint16_t*>(take(R * H * 2));
   w.D = reinterpret_cast<uint16_t*>(take(r > 0 ? static_cast<size_t>(T) * (2 * I > H ? 2 * I : H) * 2 : 16));
+  w.tv = reinterpret_cast<float*>(take(static_cast<size_t>(T) * 2 * rr * 4));
   w.tiles_gu = reinterpret_cast<tc::Tile*>(take(static_cast<size_t>(w.max_gu) * sizeof(tc::Tile)));
   w.tiles_dn = reinterpret_cast<tc::Tile*>(take(static_cast<size_t>(w.max_dn) * sizeof(tc::Tile)));
   w.n_tiles = reinterpret_cast<int*>(take(2 * 4));
@@ -501,8 +503,11 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
       return MOE_ERR_CUDA;
     kern<<<(T + pf::kStTok - 1) / pf::kStTok, 32 * pf::kStWarps, smem, st>>>(
         u, T, H, static_cast<const uint8_t*>(L->shared_gate.rows), ws.g, r, lora_g ? L->sh_lora_A[0] : nullptr,
-        lora_u ? L->sh_lora_A[1] : nullptr, I, lora_g ? L->sh_lora_B[0] : nullptr, lora_u ? L->sh_lora_B[1] : nullptr,
-        L->lora_scale, ws.D);
+        lora_u ? L->sh_lora_A[1] : nullptr, ws.tv);
+    if (lora_gu)
+      pf::lora_delta_kernel<<<dim3((T + pf::kStTok - 1) / pf::kStTok, (2 * I + pf::kDeltaOut - 1) / pf::kDeltaOut), 128, 0,
+                              st>>>(ws.tv, T, r, true, 2 * I, lora_g ? L->sh_lora_B[0] : nullptr,
+                                    lora_u ? L->sh_lora_B[1] : nullptr, L->lora_scale, ws.D);
   }
   const bool ex_gu = r > 0 && L->ex_lora_A_gu;
   if (ex_gu) {  // the routed gate/up adapters' A products on the permuted token rows
@@ -564,7 +569,9 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
         cudaSuccess)
       return MOE_ERR_CUDA;
     pf::shared_down_lora_kernel<<<(T + pf::kStTok - 1) / pf::kStTok, 256, smem, st>>>(
-        ws.Hh + static_cast<size_t>(TK) * I, T, I, H, r, L->sh_lora_A[2], L->sh_lora_B[2], L->lora_scale, ws.D);
+        ws.Hh + static_cast<size_t>(TK) * I, T, I, r, L->sh_lora_A[2], ws.tv);
+    pf::lora_delta_kernel<<<dim3((T + pf::kStTok - 1) / pf::kStTok, (H + pf::kDeltaOut - 1) / pf::kDeltaOut), 128, 0,
+                            st>>>(ws.tv, T, r, false, H, L->sh_lora_B[2], nullptr, L->lora_scale, ws.D);
   }
   if (ex)  // the routed down adapters' A products on the SwiGLU output rows
     pf::lora_a_rows_kernel<<<(TK * r + kWarps - 1) / kWarps, kThreads, 0, st>>>(

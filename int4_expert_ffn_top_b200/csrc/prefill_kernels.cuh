@@ -180,8 +180,7 @@ __global__ void __launch_bounds__(128) tile_list_kernel(const int32_t* __restric
 // Shared expert's gate and gate/up LoRA deltas for many tokens, in one pass over u:
 //   g[t] = sigmoid(w . u_t), w the 8-bit gate row (affine groups of 64): per group s * sum (q - 128) u + (b + 128 s) * sum u;
 //   the LoRA-A products t1 = A_gate u_t and t2 = A_up u_t (r values each; a projection without adapter gets
-//   zeros), then D[t][o] = fp16(scale * B[o] . t) for the 2I interleaved gate/up rows o (even: gate row o / 2
-//   with t1, odd: up row o / 2 with t2): the unmerged LoRA deltas the gate/up GEMM adds to its accumulators.
+//   zeros) into tv[t] = (t1, t2), from which lora_delta_kernel forms the unmerged deltas the gate/up GEMM adds.
 // A CTA takes 16 tokens and copies their rows of u into shared memory (16-byte asynchronous copies, all in flight
 // at once; rows padded by 64 bytes so that a warp's reads hit distinct banks).  Its 8 warps split the input
 // dimension into 32-wide chunks (warp w: chunks w, w + 8, ...), and the warps' partial sums are added in warp
@@ -201,25 +200,26 @@ MOE_DEV void mma_tf32(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint
                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// D[t0 + tok][o] = fp16(scale * B_o . t[tok]) for the tokens of a 16-token block and the outputs o < n_out,
+// D[t0 + tok][o] = fp16(scale * B_o . t[tok]) for the tokens of a 16-token block and outputs o_begin <= o < o_end
+// (D rows hold n_out outputs),
 // t[tok] = tS[j][tok] (j < r).  pairs = false: B_o is row o of B_even ([n_out][r]).  pairs = true (the
 // interleaved gate/up rows): B_o is row o / 2 of B_even for even o and of B_odd for odd o (each [n_out / 2][r]),
 // and the odd rows read t from tS[r + j].  A null B gives zeros.  Two outputs per thread and pass, all 16
 // tokens; a B row is read 8 ranks per 16-byte load when r is a multiple of 8.
-MOE_DEV void lora_delta_rows(const float (*tS)[kStTok], bool pairs, int r, int t0, int T, int n_out,
-                             const uint16_t* __restrict__ B_even, const uint16_t* __restrict__ B_odd, float scale,
-                             uint16_t* __restrict__ D) {
+MOE_DEV void lora_delta_rows(const float (*tS)[kStTok], bool pairs, int r, int t0, int T, int n_out, int o_begin,
+                             int o_end, const uint16_t* __restrict__ B_even, const uint16_t* __restrict__ B_odd,
+                             float scale, uint16_t* __restrict__ D) {
   const bool vec = (r & 7) == 0;
-  // two outputs blockDim.x apart per pass (same parity: blockDim.x is even), their B loads issued together
+  // two outputs blockDim.x apart per pass (same parity: blockDim.x and o_begin are even), their B loads together
 #pragma unroll 1
-  for (int o0 = threadIdx.x; o0 < n_out; o0 += 2 * blockDim.x) {
+  for (int o0 = o_begin + threadIdx.x; o0 < o_end; o0 += 2 * blockDim.x) {
     const bool odd = pairs && (o0 & 1);
     const uint16_t* B = odd ? B_odd : B_even;
     const uint16_t* src[2];
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
       const int o = o0 + m * blockDim.x;
-      src[m] = (B && o < n_out) ? B + static_cast<size_t>(pairs ? o >> 1 : o) * r : nullptr;
+      src[m] = (B && o < o_end) ? B + static_cast<size_t>(pairs ? o >> 1 : o) * r : nullptr;
     }
     const int js = odd ? r : 0;
     float acc[2][kStTok];
@@ -266,7 +266,7 @@ MOE_DEV void lora_delta_rows(const float (*tS)[kStTok], bool pairs, int r, int t
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
       const int o = o0 + m * blockDim.x;
-      if (o >= n_out) continue;
+      if (o >= o_end) continue;
 #pragma unroll
       for (int k = 0; k < kStTok; ++k)
         if (t0 + k < T)
@@ -279,14 +279,11 @@ template <int NT>  // 8-row tiles of the 2r LoRA rows (gate rows, then up rows);
 __global__ void __launch_bounds__(256) shared_tokens_kernel(const uint16_t* __restrict__ u, int T, int H,
                                                             const uint8_t* __restrict__ rec, float* __restrict__ g,
                                                             int r, const uint16_t* __restrict__ A_gate,
-                                                            const uint16_t* __restrict__ A_up, int I,
-                                                            const uint16_t* __restrict__ B_gate,
-                                                            const uint16_t* __restrict__ B_up, float scale,
-                                                            uint16_t* __restrict__ D) {
+                                                            const uint16_t* __restrict__ A_up,
+                                                            float* __restrict__ tv) {
   constexpr int NTa = NT > 0 ? NT : 1, NC = 8 * NTa;
   extern __shared__ __align__(16) uint8_t st_smem[];
   __shared__ float gred[kStWarps][kStTok];
-  __shared__ __align__(16) float tS[64][kStTok];  // [j][token]: the 2r LoRA-A products (gate's, then up's)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gi = lane >> 2, q = lane & 3;
   const int t0 = blockIdx.x * kStTok, ld = 2 * H + 64;  // staged row stride in bytes
   // stage the 16 token rows (rows past T are zeros)
@@ -411,30 +408,44 @@ __global__ void __launch_bounds__(256) shared_tokens_kernel(const uint16_t* __re
   if (NT > 0) {
     for (int i = threadIdx.x; i < kStTok * NC; i += blockDim.x) {
       const int tok = i / NC, j = i - tok * NC;
-      if (j >= 2 * r) continue;
+      if (j >= 2 * r || t0 + tok >= T) continue;
       float z = 0.f;
 #pragma unroll
       for (int w = 0; w < kStWarps; ++w) z += red[(w * kStTok + tok) * NC + j];
-      tS[j][tok] = z;  // rows past T hold zeros, like their staged u
+      tv[static_cast<size_t>(t0 + tok) * 2 * r + j] = z;
     }
-    __syncthreads();
-    lora_delta_rows(tS, true, r, t0, T, 2 * I, B_gate, B_up, scale, D);
   }
 }
 
-// Shared expert's down-projection LoRA delta for many tokens: t_t = A_down h_t (r values) and
-// D[t][o] = fp16(scale * B_down[o] . t_t), h_t the token's SwiGLU output (fp16, pair order within 8-element
-// blocks; A_down [r][I] in natural order).  A CTA takes 16 tokens: their h rows and the r rows of A_down go to
-// shared memory first (16-byte asynchronous copies, all in flight; rows padded by 16 bytes so that the eight
-// lanes of a 16-byte load phase, eight tokens, hit distinct banks); a thread then forms one or two of the
-// 16 x r products, and one output per pass of the delta.
+// The shared expert's unmerged LoRA deltas from per-token t vectors tv [T][kt] (pairs: kt = 2r, the gate's r
+// then the up's r; else kt = r): D[t][o] = fp16(scale * B_o . t_t) for the n_out outputs (lora_delta_rows).
+// Grid (token blocks of 16, output blocks of 256); 128 threads, two outputs per thread.
+constexpr int kDeltaOut = 256;
+__global__ void __launch_bounds__(128) lora_delta_kernel(const float* __restrict__ tv, int T, int r, bool pairs,
+                                                         int n_out, const uint16_t* __restrict__ B_even,
+                                                         const uint16_t* __restrict__ B_odd, float scale,
+                                                         uint16_t* __restrict__ D) {
+  __shared__ __align__(16) float tS[64][kStTok];
+  const int t0 = blockIdx.x * kStTok, kt = pairs ? 2 * r : r;
+  for (int i = threadIdx.x; i < kStTok * kt; i += blockDim.x) {
+    const int tok = i / kt, j = i - tok * kt;
+    tS[j][tok] = t0 + tok < T ? tv[static_cast<size_t>(t0 + tok) * kt + j] : 0.f;
+  }
+  __syncthreads();
+  const int o_begin = blockIdx.y * kDeltaOut, o_end = o_begin + kDeltaOut < n_out ? o_begin + kDeltaOut : n_out;
+  lora_delta_rows(tS, pairs, r, t0, T, n_out, o_begin, o_end, B_even, B_odd, scale, D);
+}
+
+// Shared expert's down-projection LoRA-A products for many tokens: tv[t] = A_down h_t (r values), h_t the
+// token's SwiGLU output (fp16, pair order within 8-element blocks; A_down [r][I] in natural order), from which
+// lora_delta_kernel forms the delta.  A CTA takes 16 tokens: their h rows and the r rows of A_down go to shared
+// memory first (16-byte asynchronous copies, all in flight; rows padded by 16 bytes so that the eight lanes of
+// a 16-byte load phase, eight tokens, hit distinct banks); a thread then forms one or two of the 16 x r products.
 inline int shared_down_lora_smem(int I, int r) { return (kStTok + r) * (2 * I + 16); }
-__global__ void __launch_bounds__(256, 2) shared_down_lora_kernel(const uint16_t* __restrict__ h, int T, int I, int H,
-                                                               int r, const uint16_t* __restrict__ A_d,
-                                                               const uint16_t* __restrict__ B_d, float scale,
-                                                               uint16_t* __restrict__ D) {
+__global__ void __launch_bounds__(256) shared_down_lora_kernel(const uint16_t* __restrict__ h, int T, int I, int r,
+                                                               const uint16_t* __restrict__ A_d,
+                                                               float* __restrict__ tv) {
   extern __shared__ __align__(16) uint8_t sd_smem[];
-  __shared__ __align__(16) float tS[32][kStTok];
   const int t0 = blockIdx.x * kStTok, ld = 2 * I + 16, n16 = I / 8;  // staged row stride in bytes
   for (int i = threadIdx.x; i < (kStTok + r) * n16; i += blockDim.x) {
     const int row = i / n16, piece = i - row * n16;
@@ -464,10 +475,8 @@ __global__ void __launch_bounds__(256, 2) shared_down_lora_kernel(const uint16_t
       acc = dot2_mix(prmt(w.y, w.w, 0x5410u), hv.z, acc);
       acc = dot2_mix(prmt(w.y, w.w, 0x7632u), hv.w, acc);
     }
-    tS[j][tok] = acc;
+    if (t0 + tok < T) tv[static_cast<size_t>(t0 + tok) * r + j] = acc;
   }
-  __syncthreads();
-  lora_delta_rows(tS, false, r, t0, T, H, B_d, nullptr, scale, D);
 }
 
 // LoRA-A products on the SwiGLU output rows: t[row][i] = A_row[i] . h[row] with
