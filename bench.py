@@ -185,9 +185,9 @@ def prefill_leg(dev, M, passes: int = 5, cfg=None):
                                         "scope": "every kernel of one layer's moe_expert_forward (the two grouped "
                                                  "GEMMs dominate), timed alone",
                                         "traffic": None,
-                                        "traffic_note": "DRAM bytes were captured for the gate/up grouped GEMM at "
-                                                        "512 tokens only; its weight bytes do not grow with tokens, "
-                                                        "so no full-size figure is scaled from it"}},
+                                        "traffic_note": "DRAM bytes are captured per launch of the gate/up grouped "
+                                                        "GEMM (ncu, 3,328 tokens); this roofline spans every kernel "
+                                                        "of the layer, so no whole-layer traffic is given"}},
     }
 
 
@@ -1002,7 +1002,8 @@ def main():
         for key, fn in (("decode_8b", lambda: decode_leg(dev, M, DECODE_8B_CFG_ID, steps=500)),
                         ("batched_decode", lambda: batched_decode_leg(dev, M)),
                         ("prefill_8b", lambda: prefill_leg(dev, M, passes=3,
-                                                           cfg=dataclasses.replace(CONFIGS[DECODE_8B_CFG_ID], T=3328))),
+                                                           cfg=dataclasses.replace(CONFIGS[DECODE_8B_CFG_ID], T=3328,
+                                                                               name="8B-shaped prefill"))),
                         ("tiered_pool", lambda: tiered_leg(dev, M))):
             try:
                 leg = fn()
