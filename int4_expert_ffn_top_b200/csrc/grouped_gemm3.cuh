@@ -119,10 +119,8 @@ struct Args {
   uint16_t* out;
   int out_ld;
   const float* row_scale;
-  const uint16_t* lora_B1;
-  const float* lora_t1;
-  const uint16_t* lora_B2;
-  const float* lora_t2;
+  const float* lora_t1;  // routed adapters' t vectors [row][r] (SwiGLU: the gate's; down: the down's)
+  const float* lora_t2;  // SwiGLU: the up projection's
   const uint16_t* lora_Bex;
   const uint16_t* lora_Bgu_ex;  // SwiGLU, routed: per-expert B [E][2I][r] in the block's interleaved row order
   // the shared expert's unmerged LoRA deltas, computed per token beforehand: fp16 [token][lora_D_ld] (output
@@ -475,19 +473,14 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
       // per-tile inputs of the epilogue, staged once while the accumulator is still being written
       const bool swiglu = a.epi == EPI_SWIGLU;
       const bool up = swiglu && (L & 1) != 0;
-      const uint16_t* Bsrc;
-      const uint16_t* Bgu = tile.e < a.E && a.lora_Bgu_ex ? a.lora_Bgu_ex + static_cast<size_t>(tile.e) * 2 * a.out_ld * r
-                                                          : nullptr;  // SwiGLU: out_ld = I
-      if (swiglu)  // LoRA on the shared expert's gate/up, or on a routed expert's
-        Bsrc = tile.e == a.E ? (up ? a.lora_B2 : a.lora_B1) : Bgu;
-      else
-        Bsrc = tile.e < a.E ? (a.lora_Bex ? a.lora_Bex + static_cast<size_t>(tile.e) * a.out_ld * r : nullptr)
-                            : a.lora_B1;
-      const bool dtile = tile.e == a.E && a.lora_D;  // the shared expert's precomputed deltas (they take the
-                                                     // LoRA staging area: no B.t term on such a tile)
-      if (dtile) Bsrc = nullptr;
-      const bool any_lora = !dtile && (swiglu ? (tile.e == a.E ? (a.lora_B1 || a.lora_B2) : Bgu != nullptr)
-                                              : (tile.e < a.E ? a.lora_Bex != nullptr : a.lora_B1 != nullptr));
+      // a routed expert's adapter B rows (SwiGLU: [E][2I][r] in the interleaved row order, out_ld = I; down:
+      // [E][H][r]); the shared expert's rows take precomputed deltas instead
+      const uint16_t* Bsrc =
+          tile.e >= a.E ? nullptr
+          : swiglu      ? (a.lora_Bgu_ex ? a.lora_Bgu_ex + static_cast<size_t>(tile.e) * 2 * a.out_ld * r : nullptr)
+                        : (a.lora_Bex ? a.lora_Bex + static_cast<size_t>(tile.e) * a.out_ld * r : nullptr);
+      const bool dtile = tile.e == a.E && a.lora_D;  // the shared expert's precomputed deltas
+      const bool any_lora = Bsrc != nullptr;
       if (dtile) {  // [token][128 rows] fp16 into the LoRA staging area, every load in flight at once
         const uint16_t* src = a.lora_D + static_cast<size_t>(tile.row0 - a.lora_D_row0) * a.lora_D_ld + tile.mt * BM;
 #pragma unroll 1
@@ -533,14 +526,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm3_kernel(const __grid
       if (!swiglu && tile.e < a.E && a.row_scale)
         for (int i = et; i < tile.n; i += kEpi) rsc[i] = a.row_scale[tile.row0 + i];
       if (any_lora) {  // the rows' LoRA B values, read once per tile (consecutive threads: consecutive i of a row)
-        const uint16_t* Bdn = tile.e < a.E ? (a.lora_Bex ? a.lora_Bex + static_cast<size_t>(tile.e) * a.out_ld * r : nullptr)
-                                           : a.lora_B1;
         for (int i = et; i < BM * r; i += kEpi) {
           const int row = i / r, j = i - row * r, oo = tile.mt * BM + row;
-          const bool per_proj = swiglu && tile.e == a.E;
-          const uint16_t* src = swiglu ? (per_proj ? ((row & 1) ? a.lora_B2 : a.lora_B1) : Bgu) : Bdn;
-          bls[j * BM + row] =
-              src ? a.lora_scale * half_bits_to_float(src[static_cast<size_t>(per_proj ? oo >> 1 : oo) * r + j]) : 0.f;
+          bls[j * BM + row] = a.lora_scale * half_bits_to_float(Bsrc[static_cast<size_t>(oo) * r + j]);
         }
       }
       // the epilogue warps leave together (they meet at named barriers below)

@@ -575,7 +575,7 @@ moe_status expert_forward_gemm(const moe_layer* L, const uint16_t* u, int T, int
   }
   if (ex)  // the routed down adapters' A products on the SwiGLU output rows
     pf::lora_a_rows_kernel<<<(TK * r + kWarps - 1) / kWarps, kThreads, 0, st>>>(
-        ws.Hh, I, TK, TK, 0, r, nullptr, L->ex_lora_A, ws.idx, ws.perm, ws.t1);
+        ws.Hh, I, TK, r, L->ex_lora_A, ws.idx, ws.perm, ws.t1);
   {  // down (+ LoRA), routed rows scaled by their gating weight
     gg3::Args a = base_args();
     a.tiles = ws.tiles_dn;

@@ -479,20 +479,17 @@ __global__ void __launch_bounds__(256) shared_down_lora_kernel(const uint16_t* _
   }
 }
 
-// LoRA-A products on the SwiGLU output rows: t[row][i] = A_row[i] . h[row] with
-// A = A_down_shared for rows >= TK, else the routed expert's A (if any).
-// One warp per (row, i); h rows are fp16 in pair order, A rows in natural order.
-__global__ void __launch_bounds__(kThreads) lora_a_rows_kernel(const uint16_t* __restrict__ h, int I, int TK, int nrows,
-                                                               int row_begin, int r, const uint16_t* __restrict__ A_sd,
+// The routed down adapters' LoRA-A products on the SwiGLU output rows of the routed slots (rows < TK):
+// t[row][i] = A_e[i] . h[row], e the row's expert (A_ex [E][r][I]).  One warp per (row, i); h rows are fp16 in
+// pair order, A rows in natural order.
+__global__ void __launch_bounds__(kThreads) lora_a_rows_kernel(const uint16_t* __restrict__ h, int I, int TK, int r,
                                                                const uint16_t* __restrict__ A_ex,
                                                                const int32_t* __restrict__ idx,
                                                                const int32_t* __restrict__ perm, float* __restrict__ t) {
   const int gw = blockIdx.x * kWarps + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (gw >= nrows * r) return;
-  const int row = row_begin + gw / r, i = gw % r;
-  const uint16_t* A;
-  if (row >= TK) A = A_sd + static_cast<size_t>(i) * I;
-  else A = A_ex + (static_cast<size_t>(idx[perm[row]]) * r + i) * I;
+  if (gw >= TK * r) return;
+  const int row = gw / r, i = gw % r;
+  const uint16_t* A = A_ex + (static_cast<size_t>(idx[perm[row]]) * r + i) * I;
   const uint16_t* hr = h + static_cast<size_t>(row) * I;
   float acc = 0.f;
   for (int c = lane; c < I / 8; c += 32) {
