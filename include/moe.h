@@ -193,7 +193,9 @@ moe_status moe_route_topk(const moe_layer* L, const uint16_t* u, int32_t T, int3
  *   CUDA cores (fp32 accumulation of exact fp16 x int4-code products); T*K >=
  *   48 slots (with H and 2I multiples of 128) run grouped GEMMs on the tcgen05
  *   tensor cores over per-expert token buckets, where the dequantised weights
- *   and the SwiGLU output are rounded to fp16 and products accumulate in fp32.
+ *   and the SwiGLU output are rounded to fp16 and products accumulate in fp32;
+ *   there the shared expert's LoRA deltas (scale * B A x per token and output)
+ *   are formed in fp32 and rounded to fp16 before they join the accumulator.
  * Bounded waits: every device-side wait of the tensor-core path gives up after
  *   2 s, so a call always completes; a wait that ran out stores MOE_ERR_TIMEOUT
  *   in err_word (see Errors) and leaves the output undefined.
