@@ -53,7 +53,8 @@
  *     of I inputs.  Every row, and every run of rows one unit of work needs,
  *     is one contiguous span (one bulk copy / one coalesced warp read).
  * Supported shapes: H a power of two in [256, 4096], I a power of two in
- *   [128, 2048], I_s == I, 1 <= K <= 8, K <= E <= 256, LoRA rank r <= 32,
+ *   [128, 2048], I_s == I, 1 <= K <= 8, K <= E <= 256, LoRA rank r one of
+ *   0 (no adapters), 8, 16, 24, 32 (the adapters move in 16-byte units),
  *   Prerouter E % 8 == 0 and P % 8 == 0, 0 <= T <= MOE_MAX_TOKENS tokens per
  *   call.
  */

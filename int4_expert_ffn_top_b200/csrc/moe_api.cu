@@ -39,7 +39,9 @@ moe_status check_layer(const moe_layer* L, int T, int K) {
   if (!L) return MOE_ERR_INVALID_ARG;
   if (T < 0 || T > MOE_MAX_TOKENS || K < 1 || K > 8) return MOE_ERR_UNSUPPORTED;
   if (!h_ok(L->H) || !i_ok(L->I) || L->I_s != L->I) return MOE_ERR_UNSUPPORTED;
-  if (L->E < K || L->E > 256 || L->r < 0 || L->r > 32) return MOE_ERR_UNSUPPORTED;
+  // LoRA rank a multiple of 8 (0: none): the LoRA tensors move in 16-byte units (bulk copies of 4r- and
+  // 2r-byte row runs, 16-byte loads of B rows), which other ranks would misalign
+  if (L->E < K || L->E > 256 || L->r < 0 || L->r > 32 || L->r % 8 != 0) return MOE_ERR_UNSUPPORTED;
   if (!qrows_ok(L->router, L->E, L->H, 8)) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }

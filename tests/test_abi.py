@@ -93,6 +93,9 @@ def test_host_side_rejections(lib):
     L.H = 2000
     assert lib.moe_route_topk(ctypes.byref(L), None, 1, 4, None, None, None, None, None) == _lib.MOE_ERR_UNSUPPORTED
     L.H = 2048
+    L.r = 12  # LoRA ranks are multiples of 8
+    assert lib.moe_route_topk(ctypes.byref(L), None, 1, 4, None, None, None, None, None) == _lib.MOE_ERR_UNSUPPORTED
+    L.r = 16
     # router matrix missing
     assert lib.moe_route_topk(ctypes.byref(L), None, 1, 4, None, None, None, None, None) == _lib.MOE_ERR_INVALID_ARG
     assert lib.moe_expert_forward(ctypes.byref(L), None, 1, 4, None, None, None, 0, None, None, 0,
