@@ -1,6 +1,7 @@
 // Supporting kernels of the many-token (grouped GEMM) expert path: parallel
 // deterministic token buckets, the permuted fp16 token matrix, the device-side
-// tile list, LoRA-A products for many tokens, and the gather-combine.
+// tile list, the shared expert's 8-bit gate and LoRA-A products and its per-token
+// LoRA deltas, the routed adapters' LoRA-A products, and the gather-combine.
 #pragma once
 
 #include "grouped_gemm3.cuh"
@@ -177,7 +178,7 @@ __global__ void __launch_bounds__(128) tile_list_kernel(const int32_t* __restric
   }
 }
 
-// Shared expert's gate and gate/up LoRA deltas for many tokens, in one pass over u:
+// Shared expert's gate and gate/up LoRA-A products for many tokens, in one pass over u:
 //   g[t] = sigmoid(w . u_t), w the 8-bit gate row (affine groups of 64): per group s * sum (q - 128) u + (b + 128 s) * sum u;
 //   the LoRA-A products t1 = A_gate u_t and t2 = A_up u_t (r values each; a projection without adapter gets
 //   zeros) into tv[t] = (t1, t2), from which lora_delta_kernel forms the unmerged deltas the gate/up GEMM adds.
@@ -200,9 +201,9 @@ MOE_DEV void mma_tf32(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint
                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// D[t0 + tok][o] = fp16(scale * B_o . t[tok]) for the tokens of a 16-token block and outputs o_begin <= o < o_end
-// (D rows hold n_out outputs),
-// t[tok] = tS[j][tok] (j < r).  pairs = false: B_o is row o of B_even ([n_out][r]).  pairs = true (the
+// D[t0 + tok][o] = fp16(scale * B_o . t[tok]) for the tokens of a 16-token block and the outputs
+// o_begin <= o < o_end (a row of D holds n_out outputs), t[tok] = tS[j][tok] (j < r).
+// pairs = false: B_o is row o of B_even ([n_out][r]).  pairs = true (the
 // interleaved gate/up rows): B_o is row o / 2 of B_even for even o and of B_odd for odd o (each [n_out / 2][r]),
 // and the odd rows read t from tS[r + j].  A null B gives zeros.  Two outputs per thread and pass, all 16
 // tokens; a B row is read 8 ranks per 16-byte load when r is a multiple of 8.
