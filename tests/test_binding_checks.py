@@ -187,3 +187,27 @@ def test_stack_structs_refuse_an_empty_stack_or_mismatched_heads():
         M.StackStructs([FakeLayer(), FakeLayer()], [FakeHead()])
     st = M.StackStructs([FakeLayer()], [FakeHead()])
     assert st.heads_ptr() is not None
+
+
+def test_tier_calls_pass_arguments_in_abi_order(rec):
+    tp = object.__new__(M.TieredPool)  # the constructor needs pinned host memory; the calls do not
+    tp.handle = ctypes.c_void_p(1234)
+    try:
+        idx, slot, err = i32(T, K), i32(T, K), i32(1)
+        tp.acquire([3, 1], idx, slot, err_word=err, stream=0)
+        name, a = rec.calls[-1]
+        assert name == "moe_tier_acquire"
+        assert a[0] is tp.handle and a[2] == 2 and a[3:] == (idx.data_ptr(), T * K, slot.data_ptr(), err.data_ptr(), 0)
+        n = len(rec.calls)
+        with pytest.raises(ValueError):
+            tp.acquire([3], idx, i32(T * K - 1), stream=0)  # idx_slot smaller than idx
+        with pytest.raises(ValueError):
+            tp.acquire([3], cu(torch.zeros((T, K), dtype=torch.int64)), slot, stream=0)  # wrong element type
+        assert len(rec.calls) == n  # neither reached the library
+        tp.prefetch([5, 6, 7], stream=0)
+        name, a = rec.calls[-1]
+        assert name == "moe_tier_prefetch" and a[0] is tp.handle and a[2] == 3 and a[3] == 0
+        tp.release(stream=0)
+        assert rec.calls[-1] == ("moe_tier_release", (tp.handle, 0))
+    finally:
+        tp.handle = None  # the fake handle must never reach the real library
